@@ -1,0 +1,323 @@
+"""Pins of the CPU oracle against facts the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: numbers the
+Nemotron-3-Ultra architecture report prints (section 2.3.4 parameter shapes,
+section 3.1.3 FLOP total, section 8.1 E2M1 value set), closed forms, brute force
+on tiny inputs, libm and exact rational arithmetic.
+"""
+import fractions
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+ULTRA = dict(D=8192, L=2048, E=512, F=5120, Fs=10240)
+
+
+# --- shapes and work (report section 2.3.4, 2.3.8, 3.1.3) -------------------
+
+def test_param_counts_match_report():
+    c = O.param_count(**ULTRA)
+    assert c["gate"] == 4_194_304            # gate.weight 512 x 8192
+    assert c["bias"] == 512                  # e_score_correction_bias
+    assert c["latent"] == 2 * 16_777_216     # fc1 + fc2 latent projections
+    assert c["experts"] == 10_737_418_240    # 512 experts x 20,971,520
+    assert c["shared"] == 2 * 83_886_080     # shared up + down
+    assert c["total"] == 10_942_939_648      # "approx 10.94B"
+    assert round(c["total"] / 1e9, 2) == 10.94
+
+
+def test_tiny_param_count():
+    assert O.param_count(D=256, L=64, E=16, F=128, Fs=256)["total"] == 430_096
+
+
+def test_activated_params_and_flops_match_report():
+    # activated parameters per MoE layer ~ 667.5M (section 2.3.8, which sums
+    # rounded terms: 4.19M + 33.55M + 22 x 21M + 167.77M)
+    act = 4_194_304 + 2 * 16_777_216 + 22 * 20_971_520 + 167_772_160
+    assert abs(act / 667.5e6 - 1) < 1e-3
+    f = O.flops_per_token(D=8192, L=2048, E=512, k=22, F=5120, Fs=10240)
+    # every activated weight is used once per token in a multiply-add
+    assert f["total"] == 2 * act
+    assert round(f["total"] / 1e9, 2) == 1.33   # section 3.1.3: ~1.33e9 * T
+
+
+# --- router logits: fixed-order fp64 dot products ----------------------------
+
+def _dot_sequential(a, b):
+    """The stated order, one scalar at a time, from dot_spec_order."""
+    order = O.dot_spec_order(len(a))
+    part = [0.0] * 32
+    for p in range(32):
+        for k in order[p]:
+            part[p] = part[p] + float(a[k]) * float(b[k])
+    for off in (16, 8, 4, 2, 1):
+        for j in range(off):
+            part[j] = part[j] + part[j + off]
+    return part[0]
+
+
+@pytest.mark.parametrize("K", [8, 256, 300, 1000])
+def test_dot_spec_follows_stated_order(K):
+    rng = np.random.RandomState(K)
+    a = (rng.standard_normal(K) * np.exp(rng.uniform(-8, 8, K))).astype(np.float32)
+    b = rng.standard_normal(K).astype(np.float32)
+    assert O.dot_spec(a, b) == _dot_sequential(a, b)
+
+
+@pytest.mark.parametrize("K", [256, 8192])
+def test_dot_spec_within_summation_bound(K):
+    rng = np.random.RandomState(1)
+    a = rng.standard_normal(K).astype(np.float32)
+    b = rng.standard_normal(K).astype(np.float32)
+    exact = sum(fractions.Fraction(float(x)) * fractions.Fraction(float(y))
+                for x, y in zip(a, b))
+    got = O.dot_spec(a, b)
+    u = 2.0 ** -53
+    bound = (K * u / (1 - K * u)) * float(np.sum(np.abs(a.astype(np.float64) * b)))
+    assert abs(got - float(exact)) <= bound
+
+
+def test_dot_spec_exact_on_integers():
+    rng = np.random.RandomState(2)
+    a = rng.randint(-100, 100, 4096).astype(np.float64)
+    b = rng.randint(-100, 100, 4096).astype(np.float64)
+    assert O.dot_spec(a, b) == float(np.dot(a.astype(np.int64), b.astype(np.int64)))
+
+
+def test_router_logits_broadcast_shape():
+    x = np.ones((3, 256), np.float32)
+    w = np.arange(5 * 256, dtype=np.float32).reshape(5, 256) / 256
+    l = O.router_logits(x, w)
+    assert l.dtype == np.float32 and l.shape == (3, 5)
+    assert l[0, 1] == np.float32(sum(range(256, 512)) / 256)
+
+
+# --- sigmoid gating (section 5.3) --------------------------------------------
+
+# ln 2 to 40 digits, as a rational
+_LN2_Q = fractions.Fraction("0.6931471805599453094172321214581765680755")
+
+
+def _ulp_diff(a, b):
+    ia = np.asarray(a, np.float64).view(np.int64)
+    ib = np.asarray(b, np.float64).view(np.int64)
+    return np.abs(ia - ib)
+
+
+def test_exp_spec_against_libm():
+    a = np.concatenate([np.linspace(-80, 80, 200001),
+                        np.random.RandomState(3).uniform(-80, 80, 100000)])
+    ref = np.array([math.exp(v) for v in a])
+    assert _ulp_diff(O.exp_spec(a), ref).max() <= 2
+
+
+def test_exp_spec_special_values():
+    assert O.exp_spec(np.array([0.0]))[0] == 1.0
+    for n in range(-100, 101, 7):        # 2**n at n*ln 2 (argument rounded to fp64)
+        a = n * math.log(2)
+        v = O.exp_spec(np.array([a]))[0]
+        rel_arg = abs(float(fractions.Fraction(a) - n * _LN2_Q))   # |a - n ln 2|
+        assert abs(v / 2.0 ** n - 1) <= rel_arg + 4e-16
+    x = np.linspace(-80, 80, 100001)
+    assert np.all(np.diff(O.exp_spec(x)) > 0)            # strictly increasing
+
+
+def test_sigmoid_spec_against_libm_fp32():
+    l = np.concatenate([np.linspace(-90, 90, 100001),
+                        np.random.RandomState(4).standard_normal(100000) * 3]
+                       ).astype(np.float32)
+    ref = np.array([1.0 / (1.0 + math.exp(-min(max(float(v), -80), 80)))
+                    for v in l]).astype(np.float32)
+    got = O.sigmoid_spec(l)
+    d = np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32))
+    assert d.max() <= 1 and (d == 0).mean() > 0.999
+    assert O.sigmoid_spec(np.array([0.0], np.float32))[0] == np.float32(0.5)
+    assert np.all((got > 0) & (got <= 1))
+
+
+# --- selection (sections 5.4-5.6) ---------------------------------------------
+
+def _brute_topk(c, k):
+    """The subset of size k whose members all rank above every non-member under
+    the order (score desc, index asc), found by enumerating every subset."""
+    E = len(c)
+    key = lambda e: (-float(c[e]), e)
+    found = []
+    for sub in itertools.combinations(range(E), k):
+        rest = [e for e in range(E) if e not in sub]
+        if all(key(a) < key(b) for a in sub for b in rest):
+            found.append(sub)
+    assert len(found) == 1
+    return sorted(found[0], key=key)
+
+
+def test_select_topk_brute_force_with_ties():
+    rng = np.random.RandomState(5)
+    for _ in range(300):
+        E = rng.randint(2, 9)
+        k = rng.randint(1, min(3, E) + 1)
+        c = (rng.randint(0, 4, size=(1, E)) / 4.0).astype(np.float32)  # many ties
+        got = O.select_topk(c, k)[0].tolist()
+        assert got == _brute_topk(c[0], k)
+
+
+def test_zero_bias_gives_plain_topk_of_scores():
+    rng = np.random.RandomState(6)
+    l = rng.standard_normal((50, 64)).astype(np.float32)
+    s, _, idx, _ = O.route(l, np.zeros(64, np.float32), 6, 5.0)
+    for t in range(50):
+        ref = sorted(range(64), key=lambda e: (-float(s[t, e]), e))[:6]
+        assert idx[t].tolist() == ref
+
+
+def test_bias_changes_choice_but_not_weights():
+    # hand example: s = sigmoid(l) with l = 0, ln 3, -ln 3, 0  ->  .5 .75 .25 .5
+    l = np.array([[0.0, math.log(3), -math.log(3), 0.0]], np.float32)
+    bias = np.array([0.0, -1.0, 0.0, 0.3], np.float32)
+    s, choice, idx, w = O.route(l, bias, 2, 5.0)
+    assert np.allclose(s[0], [0.5, 0.75, 0.25, 0.5], atol=1e-7)
+    assert idx[0].tolist() == [3, 0]          # choices .8, .5, .25, -.25
+    # weights use the raw scores .5 and .5: normalised to 1/2 each, times 5
+    assert w[0].tolist() == [2.5, 2.5]
+
+
+def test_weights_sum_to_scaling_factor():
+    rng = np.random.RandomState(7)
+    l = (rng.standard_normal((200, 512)) * 2).astype(np.float32)
+    b = (rng.standard_normal(512) * 0.1).astype(np.float32)
+    _, _, idx, w = O.route(l, b, 22, 5.0)
+    assert np.all(np.abs(w.astype(np.float64).sum(1) / 5.0 - 1) < 2 ** -20)
+    assert np.all((w > 0) & (w <= 5.0))
+    assert np.all([len(set(r)) == 22 for r in idx.tolist()])
+
+
+def test_top1_weight_is_exactly_the_scaling_factor():
+    l = np.random.RandomState(8).standard_normal((30, 16)).astype(np.float32)
+    _, _, _, w = O.route(l, np.zeros(16, np.float32), 1, 5.0)
+    assert np.all(w == np.float32(5.0))
+
+
+def test_group_routing_hand_example():
+    # 2 groups of 3; group scores (top-2 sums): g0 = .9+.1 = 1.0, g1 = .8+.7 = 1.5
+    c = np.array([[0.9, 0.1, 0.0, 0.8, 0.7, 0.05]], np.float32)
+    m = O.group_mask(c, 2, 1)
+    assert m[0].tolist() == [False] * 3 + [True] * 3
+    assert O.select_topk(c, 2, m)[0].tolist() == [3, 4]
+    assert O.group_mask(c, 1, 1).all()
+
+
+def test_max_violation_when_one_set_takes_everything():
+    idx = np.tile(np.arange(22, dtype=np.int32), (64, 1))
+    counts, _, _, _ = O.dispatch(idx, 512)
+    assert abs(O.max_violation(counts) - 512 / 22) < 1e-12
+    assert round(512 / 22, 2) == 23.27   # report section 10.3 / explainer figure
+
+
+def test_dispatch_against_comparison_sort():
+    rng = np.random.RandomState(9)
+    T, E, k = 97, 40, 5
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, pos = O.dispatch(idx, E)
+    flat = idx.reshape(-1)
+    order = np.argsort(flat.astype(np.int64) * (T * k) + np.arange(T * k), kind="stable")
+    assert perm.tolist() == order.tolist()
+    assert counts.tolist() == np.bincount(flat, minlength=E).tolist()
+    assert offsets[-1] == T * k and np.all(np.diff(offsets) == counts)
+    assert np.all(perm[pos.reshape(-1)] == np.arange(T * k))
+
+
+# --- printed values (tests/golden/report_values.json) ------------------------
+
+import json
+import os
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                     "report_values.json")))
+
+
+def test_golden_param_counts():
+    g = GOLDEN["param_counts"]
+    c = O.param_count(**ULTRA)
+    assert c["gate"] == g["gate_weight"] and c["bias"] == g["e_score_correction_bias"]
+    assert c["latent"] == g["fc1_latent_proj"] + g["fc2_latent_proj"]
+    assert c["experts"] == g["all_experts"] == 512 * g["one_expert"]
+    assert c["shared"] == g["shared_up"] + g["shared_down"]
+    assert round(c["total"] / 1e9, 2) == g["layer_total_billions_2dp"]
+    assert round(O.flops_per_token(D=8192, L=2048, E=512, k=22, F=5120, Fs=10240)
+                 ["total"] / 1e9, 2) == GOLDEN["moe_flops_per_token_billions_2dp"]
+
+
+# --- NVFP4 codec (section 8.1; NVFP4 format details) -------------------------
+
+def test_e2m1_value_set_matches_report():
+    vals = sorted(set(abs(v) for v in O.E2M1_TABLE.tolist()))
+    assert vals == GOLDEN["e2m1_values"]
+    assert sorted(set(O.E2M1_TABLE.tolist())) == sorted(
+        set(GOLDEN["e2m1_values"]) | {-v for v in GOLDEN["e2m1_values"]})
+
+
+def test_e2m1_exhaustive_roundtrip_and_ties():
+    for c in range(16):
+        v = O.e2m1_value(c)
+        assert O.e2m1_encode(v) == (0 if c == 8 else c)     # -0 encodes as +0
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0,
+            5.0: 4.0, 7.0: 6.0, 100.0: 6.0}
+    for x, v in ties.items():
+        assert O.e2m1_value(O.e2m1_encode(x)) == v
+        assert O.e2m1_value(O.e2m1_encode(-x)) == -v
+
+
+def test_e4m3_exhaustive():
+    finite = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    assert len(finite) == 254
+    assert max(O.e4m3_value(c) for c in finite) == 448.0
+    assert O.e4m3_value(1) == 2.0 ** -9                      # smallest subnormal
+    assert O.e4m3_value(0x08) == 2.0 ** -6                   # smallest normal
+    for c in range(0x7F):
+        assert O.e4m3_encode(O.e4m3_value(c)) == c
+    assert O.e4m3_encode(1000.0) == 0x7E                      # satfinite
+    # ties between neighbours go to the even code
+    for c in range(0, 0x7E):
+        mid = (O.e4m3_value(c) + O.e4m3_value(c + 1)) / 2
+        assert O.e4m3_encode(mid) == (c if c % 2 == 0 else c + 1)
+
+
+def test_nvfp4_roundtrip_of_representable_values_is_exact():
+    rng = np.random.RandomState(10)
+    rows, K = 24, 128
+    sg = np.float32(1.25 * 2.0 ** -7)      # short mantissa: q*s_b*s_g exact in fp32
+    sb = rng.randint(0x20, 0x60, size=(rows, K // 16)).astype(np.uint8)
+    q = rng.randint(0, 16, size=(rows, K)).astype(np.uint8)
+    q[:, ::16] = 7                      # every block holds +6: its amax is 6*scale
+    w = O.nvfp4_dequantize(q, sb, sg).astype(np.float32)
+    assert np.all(w.astype(np.float64) == O.nvfp4_dequantize(q, sb, sg))
+    q2, sb2 = O.nvfp4_quantize(w, sg)
+    assert np.array_equal(O.nvfp4_dequantize(q2, sb2, sg),
+                          O.nvfp4_dequantize(q, sb, sg))
+
+
+def test_nvfp4_error_bound_and_scales():
+    rng = np.random.RandomState(11)
+    w = (rng.standard_normal((64, 256)) * 0.02).astype(np.float32)
+    sg = O.nvfp4_global_scale(w)
+    assert sg == np.float32(np.abs(w).max() / np.float32(2688.0))
+    q, sb = O.nvfp4_quantize(w, sg)
+    assert q.max() < 16 and np.all((sb & 0x7F) != 0x7F)
+    deq = O.nvfp4_dequantize(q, sb, sg)
+    scale = O.E4M3_TABLE[sb].astype(np.float32) * sg
+    err = np.abs(deq - w).reshape(64, 16, 16)
+    # worst grid gap is 2 (between 4 and 6): half of it times the block scale,
+    # or the saturation overshoot when the rounded block scale came out small
+    over = np.maximum(np.abs(w).reshape(64, 16, 16) - 6 * scale[..., None], 0)
+    assert np.all(err <= scale[..., None] * 1.0 + over + 1e-12)
+    rel = np.linalg.norm(deq - w) / np.linalg.norm(w)
+    assert rel < 0.12
+
+
+def test_pack_e2m1_low_nibble_first():
+    c = np.array([[1, 2, 15, 0]], np.uint8)
+    assert O.pack_e2m1(c).tolist() == [[0x21, 0x0F]]
