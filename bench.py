@@ -1,0 +1,333 @@
+"""Benchmark of the LatentMoE layer on B200: tokens/s of one layer forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl ours|reference]
+
+A step is one moe_forward over one batch of T synthetic tokens (router, routing
+bookkeeping, latent projection, routed experts, combine, fc2 and the shared
+expert).  Default workload: the Ultra-shape decode layer, bf16, T=64.  With N>1
+(torchrun) every rank runs its own replica on its own tokens (weak scaling, no
+collective on the data path); value = all ranks' tokens / max-over-ranks time.
+`--impl reference` times the CPU oracle on the host cores instead.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LatentMoE layer tokens/s at Ultra shape (T=64 decode, T=8192 prefill); % roofline"
+UNIT = "tokens/s"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="ultra_decode_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampler over the timed region (SM clock, throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    return rank, world, local
+
+
+def _expert_bytes(cfg, n_touched):
+    """Bytes of one expert matrix set actually streamed: dense bf16/fp32."""
+    es = 4 if cfg.dtype == "fp32" else 2
+    return n_touched * cfg.F * cfg.L * es
+
+
+def _oracle_sample(cfg, W, x, n_tok):
+    """Time the oracle, as it stands, on the first n_tok token rows."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    rows = x[:n_tok]
+    f = lambda t: t.detach().float().cpu().numpy()
+    xs, g, b = f(rows), f(W["w_gate"]), f(W["gate_bias"])
+    dense = [f(W[n]) for n in ("w_fc1", "w_fc2", "w_shared_up", "w_shared_down")]
+    l = O.router_logits(xs, g)
+    _, _, idx, _ = O.route(l, b, cfg.k, cfg.rsf)
+    need = sorted(set(idx.reshape(-1).tolist()))
+    up = {e: W["w_up"][e].double().cpu().numpy() for e in need}
+    dn = {e: W["w_down"][e].double().cpu().numpy() for e in need}
+    t0 = time.perf_counter()
+    O.forward(xs, g, b, *dense, lambda e: up[e], lambda e: dn[e], k=cfg.k, rsf=cfg.rsf,
+              expert_fmt=cfg.expert_fmt)
+    dt = time.perf_counter() - t0
+    return n_tok / dt, dt
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def _gen_device():
+    import torch
+    return "cuda" if torch.cuda.is_available() else "cpu"
+
+
+def run_reference(a):
+    rank, world, _ = _dist()
+    if rank != 0:
+        return 0
+    import torch
+    from latentmoe_expert_routing_b200 import inputs as I
+    cfg = I.CONFIGS[a.config]
+    dev = _gen_device()
+    W = _weights(cfg, dev)
+    x = I.hidden(cfg, dev)
+    n_tok = cfg.T if cfg.T * cfg.D <= 64 * 256 else 2
+    for _ in range(a.warmup):
+        _oracle_sample(cfg, W, x, n_tok)
+    times = [_oracle_sample(cfg, W, x, n_tok)[1] for _ in range(a.steps)]
+    value = n_tok * a.steps / sum(times)
+    sample = f"first {n_tok} of {cfg.T} tokens per step, fp64 numpy oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": 1e3 * sum(times) / a.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "sample_tokens": n_tok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}))
+    return 0
+
+
+def _weights(cfg, dev):
+    from latentmoe_expert_routing_b200 import inputs as I
+    import torch
+    dt = torch.float32 if cfg.dtype == "fp32" else torch.bfloat16
+    up = torch.empty(cfg.E, cfg.F, cfg.L, dtype=dt, device=dev)
+    down = torch.empty(cfg.E, cfg.L, cfg.F, dtype=dt, device=dev)
+    I.w_up_into(cfg, up)
+    I.w_down_into(cfg, down)
+    return dict(w_gate=I.w_gate(cfg, dev), gate_bias=I.gate_bias(cfg, dev),
+                w_fc1=I.w_fc1(cfg, dev), w_fc2=I.w_fc2(cfg, dev),
+                w_shared_up=I.w_shared_up(cfg, dev),
+                w_shared_down=I.w_shared_down(cfg, dev), w_up=up, w_down=down)
+
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    from latentmoe_expert_routing_b200 import binding as B
+    from latentmoe_expert_routing_b200 import inputs as I
+    from latentmoe_expert_routing_b200 import layer as LY
+    cfg = I.CONFIGS[a.config]
+    W = _weights(cfg, "cuda")
+    lay = LY.layer_for(cfg, W, out_dtype=cfg.dtype)
+    x = I.hidden(cfg, "cuda", T=cfg.T, start_row=0) if rank == 0 else \
+        I.hidden(cfg.replace(seed=rank), "cuda")
+    T = cfg.T
+    tdt = x.dtype
+    out = torch.empty(T, cfg.D, dtype=tdt, device="cuda")
+    idx = torch.empty(T, cfg.k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(T, cfg.k, dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream()
+
+    def step():
+        lay(x, out, idx, wts)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(a.warmup, 3)):
+        step()
+    lay.sync()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        e0.record(st)
+        for _ in range(a.steps):
+            step()
+        e1.record(st)
+        torch.cuda.synchronize()
+    barrier()
+    lay.sync()
+    ms = e0.elapsed_time(e1) / a.steps
+    ms_t = torch.tensor([ms], device="cuda")
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # per-stage durations (CUDA events recorded by the library on this stream)
+    B.moe_profile_enable(lay.handle, 1)
+    stages = []
+    for _ in range(5):
+        step()
+        stages.append(B.moe_profile_read(lay.handle))
+    B.moe_profile_enable(lay.handle, 0)
+    stage_ms = {k: statistics.median(s[k] for s in stages) for k in stages[0]}
+    counts, _, _, _ = lay.routing(T)
+    n_touched = int((counts > 0).sum().item())
+
+    # end to end through the host entry point: pinned H2D of x, D2H of out
+    xh = x.cpu().pin_memory()
+    oh = torch.empty(T, cfg.D, dtype=tdt).pin_memory()
+    for _ in range(2):
+        lay.forward_host(xh, oh)
+    barrier()
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(st)
+    for _ in range(a.steps):
+        lay.forward_host(xh, oh)
+    h1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([h0.elapsed_time(h1) / a.steps], device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        n_tok = min(T, 4 if cfg.D >= 4096 else T)
+        v, dt = _oracle_sample(cfg, W, x, n_tok)
+        cpu = {"value": v, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+               "sample": f"first {n_tok} of {T} tokens, one fp64 numpy oracle forward "
+                         f"({dt:.1f} s)"}
+
+    hbm, tf, tf_sus, src = _peaks()
+    # dominant kernel: the grouped expert GEMMs streaming the touched experts'
+    # weights (up and down, one launch each); algorithmic bytes per launch =
+    # touched experts x one [F, L] matrix + the activations it reads and writes
+    es = 4 if cfg.dtype == "fp32" else 2
+    P = T * cfg.k
+    b_up = _expert_bytes(cfg, n_touched) + P * cfg.L * es + P * cfg.F * es
+    b_dn = _expert_bytes(cfg, n_touched) + P * cfg.F * es + P * cfg.L * 4
+    t_launch = (stage_ms["expert_up"] + stage_ms["expert_down"]) / 2
+    achieved = (b_up + b_dn) / 2 / (t_launch * 1e-3) / 1e9
+    if rank == 0:
+        clk_s = clk.summary()
+        line = {
+            "metric": METRIC, "value": world * T / (ms_max * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": a.steps, "warmup": max(a.warmup, 3),
+            "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "T": T, "d_model": cfg.D, "d_latent": cfg.L,
+                       "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
+                       "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
+                       "parallelism": f"replicas{world}",
+                       "l2": "no flush: each step streams the touched experts' weights "
+                             f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
+            "roofline": {"kernel": "grouped_rows_kernel (expert up, expert down)",
+                         "bound": "hbm", "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak_source": src,
+                         "bytes_per_launch": (b_up + b_dn) / 2},
+            "stages_ms": stage_ms,
+            "experts_touched": n_touched,
+            "expert_weight_gbs": 2 * _expert_bytes(cfg, n_touched) /
+                                 ((stage_ms["expert_up"] + stage_ms["expert_down"]) * 1e-3) / 1e9,
+            "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,
+            "clocks": clk_s,
+            "gpu_launches": 10 * a.steps,
+            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": T * cfg.D * es,
+                    "d2h_bytes_per_step": T * cfg.D * es},
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    del lay
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

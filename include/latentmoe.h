@@ -1,0 +1,165 @@
+/*
+ * latentmoe.h -- C ABI of the B200 LatentMoE feed-forward layer.
+ *
+ * The layer (Nemotron-3-Ultra architecture report, chapter 5 "LatentMoE
+ * router", section 5.6, steps 1-7):
+ *   logits = x . W_gate^T                 (router on the full d_model input)
+ *   s      = sigmoid(logits)              (section 5.3)
+ *   choice = s + e_score_correction_bias  (section 5.4; selection only)
+ *   idx    = top-k(choice)                (section 5.5 with n_group = 1)
+ *   w      = s[idx] / (sum s[idx] + 1e-20) * routed_scaling_factor
+ *   z      = x . W_fc1^T                  (fc1_latent_proj, d_model -> d_latent)
+ *   zc[t]  = sum_j w[t,j] * down_e(relu(up_e(z[t]))^2),  e = idx[t,j]
+ *   out    = zc . W_fc2^T + W_sd . relu(W_su . x)^2    (fc2 + shared expert)
+ * Shapes follow the report's section 2.3.4: every Linear weight is [out, in]
+ * row-major; routed experts are 3-D tensors up[E, F, L] and down[E, L, F].
+ *
+ * Numerics.  The router logit is defined as the fp64 sum of the exact products
+ * x[k]*W[e,k] taken in a fixed order (32 partial sums, partial p takes every
+ * k with (k/8) % 32 == p in increasing k, then p[j] += p[j+off] for off = 16,
+ * 8, 4, 2, 1), rounded once to fp32; the sigmoid is evaluated in fp64 with a
+ * fixed exp (Cody-Waite + degree-13 Taylor) and rounded to fp32.  Routing
+ * indices and weights are therefore reproducible bit for bit.  Ties in the
+ * choice score go to the lower expert index; the k slots of a token are
+ * ordered by (choice descending, expert ascending).  The expert, latent and
+ * shared-expert products accumulate in fp32; bf16 configurations round z,
+ * relu^2 activations and the combined latent to bf16 as GEMM operands.
+ *
+ * Errors.  Every call returns a moe_status; nothing is thrown across the ABI.
+ * Arguments are validated on the host before any launch.  Problems detected
+ * by a kernel set a device error word that moe_sync() reports.
+ *
+ * Streams.  `stream` arguments are cudaStream_t values passed as void*
+ * (NULL = the legacy default stream).  A handle is used on one stream at a
+ * time; calls on it are asynchronous unless stated otherwise.
+ */
+#ifndef LATENTMOE_H
+#define LATENTMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. n_group > 1)     */
+  MOE_ERR_OOM = 3,           /* device allocation failed in moe_init       */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
+  MOE_ERR_TIMEOUT = 5,       /* a bounded device wait gave up              */
+  MOE_ERR_DEVICE_CHECK = 6   /* a kernel saw an out-of-range index         */
+} moe_status;
+
+typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Routed-expert weight format (report section 8.1; NVFP4 = E2M1 elements in
+ * 16-element blocks along K, one E4M3 scale per block, one FP32 global scale
+ * per expert matrix). */
+typedef enum {
+  MOE_EXPERT_DENSE = 0,        /* experts in `dtype`                          */
+  MOE_EXPERT_NVFP4_W4A16 = 1,  /* NVFP4 weights, bf16 activations             */
+  MOE_EXPERT_NVFP4_W4A4 = 2    /* NVFP4 weights and NVFP4 expert activations  */
+} moe_expert_fmt;
+
+typedef struct {
+  int d_model;        /* D: 8192 for the Ultra shape                         */
+  int d_latent;       /* L: moe_latent_size, 2048                            */
+  int n_experts;      /* E: n_routed_experts, 512                            */
+  int top_k;          /* k: num_experts_per_tok, 22                          */
+  int d_ff;           /* F: moe_intermediate_size, 5120                      */
+  int d_ff_shared;    /* Fs: moe_shared_expert_intermediate_size, 10240      */
+  int n_group;        /* must be 1 (all experts compete)                     */
+  int topk_group;     /* must be 1                                           */
+  int max_tokens;     /* workspace is sized for up to this many tokens       */
+  float routed_scaling_factor;   /* 5.0                                      */
+  moe_dtype dtype;               /* activations and dense weights            */
+  moe_expert_fmt expert_fmt;
+  moe_dtype out_dtype;           /* dtype of `out`                           */
+} moe_config;
+
+/* Weights, all DEVICE pointers, row-major [out, in].  With borrow != 0 the
+ * library keeps the pointers and the caller must keep the memory alive and
+ * unchanged until moe_destroy(); with borrow == 0 moe_init copies them.
+ * Dense experts are read from w_up/w_down; NVFP4 formats quantise w_up/w_down
+ * at init into library-owned codes and scales (the caller's dense experts may
+ * be freed after moe_init returns). */
+typedef struct {
+  const void* w_gate;          /* [E, D]  dtype                               */
+  const float* gate_bias;      /* [E]     fp32 e_score_correction_bias        */
+  const void* w_fc1;           /* [L, D]  dtype                               */
+  const void* w_fc2;           /* [D, L]  dtype                               */
+  const void* w_shared_up;     /* [Fs, D] dtype                               */
+  const void* w_shared_down;   /* [D, Fs] dtype                               */
+  const void* w_up;            /* [E, F, L] dtype                             */
+  const void* w_down;          /* [E, L, F] dtype                             */
+  int borrow;
+} moe_weights;
+
+typedef struct moe_handle moe_handle;
+
+/* Validate cfg, allocate the workspace for cfg->max_tokens and take the
+ * weights (see moe_weights).  Synchronises `stream` before returning. */
+moe_status moe_init(moe_handle** handle, const moe_config* cfg,
+                    const moe_weights* weights, void* stream);
+
+/* One layer forward on T token rows (report section 5.6).
+ *   hidden   [T, D] dtype, device, row-major, 16-byte aligned
+ *   out      [T, D] out_dtype, device
+ *   topk_idx [T, k] int32, device, or NULL   (slot order: see Numerics)
+ *   topk_w   [T, k] fp32,  device, or NULL
+ * T = 0 returns MOE_OK with no launch; T > max_tokens is MOE_ERR_INVALID_ARG.
+ * Asynchronous on `stream`; no host synchronisation inside. */
+moe_status moe_forward(moe_handle* handle, const void* hidden, int T, void* out,
+                       int32_t* topk_idx, float* topk_w, void* stream);
+
+/* Same as moe_forward with HOST buffers: copies hidden to the device, runs the
+ * layer, copies out (and topk_idx / topk_w when non-NULL) back, and
+ * synchronises `stream` before returning.  Pinned host memory is fastest. */
+moe_status moe_forward_host(moe_handle* handle, const void* hidden_host, int T,
+                            void* out_host, int32_t* topk_idx_host,
+                            float* topk_w_host, void* stream);
+
+/* Routing bookkeeping of the last forward, device-to-device, async:
+ *   counts  [E]    int32 tokens per expert
+ *   offsets [E+1]  int32 exclusive prefix sum of counts
+ *   perm    [T*k]  int32 pair ids t*k+j grouped by expert asc, token asc
+ *   pos     [T*k]  int32 position of pair (t, j) inside perm
+ * Any pointer may be NULL. */
+moe_status moe_get_routing(moe_handle* handle, int32_t* counts, int32_t* offsets,
+                           int32_t* perm, int32_t* pos, void* stream);
+
+/* Stage timing.  With `on` != 0 every later moe_forward records a CUDA event
+ * on its stream before each stage; moe_profile_read() waits for the last
+ * forward's events and writes up to n stage durations in milliseconds, in the
+ * order MOE_STAGE_*.  Returns MOE_ERR_INVALID_ARG if no forward was profiled. */
+enum {
+  MOE_STAGE_ROUTER_LOGITS = 0,   /* fixed-order fp64 gate dot products        */
+  MOE_STAGE_ROUTE = 1,           /* sigmoid, top-k, weights, grouping         */
+  MOE_STAGE_DENSE_IN = 2,        /* fc1_latent_proj and shared up + ReLU^2    */
+  MOE_STAGE_EXPERT_UP = 3,       /* grouped up projection + ReLU^2            */
+  MOE_STAGE_EXPERT_DOWN = 4,     /* grouped down projection                   */
+  MOE_STAGE_COMBINE = 5,         /* weighted combine in slot order            */
+  MOE_STAGE_DENSE_OUT = 6,       /* fc2_latent_proj + shared down             */
+  MOE_NUM_STAGES = 7
+};
+moe_status moe_profile_enable(moe_handle* handle, int on);
+moe_status moe_profile_read(moe_handle* handle, float* stage_ms, int n);
+
+/* Drain `stream` and report (then clear) the device error word. */
+moe_status moe_sync(moe_handle* handle, void* stream);
+
+/* Free everything moe_init allocated.  NULL is ignored. */
+void moe_destroy(moe_handle* handle);
+
+const char* moe_status_string(moe_status s);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LATENTMOE_H */

@@ -1,0 +1,320 @@
+// C ABI of the LatentMoE layer: handle, workspace, validation and the launch
+// sequence of one forward (Nemotron-3-Ultra architecture report, section 5.6).
+#include <cuda_runtime.h>
+
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "latentmoe.h"
+
+using namespace lmoe;
+
+struct moe_handle {
+  moe_config cfg;
+  int device = 0;
+  std::vector<void*> owned;          // device allocations to free
+  // weights (borrowed or owned)
+  const void *w_gate = nullptr, *w_fc1 = nullptr, *w_fc2 = nullptr;
+  const void *w_su = nullptr, *w_sd = nullptr, *w_up = nullptr, *w_down = nullptr;
+  const float* bias = nullptr;
+  // workspace, sized for max_tokens
+  float* logits = nullptr;
+  int32_t *topk_idx = nullptr, *rank = nullptr, *blkcnt = nullptr, *blkpre = nullptr;
+  float* topk_w = nullptr;
+  int32_t *counts = nullptr, *offsets = nullptr, *perm = nullptr, *pos = nullptr;
+  int32_t *tiles_up = nullptr, *tiles_dn = nullptr;
+  void *z = nullptr, *h_sh = nullptr, *H = nullptr, *zc = nullptr;
+  float* Y = nullptr;
+  int* err = nullptr;
+  void *x_stage = nullptr, *out_stage = nullptr;   // moe_forward_host buffers
+  int last_T = 0;
+  int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
+  cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
+};
+
+namespace {
+
+size_t dt_size(moe_dtype d) { return d == MOE_BF16 ? 2 : 4; }
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+template <typename P>
+bool dev_alloc(moe_handle* h, P** p, size_t bytes) {
+  void* q = nullptr;
+  if (bytes == 0) bytes = 16;
+  if (cudaMalloc(&q, bytes) != cudaSuccess) { cudaGetLastError(); return false; }
+  h->owned.push_back(q);
+  *p = reinterpret_cast<P*>(q);
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status validate(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->d_model <= 0 || c->d_latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 ||
+      c->d_ff <= 0 || c->d_ff_shared <= 0 || c->max_tokens <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
+  if (c->d_model % 8 || c->d_latent % 8 || c->d_ff % 8 || c->d_ff_shared % 8)
+    return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->out_dtype != MOE_FP32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->n_group != 1 || c->topk_group != 1) return MOE_ERR_UNSUPPORTED;
+  if (c->n_experts > 1024 || c->top_k > 64) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_fmt != MOE_EXPERT_DENSE) return MOE_ERR_UNSUPPORTED;
+  if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Upper bound of the grouped-GEMM tile count: sum_e ceil(c_e / MT) * NC.
+int max_tiles(const moe_config& c, int T, int N) {
+  long P = (long)T * c.top_k;
+  long t = (P / kMT + c.n_experts) * (long)ceil_div(N, kChunk);
+  return t > 0x7fffffff ? 0x7fffffff : (int)t;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_OOM: return "device out of memory";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_CHECK: return "device-side index check failed";
+  }
+  return "unknown status";
+}
+
+int moe_version(void) { return 100; }
+
+void moe_destroy(moe_handle* h) {
+  if (!h) return;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  cudaSetDevice(h->device);
+  for (void* p : h->owned) cudaFree(p);
+  for (cudaEvent_t e : h->ev)
+    if (e) cudaEventDestroy(e);
+  cudaSetDevice(cur);
+  delete h;
+}
+
+moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* w,
+                    void* stream) {
+  if (!out || !w) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const void* ptrs[] = {w->w_gate, w->gate_bias, w->w_fc1, w->w_fc2, w->w_shared_up,
+                        w->w_shared_down, w->w_up, w->w_down};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  moe_handle* h = new (std::nothrow) moe_handle();
+  if (!h) return MOE_ERR_OOM;
+  h->cfg = *cfg;
+  cudaGetDevice(&h->device);
+  const moe_config& c = h->cfg;
+  const size_t D = c.d_model, L = c.d_latent, E = c.n_experts, F = c.d_ff, Fs = c.d_ff_shared;
+  const size_t T = c.max_tokens, k = c.top_k, P = T * k, nblk = (T + 31) / 32;
+  const size_t ds = dt_size(c.dtype);
+  cudaStream_t s = (cudaStream_t)stream;
+  bool ok = true;
+  if (w->borrow) {
+    h->w_gate = w->w_gate; h->w_fc1 = w->w_fc1; h->w_fc2 = w->w_fc2;
+    h->w_su = w->w_shared_up; h->w_sd = w->w_shared_down;
+    h->w_up = w->w_up; h->w_down = w->w_down; h->bias = w->gate_bias;
+  } else {
+    struct { const void* src; const void** dst; size_t bytes; } cp[] = {
+        {w->w_gate, &h->w_gate, E * D * ds},    {w->w_fc1, &h->w_fc1, L * D * ds},
+        {w->w_fc2, &h->w_fc2, D * L * ds},      {w->w_shared_up, &h->w_su, Fs * D * ds},
+        {w->w_shared_down, &h->w_sd, D * Fs * ds}, {w->w_up, &h->w_up, E * F * L * ds},
+        {w->w_down, &h->w_down, E * L * F * ds}, {w->gate_bias, (const void**)&h->bias, E * 4}};
+    for (auto& q : cp) {
+      void* d = nullptr;
+      ok = ok && dev_alloc(h, &d, q.bytes);
+      if (!ok) break;
+      *q.dst = d;
+      if (cudaMemcpyAsync(d, q.src, q.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+        moe_destroy(h);
+        return MOE_ERR_CUDA;
+      }
+    }
+  }
+  ok = ok && dev_alloc(h, &h->logits, T * E * 4) && dev_alloc(h, &h->topk_idx, P * 4) &&
+       dev_alloc(h, &h->topk_w, P * 4) && dev_alloc(h, &h->rank, P * 4) &&
+       dev_alloc(h, &h->blkcnt, E * nblk * 4) && dev_alloc(h, &h->blkpre, E * nblk * 4) &&
+       dev_alloc(h, &h->counts, E * 4) && dev_alloc(h, &h->offsets, (E + 1) * 4) &&
+       dev_alloc(h, &h->perm, P * 4) && dev_alloc(h, &h->pos, P * 4) &&
+       dev_alloc(h, &h->tiles_up, (E + 1) * 4) && dev_alloc(h, &h->tiles_dn, (E + 1) * 4) &&
+       dev_alloc(h, &h->z, T * L * ds) && dev_alloc(h, &h->h_sh, T * Fs * ds) &&
+       dev_alloc(h, &h->H, P * F * ds) && dev_alloc(h, &h->Y, P * L * 4) &&
+       dev_alloc(h, &h->zc, T * L * ds) && dev_alloc(h, &h->err, 16);
+  if (!ok) { moe_destroy(h); return MOE_ERR_OOM; }
+  if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    moe_destroy(h);
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
+                       int32_t* topk_idx, float* topk_w, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) { h->last_T = 0; return MOE_OK; }
+  if (!hidden || !out || !aligned16(hidden) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
+  const int F = c.d_ff, Fs = c.d_ff_shared;
+  const moe_dtype dt = c.dtype;
+  int32_t* idx = topk_idx ? topk_idx : h->topk_idx;
+  float* wts = topk_w ? topk_w : h->topk_w;
+  auto mark = [&](int stage) {
+    if (h->prof) cudaEventRecord(h->ev[stage], s);
+  };
+  mark(MOE_STAGE_ROUTER_LOGITS);
+
+  // steps 1-4: logits, sigmoid, biased selection, weights; step 6 bookkeeping
+  launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
+  mark(MOE_STAGE_ROUTE);
+  RouteArgs ra{};
+  ra.logits = h->logits; ra.bias = h->bias; ra.T = T; ra.E = E; ra.k = k;
+  ra.rsf = c.routed_scaling_factor; ra.topk_idx = idx; ra.topk_w = wts; ra.rank = h->rank;
+  ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
+  ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
+  ra.mt_up = kMT; ra.nc_up = ceil_div(F, kChunk); ra.tiles_up = h->tiles_up;
+  ra.mt_dn = kMT; ra.nc_dn = ceil_div(L, kChunk); ra.tiles_dn = h->tiles_dn;
+  ra.err = h->err;
+  launch_route(ra, s);
+  mark(MOE_STAGE_DENSE_IN);
+
+  // step 5 and the shared expert's up projection: both read x
+  DenseArgs g1{};
+  g1.A0 = hidden; g1.W0 = h->w_fc1; g1.K0 = D; g1.K1 = 0;
+  g1.out = h->z; g1.ldo = L; g1.M = T; g1.N = L; g1.epi = EPI_NONE;
+  g1.in_dt = dt; g1.out_dt = dt;
+  launch_dense(g1, s);
+  DenseArgs gs = g1;
+  gs.W0 = h->w_su; gs.out = h->h_sh; gs.ldo = Fs; gs.N = Fs; gs.epi = EPI_RELU2;
+  launch_dense(gs, s);
+  mark(MOE_STAGE_EXPERT_UP);
+
+  // step 6: routed experts in the latent space
+  GroupedArgs up{};
+  up.A = h->z; up.W = h->w_up; up.out = h->H; up.K = L; up.N = F; up.E = E; up.k = k;
+  up.offsets = h->offsets; up.perm = h->perm; up.tiles = h->tiles_up; up.gather = 1;
+  up.epi = EPI_RELU2; up.in_dt = dt; up.out_dt = dt; up.err = h->err;
+  launch_grouped(up, max_tiles(c, T, F), s);
+  mark(MOE_STAGE_EXPERT_DOWN);
+  GroupedArgs dn = up;
+  dn.A = h->H; dn.W = h->w_down; dn.out = h->Y; dn.K = F; dn.N = L; dn.perm = nullptr;
+  dn.tiles = h->tiles_dn; dn.gather = 0; dn.epi = EPI_NONE; dn.out_dt = MOE_FP32;
+  launch_grouped(dn, max_tiles(c, T, L), s);
+  mark(MOE_STAGE_COMBINE);
+  launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, dt, s);
+  mark(MOE_STAGE_DENSE_OUT);
+
+  // step 7: fc2_latent_proj and the shared expert's down projection, one GEMM
+  DenseArgs g5{};
+  g5.A0 = h->zc; g5.W0 = h->w_fc2; g5.K0 = L;
+  g5.A1 = h->h_sh; g5.W1 = h->w_sd; g5.K1 = Fs;
+  g5.out = out; g5.ldo = D; g5.M = T; g5.N = D; g5.epi = EPI_NONE;
+  g5.in_dt = dt; g5.out_dt = c.out_dtype;
+  launch_dense(g5, s);
+  mark(MOE_NUM_STAGES);
+  h->prof_valid = h->prof;
+  h->last_T = T;
+  return cuda_status(cudaGetLastError());
+}
+
+moe_status moe_forward_host(moe_handle* h, const void* hidden_host, int T, void* out_host,
+                            int32_t* topk_idx_host, float* topk_w_host, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!hidden_host || !out_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t in_bytes = (size_t)T * c.d_model * dt_size(c.dtype);
+  const size_t out_bytes = (size_t)T * c.d_model * dt_size(c.out_dtype);
+  if (!h->x_stage) {
+    const size_t mx = (size_t)c.max_tokens * c.d_model * 4;
+    if (!dev_alloc(h, &h->x_stage, mx) || !dev_alloc(h, &h->out_stage, mx)) return MOE_ERR_OOM;
+  }
+  cudaError_t e = cudaMemcpyAsync(h->x_stage, hidden_host, in_bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  moe_status st = moe_forward(h, h->x_stage, T, h->out_stage, nullptr, nullptr, s);
+  if (st != MOE_OK) return st;
+  const size_t P = (size_t)T * c.top_k;
+  e = cudaMemcpyAsync(out_host, h->out_stage, out_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && topk_idx_host)
+    e = cudaMemcpyAsync(topk_idx_host, h->topk_idx, P * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && topk_w_host)
+    e = cudaMemcpyAsync(topk_w_host, h->topk_w, P * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+moe_status moe_get_routing(moe_handle* h, int32_t* counts, int32_t* offsets, int32_t* perm,
+                           int32_t* pos, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int E = h->cfg.n_experts;
+  const size_t P = (size_t)h->last_T * h->cfg.top_k;
+  cudaError_t e = cudaSuccess;
+  if (counts) e = cudaMemcpyAsync(counts, h->counts, E * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && offsets)
+    e = cudaMemcpyAsync(offsets, h->offsets, (E + 1) * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && perm && P)
+    e = cudaMemcpyAsync(perm, h->perm, P * 4, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess && pos && P)
+    e = cudaMemcpyAsync(pos, h->pos, P * 4, cudaMemcpyDeviceToDevice, s);
+  return cuda_status(e);
+}
+
+moe_status moe_profile_enable(moe_handle* h, int on) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (on && !h->ev[0]) {
+    for (cudaEvent_t& e : h->ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  h->prof = on ? 1 : 0;
+  h->prof_valid = 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_handle* h, float* stage_ms, int n) {
+  if (!h || !stage_ms || n <= 0 || !h->prof_valid) return MOE_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(h->ev[MOE_NUM_STAGES]) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int i = 0; i < n && i < MOE_NUM_STAGES; ++i)
+    if (cudaEventElapsedTime(&stage_ms[i], h->ev[i], h->ev[i + 1]) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_sync(moe_handle* h, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (word) {
+    cudaMemset(h->err, 0, sizeof(int));
+    return (word & DEV_ERR_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE_CHECK;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,308 @@
+// Router of the LatentMoE layer (Nemotron-3-Ultra architecture report,
+// chapter 5: section 5.3 sigmoid gating, 5.4 correction bias, 5.5 top-k,
+// 5.6 steps 1-4 and the token->expert grouping of step 6).
+//
+//   router_logits_kernel : l[t,e] = fp32(fixed-order fp64 dot(x[t], W_gate[e]))
+//   route_kernel         : sigmoid, +bias, warp top-k, weights, per-block masks
+//   route_scan_kernel    : per-expert counts, exclusive offsets, tile offsets
+//   route_perm_kernel    : perm (expert asc, token asc) and its inverse pos
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lmoe {
+
+// ---------------------------------------------------------------------------
+// Router logits.  One warp per (expert, group of TT tokens).  Lane p owns the
+// partial sum of every k with (k/8) % 32 == p, added in increasing k with fp64
+// FMAs (each bf16*bf16 or fp32*fp32 product is exact in fp64, so the FMA
+// equals adding the exact product); the 32 partials are then combined by
+// shfl_down with offsets 16, 8, 4, 2, 1 and lane 0 holds the sum.
+// ---------------------------------------------------------------------------
+template <typename T, int TT>
+__global__ void __launch_bounds__(256)
+router_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg,
+                     float* __restrict__ logits, int n_tok, int D, int E) {
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int t0 = blockIdx.y * TT;
+  if (e >= E) return;
+  double acc[TT];
+#pragma unroll
+  for (int i = 0; i < TT; ++i) acc[i] = 0.0;
+  const T* wrow = wg + (size_t)e * D;
+  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
+    float w[8];
+    load8(wrow + k0, w);
+#pragma unroll
+    for (int i = 0; i < TT; ++i) {
+      if (t0 + i < n_tok) {
+        float xv[8];
+        load8(x + (size_t)(t0 + i) * D + k0, xv);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[i] = fma((double)xv[r], (double)w[r], acc[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < TT; ++i) {
+    double v = acc[i];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v = __dadd_rn(v, __shfl_down_sync(0xffffffffu, v, off));
+    if (lane == 0 && t0 + i < n_tok) logits[(size_t)(t0 + i) * E + e] = __double2float_rn(v);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// exp in fp64 from IEEE +, *, rint and scalbn only: a = n ln2 + r with a
+// two-part (Cody-Waite) ln 2 whose high part has 32 significant bits, then the
+// degree-13 Taylor polynomial of exp(r) by Horner.  The explicit _rn
+// intrinsics keep the compiler from contracting a*b+c into an FMA, so the
+// result is the same bit pattern on any IEEE machine that does the same steps.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double exp_fixed(double a) {
+  const double kInvLn2 = 0x1.71547652b82fep+0;
+  const double kLn2Hi = 0x1.62e42fee00000p-1;
+  const double kLn2Lo = 0x1.a39ef35793c76p-33;
+  const double c[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1,
+                        0x1.5555555555555p-3, 0x1.5555555555555p-5, 0x1.1111111111111p-7,
+                        0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
+                        0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+                        0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+  double n = rint(__dmul_rn(a, kInvLn2));
+  double r = __dsub_rn(__dsub_rn(a, __dmul_rn(n, kLn2Hi)), __dmul_rn(n, kLn2Lo));
+  double p = c[13];
+#pragma unroll
+  for (int i = 12; i >= 0; --i) p = __dadd_rn(__dmul_rn(p, r), c[i]);
+  return scalbn(p, (int)n);
+}
+
+__device__ __forceinline__ float sigmoid_fixed(float l) {
+  double a = -fmin(fmax((double)l, -80.0), 80.0);
+  return __double2float_rn(__ddiv_rn(1.0, __dadd_rn(1.0, exp_fixed(a))));
+}
+
+// (c, e) ranks above (c2, e2): larger score, or equal score and lower index.
+__device__ __forceinline__ bool ranks_above(float c, int e, float c2, int e2) {
+  return c > c2 || (c == c2 && e < e2);
+}
+
+// ---------------------------------------------------------------------------
+// Selection and weights.  Block = 32 warps = 32 consecutive tokens, one warp
+// per token; lane l holds experts l, l+32, ... (EPL of them).  k rounds of a
+// warp arg-max over (choice desc, expert asc) give the slots in order.  The
+// raw scores of the winners are summed in fp32 in slot order and the weights
+// are (r / (S + 1e-20)) * rsf, all with round-to-nearest intrinsics.
+// Each selected expert ORs the token's bit into mask[e]; a token's rank among
+// the block's tokens that chose e is the popcount of the lower bits, and the
+// block's count of e is the popcount of the mask.
+// ---------------------------------------------------------------------------
+constexpr int kMaxTopK = 64;
+
+template <int EPL>
+__global__ void __launch_bounds__(1024)
+route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+             int n_tok, int E, int k, float rsf,
+             int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+             int32_t* __restrict__ rank, int32_t* __restrict__ blkcnt, int nblk,
+             int* __restrict__ err) {
+  extern __shared__ uint32_t mask[];                 // [E]
+  __shared__ float rsel[32][kMaxTopK];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * 32 + warp;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) mask[e] = 0u;
+  __syncthreads();
+  if (t < n_tok) {
+    float s[EPL], c[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E) {
+        s[i] = sigmoid_fixed(logits[(size_t)t * E + e]);
+        c[i] = __fadd_rn(s[i], bias[e]);
+      } else {
+        s[i] = 0.f;
+        c[i] = -INFINITY;
+      }
+    }
+    uint32_t taken = 0u;                             // bit i: expert lane+32i chosen
+    for (int j = 0; j < k; ++j) {
+      float bc = -INFINITY;
+      int be = 0x7fffffff, bi = -1;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !(taken >> i & 1u) && (bi < 0 || ranks_above(c[i], e, bc, be))) {
+          bc = c[i]; be = e; bi = i;
+        }
+      }
+      float wc = bc;
+      int we = be;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        float oc = __shfl_xor_sync(0xffffffffu, wc, off);
+        int oe = __shfl_xor_sync(0xffffffffu, we, off);
+        if (oe != 0x7fffffff && (we == 0x7fffffff || ranks_above(oc, oe, wc, we))) {
+          wc = oc; we = oe;
+        }
+      }
+      float r = 0.f;
+      if (we != 0x7fffffff && (we & 31) == lane) {
+        const int i = we >> 5;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q)
+          if (q == i) { r = s[q]; taken |= 1u << q; }
+        atomicOr(&mask[we], 1u << warp);
+      }
+      r = __shfl_sync(0xffffffffu, r, we & 31);
+      if (lane == 0) {
+        rsel[warp][j] = r;
+        topk_idx[(size_t)t * k + j] = we;
+        if (we < 0 || we >= E) atomicOr(err, DEV_ERR_INDEX);
+      }
+    }
+    __syncwarp();
+    float S = 0.f;
+    for (int j = 0; j < k; ++j) S = __fadd_rn(S, rsel[warp][j]);
+    const float den = __fadd_rn(S, 1e-20f);
+    for (int j = lane; j < k; j += 32)
+      topk_w[(size_t)t * k + j] = __fmul_rn(__fdiv_rn(rsel[warp][j], den), rsf);
+  }
+  __syncthreads();
+  if (t < n_tok) {
+    for (int j = lane; j < k; j += 32) {
+      const int e = topk_idx[(size_t)t * k + j];
+      rank[(size_t)t * k + j] = __popc(mask[e] & ((1u << warp) - 1u));
+    }
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    blkcnt[(size_t)e * nblk + blockIdx.x] = __popc(mask[e]);
+}
+
+// ---------------------------------------------------------------------------
+// Counts and offsets, one block of 1024 threads.  Warp w scans the per-block
+// counts of experts w, w+32, ... over the token blocks (blkpre = exclusive
+// prefix over blocks), then the block scans the per-expert totals into the
+// exclusive offsets and into the tile offsets of the two grouped GEMMs
+// (tiles of an expert = ceil(count / mt) * n_chunks).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+// Exclusive scan of val over the 1024 threads; returns the prefix, and the
+// grand total in *total (all threads).
+__device__ int block_excl_scan(int val, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = warp_incl_scan(val, lane);
+  __syncthreads();
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+    int wi = warp_incl_scan(w, lane);
+    warp_tot[lane] = wi - w;
+    if (lane == 31) warp_tot[32] = wi;
+  }
+  __syncthreads();
+  int r = warp_tot[warp] + incl - val;
+  *total = warp_tot[32];
+  return r;
+}
+
+__global__ void __launch_bounds__(1024)
+route_scan_kernel(const int32_t* __restrict__ blkcnt, int nblk, int E,
+                  int32_t* __restrict__ blkpre, int32_t* __restrict__ counts,
+                  int32_t* __restrict__ offsets, int mt_up, int nc_up,
+                  int32_t* __restrict__ tiles_up, int mt_dn, int nc_dn,
+                  int32_t* __restrict__ tiles_dn) {
+  __shared__ int tot[1024];
+  __shared__ int wt[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = warp; e < E; e += 32) {
+    int run = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < nblk ? blkcnt[(size_t)e * nblk + b] : 0;
+      const int incl = warp_incl_scan(v, lane);
+      if (b < nblk) blkpre[(size_t)e * nblk + b] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) tot[e] = run;
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int c = e < E ? tot[e] : 0;
+  int all;
+  const int off = block_excl_scan(c, wt, &all);
+  if (e < E) { counts[e] = c; offsets[e] = off; }
+  if (e == 0) offsets[E] = all;
+  const int tu = e < E ? (c + mt_up - 1) / mt_up * nc_up : 0;
+  const int ou = block_excl_scan(tu, wt, &all);
+  if (e < E) tiles_up[e] = ou;
+  if (e == 0) tiles_up[E] = all;
+  const int td = e < E ? (c + mt_dn - 1) / mt_dn * nc_dn : 0;
+  const int od = block_excl_scan(td, wt, &all);
+  if (e < E) tiles_dn[e] = od;
+  if (e == 0) tiles_dn[E] = all;
+}
+
+// pos[t*k+j] = offsets[e] + (pairs of e in earlier token blocks) + rank in block
+__global__ void route_perm_kernel(const int32_t* __restrict__ topk_idx,
+                                  const int32_t* __restrict__ rank,
+                                  const int32_t* __restrict__ blkpre,
+                                  const int32_t* __restrict__ offsets, int n_tok,
+                                  int k, int nblk, int32_t* __restrict__ perm,
+                                  int32_t* __restrict__ pos) {
+  const long p = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= (long)n_tok * k) return;
+  const int t = (int)(p / k);
+  const int e = topk_idx[p];
+  const int q = offsets[e] + blkpre[(size_t)e * nblk + (t >> 5)] + rank[p];
+  pos[p] = q;
+  perm[q] = (int32_t)p;
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers
+// ---------------------------------------------------------------------------
+void launch_router_logits(const void* x, const void* wg, float* logits, int T,
+                          int D, int E, moe_dtype dt, cudaStream_t st) {
+  constexpr int TT = 8;
+  dim3 grid(ceil_div(E, 8), ceil_div(T, TT));
+  if (dt == MOE_BF16)
+    router_logits_kernel<__nv_bfloat16, TT><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)x, (const __nv_bfloat16*)wg, logits, T, D, E);
+  else
+    router_logits_kernel<float, TT><<<grid, 256, 0, st>>>(
+        (const float*)x, (const float*)wg, logits, T, D, E);
+}
+
+template <int EPL>
+static void route_launch_epl(const RouteArgs& a, cudaStream_t st) {
+  route_kernel<EPL><<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(
+      a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w, a.rank,
+      a.blkcnt, a.nblk, a.err);
+}
+
+void launch_route(const RouteArgs& a, cudaStream_t st) {
+  const int epl = (a.E + 31) / 32;
+  if (epl <= 1) route_launch_epl<1>(a, st);
+  else if (epl <= 2) route_launch_epl<2>(a, st);
+  else if (epl <= 4) route_launch_epl<4>(a, st);
+  else if (epl <= 8) route_launch_epl<8>(a, st);
+  else if (epl <= 16) route_launch_epl<16>(a, st);
+  else route_launch_epl<32>(a, st);
+  route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
+                                        a.offsets, a.mt_up, a.nc_up, a.tiles_up,
+                                        a.mt_dn, a.nc_dn, a.tiles_dn);
+  const long P = (long)a.T * a.k;
+  route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
+      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+}
+
+}  // namespace lmoe

@@ -1,0 +1,118 @@
+"""torch-facing wrapper of one liblatentmoe handle (marshalling only).
+
+    layer = LatentMoE(dims, weights, max_tokens=T, out_dtype="fp32")
+    out, topk_idx, topk_w = layer(x)          # x: [T, d_model] on cuda
+
+torch provides the device buffers and the current stream; every step of the
+layer runs in the CUDA library.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+_TORCH_DT = {"fp32": torch.float32, "bf16": torch.bfloat16}
+
+
+class LatentMoE:
+    """One LatentMoE layer bound to device weights (borrowed, not copied).
+
+    weights: dict with w_gate [E,D], gate_bias [E] fp32, w_fc1 [L,D],
+    w_fc2 [D,L], w_shared_up [Fs,D], w_shared_down [D,Fs], w_up [E,F,L],
+    w_down [E,L,F], all contiguous cuda tensors in `dtype` (bias fp32)."""
+
+    def __init__(self, D, L, E, k, F, Fs, weights, *, max_tokens, rsf=5.0,
+                 dtype="bf16", expert_fmt="dense", out_dtype=None,
+                 n_group=1, topk_group=1):
+        self.dims = dict(D=D, L=L, E=E, k=k, F=F, Fs=Fs)
+        self.dtype = dtype
+        self.out_dtype = out_dtype or dtype
+        self.max_tokens = max_tokens
+        self._w = {n: t.contiguous() for n, t in weights.items()}
+        for n, t in self._w.items():
+            if not t.is_cuda:
+                raise ValueError(f"weight {n} must be a cuda tensor")
+        cfg = B.moe_config(D, L, E, k, F, Fs, n_group, topk_group, max_tokens,
+                           float(rsf), B.DTYPE[dtype], B.EXPERT_FMT[expert_fmt],
+                           B.DTYPE[self.out_dtype])
+        w = B.moe_weights(*(self._w[n].data_ptr() for n in (
+            "w_gate", "gate_bias", "w_fc1", "w_fc2", "w_shared_up",
+            "w_shared_down", "w_up", "w_down")), 1)
+        self.cfg = cfg
+        self.handle = B.moe_init(cfg, w, torch.cuda.current_stream().cuda_stream)
+
+    @property
+    def stream(self) -> int:
+        return torch.cuda.current_stream().cuda_stream
+
+    def __call__(self, x, out=None, topk_idx=None, topk_w=None):
+        T = x.shape[0]
+        D, k = self.dims["D"], self.dims["k"]
+        if x.dtype != _TORCH_DT[self.dtype] or not x.is_cuda or x.shape[1] != D:
+            raise ValueError("x must be a cuda [T, d_model] tensor in the layer dtype")
+        x = x.contiguous()
+        if out is None:
+            out = torch.empty(T, D, dtype=_TORCH_DT[self.out_dtype], device=x.device)
+        if topk_idx is None:
+            topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+        B.moe_forward(self.handle, x.data_ptr(), T, out.data_ptr(),
+                      topk_idx.data_ptr(), topk_w.data_ptr(), self.stream)
+        return out, topk_idx, topk_w
+
+    def forward_host(self, x_host, out_host, topk_idx_host=None, topk_w_host=None):
+        """Host buffers in and out (pinned is fastest); synchronises."""
+        B.moe_forward_host(self.handle, x_host.data_ptr(), x_host.shape[0],
+                           out_host.data_ptr(),
+                           None if topk_idx_host is None else topk_idx_host.data_ptr(),
+                           None if topk_w_host is None else topk_w_host.data_ptr(),
+                           self.stream)
+        return out_host
+
+    def routing(self, T):
+        """(counts[E], offsets[E+1], perm[T*k], pos[T*k]) of the last forward."""
+        E, k = self.dims["E"], self.dims["k"]
+        dev = torch.device("cuda")
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+        pos = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+        B.moe_get_routing(self.handle, counts.data_ptr(), offsets.data_ptr(),
+                          perm.data_ptr(), pos.data_ptr(), self.stream)
+        return counts, offsets, perm[:T * k], pos[:T * k]
+
+    def sync(self):
+        B.moe_sync(self.handle, self.stream)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            B.moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def weights_for(cfg, device="cuda"):
+    """Generate a config's synthetic weights on `device` (inputs module)."""
+    from . import inputs as I
+    dt = _TORCH_DT[cfg.dtype]
+    up = torch.empty(cfg.E, cfg.F, cfg.L, dtype=dt, device=device)
+    down = torch.empty(cfg.E, cfg.L, cfg.F, dtype=dt, device=device)
+    I.w_up_into(cfg, up)
+    I.w_down_into(cfg, down)
+    return dict(w_gate=I.w_gate(cfg, device), gate_bias=I.gate_bias(cfg, device),
+                w_fc1=I.w_fc1(cfg, device), w_fc2=I.w_fc2(cfg, device),
+                w_shared_up=I.w_shared_up(cfg, device),
+                w_shared_down=I.w_shared_down(cfg, device), w_up=up, w_down=down)
+
+
+def layer_for(cfg, weights, max_tokens=None, out_dtype=None):
+    return LatentMoE(cfg.D, cfg.L, cfg.E, cfg.k, cfg.F, cfg.Fs, weights,
+                     max_tokens=max_tokens or cfg.T, rsf=cfg.rsf, dtype=cfg.dtype,
+                     expert_fmt=cfg.expert_fmt, out_dtype=out_dtype)

@@ -1,0 +1,84 @@
+"""The C-ABI library: it builds, loads and exports every declared entry point,
+and host-side validation answers without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", "latentmoe.h")]
+
+
+def _declared():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def B():
+    from latentmoe_expert_routing_b200 import build
+    build.build()
+    from latentmoe_expert_routing_b200 import binding
+    return binding
+
+
+def test_every_declared_symbol_is_exported(B):
+    names = _declared()
+    assert "moe_forward" in names and "moe_init" in names
+    for n in names:
+        assert hasattr(B.lib, n), n
+    bound = {s[0] for s in B.SIGNATURES}
+    assert set(names) <= bound, set(names) - bound
+
+
+def test_status_strings_and_version(B):
+    assert B.status_string(0) == "ok"
+    assert "unsupported" in B.status_string(B.MOE_ERR_UNSUPPORTED)
+    assert B.moe_version() >= 100
+
+
+def _cfg(B, **kw):
+    d = dict(d_model=256, d_latent=64, n_experts=16, top_k=4, d_ff=128,
+             d_ff_shared=256, n_group=1, topk_group=1, max_tokens=64,
+             routed_scaling_factor=5.0, dtype=B.MOE_FP32,
+             expert_fmt=B.MOE_EXPERT_DENSE, out_dtype=B.MOE_FP32)
+    d.update(kw)
+    return B.moe_config(**d)
+
+
+def _w(B, ptr=4096):
+    return B.moe_weights(*([ptr] * 8), 1)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(top_k=17), 1), (dict(d_model=0), 1), (dict(d_latent=60), 1),
+    (dict(max_tokens=0), 1), (dict(dtype=7), 1),
+    (dict(n_group=2), 2), (dict(topk_group=2), 2), (dict(n_experts=2048), 2),
+    (dict(top_k=80, n_experts=100), 2),
+])
+def test_init_rejects_bad_config_before_any_launch(B, kw, status):
+    h = ctypes.c_void_p()
+    cfg = _cfg(B, **kw)
+    assert B.lib.moe_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(_w(B)), None) == status
+    assert not h.value
+
+
+def test_init_rejects_null_and_misaligned_weights(B):
+    h = ctypes.c_void_p()
+    cfg = _cfg(B)
+    assert B.lib.moe_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(_w(B, 0)), None) == 1
+    assert B.lib.moe_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(_w(B, 4100)), None) == 1
+    assert B.lib.moe_init(None, ctypes.byref(cfg), ctypes.byref(_w(B)), None) == 1
+
+
+def test_calls_on_null_handle(B):
+    assert B.lib.moe_forward(None, None, 1, None, None, None, None) == 1
+    assert B.lib.moe_forward_host(None, None, 1, None, None, None, None) == 1
+    assert B.lib.moe_get_routing(None, None, None, None, None, None) == 1
+    assert B.lib.moe_sync(None, None) == 1
+    B.lib.moe_destroy(None)
