@@ -148,6 +148,36 @@ enum {
 moe_status moe_profile_enable(moe_handle* handle, int on);
 moe_status moe_profile_read(moe_handle* handle, float* stage_ms, int n);
 
+/* Router only -- logits, sigmoid, biased top-k and weights, the same results
+ * bit for bit as moe_forward's topk_idx / topk_w -- for callers that cannot
+ * allocate device memory.  The report has no counterpart of this entry point.
+ *
+ * Some callers may not call cudaMalloc or let a library call it: a serving
+ * loop that owns every byte of a fixed HBM budget, a framework whose allocator
+ * must account for all device memory, or a latency-critical path that cannot
+ * afford cudaMalloc's implicit device synchronisation.  This call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.  Its
+ * scratch (logits, ranks, per-block counts, an error word) is one fixed 8 MiB
+ * array in the library's device image, which every GPU that loads the library
+ * holds until the process exits.  The scratch needed is
+ *   256 + align256(4*T*E) + align256(4*T*k) + align256(4*E*ceil(T/32)) bytes
+ * (T <= 3812 tokens at E = 512, k = 22); larger T returns MOE_ERR_INVALID_ARG.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls on a device share the one array and
+ * it keeps the last call's contents, so calls that overlap on the GPU (other
+ * streams, other host threads) race: serialise them.  The error word is
+ * cleared at the start of each call.
+ *   hidden [T, d_model] dtype, w_gate [n_experts, d_model] dtype, gate_bias
+ *   [n_experts] fp32, topk_idx [T, top_k] int32, topk_w [T, top_k] fp32: all
+ *   device pointers, hidden and w_gate 16-byte aligned.  Asynchronous. */
+moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
+                             const float* gate_bias, int T, int d_model,
+                             int n_experts, int top_k, float routed_scaling_factor,
+                             moe_dtype dtype, int32_t* topk_idx, float* topk_w,
+                             void* stream);
+
 /* Drain `stream` and report (then clear) the device error word. */
 moe_status moe_sync(moe_handle* handle, void* stream);
 

@@ -56,6 +56,8 @@ SIGNATURES = [
     ("moe_get_routing", _i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     ("moe_profile_enable", _i, [_vp, _i]),
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
+    ("moe_route_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i,
+                               _vp, _vp, _vp]),
     ("moe_sync", _i, [_vp, _vp]),
     ("moe_destroy", None, [_vp]),
     ("moe_status_string", ctypes.c_char_p, [_i]),
@@ -123,6 +125,14 @@ def moe_profile_read(h):
     buf = (ctypes.c_float * MOE_NUM_STAGES)()
     _check(_lib.moe_profile_read(h, buf, MOE_NUM_STAGES), "moe_profile_read")
     return dict(zip(STAGES, list(buf)))
+
+
+def moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts, top_k, rsf,
+                      dtype, topk_idx, topk_w, stream):
+    """Router with no device allocation (scratch in a fixed library array)."""
+    _check(_lib.moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts,
+                                  top_k, rsf, dtype, topk_idx, topk_w, stream),
+           "moe_route_noalloc")
 
 
 def moe_sync(h, stream):

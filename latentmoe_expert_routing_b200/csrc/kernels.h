@@ -71,3 +71,9 @@ void launch_combine(const float* Y, const float* topk_w, const int32_t* pos,
                     void* zc, int T, int k, int L, moe_dtype out_dt, cudaStream_t st);
 
 }  // namespace lmoe
+
+namespace lmoe {
+// Selection-only launch (sigmoid, +bias, top-k, weights) over precomputed
+// logits; rank / blkcnt are written for a caller that goes on to group pairs.
+void launch_route_select(const RouteArgs& a, cudaStream_t st);
+}  // namespace lmoe

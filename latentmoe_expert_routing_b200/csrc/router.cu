@@ -289,6 +289,16 @@ static void route_launch_epl(const RouteArgs& a, cudaStream_t st) {
       a.blkcnt, a.nblk, a.err);
 }
 
+void launch_route_select(const RouteArgs& a, cudaStream_t st) {
+  const int epl = (a.E + 31) / 32;
+  if (epl <= 1) route_launch_epl<1>(a, st);
+  else if (epl <= 2) route_launch_epl<2>(a, st);
+  else if (epl <= 4) route_launch_epl<4>(a, st);
+  else if (epl <= 8) route_launch_epl<8>(a, st);
+  else if (epl <= 16) route_launch_epl<16>(a, st);
+  else route_launch_epl<32>(a, st);
+}
+
 void launch_route(const RouteArgs& a, cudaStream_t st) {
   const int epl = (a.E + 31) / 32;
   if (epl <= 1) route_launch_epl<1>(a, st);
