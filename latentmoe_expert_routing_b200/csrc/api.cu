@@ -30,11 +30,19 @@ struct moe_handle {
   int* err = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;   // moe_forward_host buffers
   int last_T = 0;
+  // tensor-core path (bf16): permuted latent rows and cached TMA maps
+  void* z_perm = nullptr;
+  CUtensorMap wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
+  CUtensorMap am_zp[3], am_H[3], am_zc[3], am_hsh[3];   // token boxes of 16, 64, 256 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
   cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
 };
 
 namespace {
+
+const int kNT[3] = {16, 64, 256};
+
+int nt_index(long rows_per_group) { return rows_per_group <= 16 ? 0 : rows_per_group <= 64 ? 1 : 2; }
 
 size_t dt_size(moe_dtype d) { return d == MOE_BF16 ? 2 : 4; }
 
@@ -74,6 +82,71 @@ int max_tiles(const moe_config& c, int T, int N) {
   long P = (long)T * c.top_k;
   long t = (P / kMT + c.n_experts) * (long)ceil_div(N, kChunk);
   return t > 0x7fffffff ? 0x7fffffff : (int)t;
+}
+
+// Tensor-core path for bf16 layers: G1 (fc1, shared up), row gather, grouped
+// up / down, combine, G5 (fc2 + shared down) -- all tcgen05 GEMMs but the gather
+// and the combine.
+template <typename Mark>
+moe_status forward_umma(moe_handle* h, const void* hidden, int T, void* out,
+                        const float* wts, Mark& mark, cudaStream_t s) {
+  const moe_config& c = h->cfg;
+  const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
+  const int F = c.d_ff, Fs = c.d_ff_shared;
+  const long P = (long)T * k;
+  const int di = nt_index(T), gi = nt_index(P / E);
+  const int ntd = kNT[di], ntg = kNT[gi];
+  cudaError_t e;
+
+  UmmaLaunch g{};
+  g.args.err = h->err;
+  g.args.E = 1;
+  g.args.M = T;
+  g.nt = ntd;
+  // step 5: z = x W_fc1^T, and the shared expert's up projection (both read x)
+  if (!make_tmap_bf16(&g.amap0, hidden, T, D, ntd)) return MOE_ERR_CUDA;
+  g.wmap0 = h->wm_fc1;
+  g.args.K0 = D; g.args.K1 = 0; g.args.n_out = L; g.args.ldo = L;
+  g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
+  g.args.out = h->z; g.epi = UMMA_EPI_BF16; g.max_tiles = g.args.dense_tiles;
+  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  g.wmap0 = h->wm_su;
+  g.args.n_out = Fs; g.args.ldo = Fs;
+  g.args.dense_tiles = ceil_div(Fs, 128) * ceil_div(T, ntd);
+  g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
+  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(MOE_STAGE_EXPERT_UP);
+
+  // step 6: routed experts on permuted latent rows (grouped by expert)
+  launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
+  UmmaLaunch u{};
+  u.args.err = h->err;
+  u.args.E = E; u.args.offsets = h->offsets;
+  u.nt = ntg;
+  u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
+  u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
+  u.args.tiles = h->tiles_up; u.args.out = h->H; u.epi = UMMA_EPI_BF16_RELU2;
+  u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
+  if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(MOE_STAGE_EXPERT_DOWN);
+  u.wmap0 = h->wm_dn; u.amap0 = h->am_H[gi];
+  u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
+  u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
+  u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
+  if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(MOE_STAGE_COMBINE);
+  launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
+  mark(MOE_STAGE_DENSE_OUT);
+
+  // step 7: out = zc W_fc2^T + h_sh W_sd^T, one accumulator over K = L + Fs
+  g.wmap0 = h->wm_fc2; g.amap0 = h->am_zc[di];
+  g.wmap1 = h->wm_sd; g.amap1 = h->am_hsh[di];
+  g.args.K0 = L; g.args.K1 = Fs; g.args.n_out = D; g.args.ldo = D;
+  g.args.dense_tiles = ceil_div(D, 128) * ceil_div(T, ntd);
+  g.args.out = out; g.epi = c.out_dtype == MOE_BF16 ? UMMA_EPI_BF16 : UMMA_EPI_F32;
+  g.max_tiles = g.args.dense_tiles;
+  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 }  // namespace
@@ -158,6 +231,25 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
        dev_alloc(h, &h->H, P * F * ds) && dev_alloc(h, &h->Y, P * L * 4) &&
        dev_alloc(h, &h->zc, T * L * ds) && dev_alloc(h, &h->err, 16);
   if (!ok) { moe_destroy(h); return MOE_ERR_OOM; }
+  if (c.dtype == MOE_BF16) {
+    if (c.d_model % 64 || c.d_latent % 64 || c.d_ff % 64 || c.d_ff_shared % 64) {
+      moe_destroy(h);
+      return MOE_ERR_UNSUPPORTED;
+    }
+    if (!dev_alloc(h, &h->z_perm, P * L * 2)) { moe_destroy(h); return MOE_ERR_OOM; }
+    bool m = make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
+             make_tmap_bf16(&h->wm_su, h->w_su, Fs, D, 128) &&
+             make_tmap_bf16(&h->wm_up, h->w_up, E * F, L, 128) &&
+             make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128) &&
+             make_tmap_bf16(&h->wm_fc2, h->w_fc2, D, L, 128) &&
+             make_tmap_bf16(&h->wm_sd, h->w_sd, D, Fs, 128);
+    for (int i = 0; i < 3 && m; ++i)
+      m = make_tmap_bf16(&h->am_zp[i], h->z_perm, P, L, kNT[i]) &&
+          make_tmap_bf16(&h->am_H[i], h->H, P, F, kNT[i]) &&
+          make_tmap_bf16(&h->am_zc[i], h->zc, T, L, kNT[i]) &&
+          make_tmap_bf16(&h->am_hsh[i], h->h_sh, T, Fs, kNT[i]);
+    if (!m) { moe_destroy(h); return MOE_ERR_CUDA; }
+  }
   if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess) {
     moe_destroy(h);
@@ -193,45 +285,57 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.rsf = c.routed_scaling_factor; ra.topk_idx = idx; ra.topk_w = wts; ra.rank = h->rank;
   ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
   ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
-  ra.mt_up = kMT; ra.nc_up = ceil_div(F, kChunk); ra.tiles_up = h->tiles_up;
-  ra.mt_dn = kMT; ra.nc_dn = ceil_div(L, kChunk); ra.tiles_dn = h->tiles_dn;
+  if (dt == MOE_BF16) {           // tensor-core tiles: 128 weight rows x NT pairs
+    const int nt = kNT[nt_index((long)T * k / E)];
+    ra.mt_up = nt; ra.nc_up = ceil_div(F, 128);
+    ra.mt_dn = nt; ra.nc_dn = ceil_div(L, 128);
+  } else {
+    ra.mt_up = kMT; ra.nc_up = ceil_div(F, kChunk);
+    ra.mt_dn = kMT; ra.nc_dn = ceil_div(L, kChunk);
+  }
+  ra.tiles_up = h->tiles_up; ra.tiles_dn = h->tiles_dn;
   ra.err = h->err;
   launch_route(ra, s);
   mark(MOE_STAGE_DENSE_IN);
 
-  // step 5 and the shared expert's up projection: both read x
-  DenseArgs g1{};
-  g1.A0 = hidden; g1.W0 = h->w_fc1; g1.K0 = D; g1.K1 = 0;
-  g1.out = h->z; g1.ldo = L; g1.M = T; g1.N = L; g1.epi = EPI_NONE;
-  g1.in_dt = dt; g1.out_dt = dt;
-  launch_dense(g1, s);
-  DenseArgs gs = g1;
-  gs.W0 = h->w_su; gs.out = h->h_sh; gs.ldo = Fs; gs.N = Fs; gs.epi = EPI_RELU2;
-  launch_dense(gs, s);
-  mark(MOE_STAGE_EXPERT_UP);
+  if (dt == MOE_BF16) {
+    moe_status us = forward_umma(h, hidden, T, out, wts, mark, s);
+    if (us != MOE_OK) return us;
+  } else {
+    // step 5 and the shared expert's up projection: both read x
+    DenseArgs g1{};
+    g1.A0 = hidden; g1.W0 = h->w_fc1; g1.K0 = D; g1.K1 = 0;
+    g1.out = h->z; g1.ldo = L; g1.M = T; g1.N = L; g1.epi = EPI_NONE;
+    g1.in_dt = dt; g1.out_dt = dt;
+    launch_dense(g1, s);
+    DenseArgs gs = g1;
+    gs.W0 = h->w_su; gs.out = h->h_sh; gs.ldo = Fs; gs.N = Fs; gs.epi = EPI_RELU2;
+    launch_dense(gs, s);
+    mark(MOE_STAGE_EXPERT_UP);
 
-  // step 6: routed experts in the latent space
-  GroupedArgs up{};
-  up.A = h->z; up.W = h->w_up; up.out = h->H; up.K = L; up.N = F; up.E = E; up.k = k;
-  up.offsets = h->offsets; up.perm = h->perm; up.tiles = h->tiles_up; up.gather = 1;
-  up.epi = EPI_RELU2; up.in_dt = dt; up.out_dt = dt; up.err = h->err;
-  launch_grouped(up, max_tiles(c, T, F), s);
-  mark(MOE_STAGE_EXPERT_DOWN);
-  GroupedArgs dn = up;
-  dn.A = h->H; dn.W = h->w_down; dn.out = h->Y; dn.K = F; dn.N = L; dn.perm = nullptr;
-  dn.tiles = h->tiles_dn; dn.gather = 0; dn.epi = EPI_NONE; dn.out_dt = MOE_FP32;
-  launch_grouped(dn, max_tiles(c, T, L), s);
-  mark(MOE_STAGE_COMBINE);
-  launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, dt, s);
-  mark(MOE_STAGE_DENSE_OUT);
+    // step 6: routed experts in the latent space
+    GroupedArgs up{};
+    up.A = h->z; up.W = h->w_up; up.out = h->H; up.K = L; up.N = F; up.E = E; up.k = k;
+    up.offsets = h->offsets; up.perm = h->perm; up.tiles = h->tiles_up; up.gather = 1;
+    up.epi = EPI_RELU2; up.in_dt = dt; up.out_dt = dt; up.err = h->err;
+    launch_grouped(up, max_tiles(c, T, F), s);
+    mark(MOE_STAGE_EXPERT_DOWN);
+    GroupedArgs dn = up;
+    dn.A = h->H; dn.W = h->w_down; dn.out = h->Y; dn.K = F; dn.N = L; dn.perm = nullptr;
+    dn.tiles = h->tiles_dn; dn.gather = 0; dn.epi = EPI_NONE; dn.out_dt = MOE_FP32;
+    launch_grouped(dn, max_tiles(c, T, L), s);
+    mark(MOE_STAGE_COMBINE);
+    launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, dt, s);
+    mark(MOE_STAGE_DENSE_OUT);
 
-  // step 7: fc2_latent_proj and the shared expert's down projection, one GEMM
-  DenseArgs g5{};
-  g5.A0 = h->zc; g5.W0 = h->w_fc2; g5.K0 = L;
-  g5.A1 = h->h_sh; g5.W1 = h->w_sd; g5.K1 = Fs;
-  g5.out = out; g5.ldo = D; g5.M = T; g5.N = D; g5.epi = EPI_NONE;
-  g5.in_dt = dt; g5.out_dt = c.out_dtype;
-  launch_dense(g5, s);
+    // step 7: fc2_latent_proj and the shared expert's down projection, one GEMM
+    DenseArgs g5{};
+    g5.A0 = h->zc; g5.W0 = h->w_fc2; g5.K0 = L;
+    g5.A1 = h->h_sh; g5.W1 = h->w_sd; g5.K1 = Fs;
+    g5.out = out; g5.ldo = D; g5.M = T; g5.N = D; g5.epi = EPI_NONE;
+    g5.in_dt = dt; g5.out_dt = c.out_dtype;
+    launch_dense(g5, s);
+  }
   mark(MOE_NUM_STAGES);
   h->prof_valid = h->prof;
   h->last_T = T;

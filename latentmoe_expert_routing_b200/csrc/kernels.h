@@ -77,3 +77,33 @@ namespace lmoe {
 // logits; rank / blkcnt are written for a caller that goes on to group pairs.
 void launch_route_select(const RouteArgs& a, cudaStream_t st);
 }  // namespace lmoe
+
+#include <cuda.h>
+namespace lmoe {
+// Tensor-core GEMM (umma_gemm.cu): out[a_row, n] = epi(sum_s A_s[a_row, :] . W_s[w_row, :])
+struct UmmaArgs {
+  int K0, K1;               // K of segment 0 and 1 (multiples of 64; K1 = 0: none)
+  int n_out;                // output columns = weight rows per group
+  int ldo;                  // output row stride (elements)
+  int w_group_rows;         // row offset between groups in the weight maps
+  int E;                    // groups (grouped mode)
+  const int32_t* offsets;   // [E+1] A-row offsets (grouped) or NULL (dense)
+  const int32_t* tiles;     // [E+1] tile offsets (grouped)
+  int M;                    // A rows (dense mode)
+  int dense_tiles;          // tile count (dense mode)
+  void* out;
+  int* err;
+};
+enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2 };
+struct UmmaLaunch {
+  CUtensorMap wmap0, amap0, wmap1, amap1;
+  UmmaArgs args;
+  int nt;                   // token rows per tile: 16, 64 or 256
+  UmmaEpi epi;
+  int max_tiles;            // upper bound of the tile count (grid clamp)
+};
+bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
+cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
+void launch_gather_rows(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
+                        cudaStream_t st);
+}  // namespace lmoe

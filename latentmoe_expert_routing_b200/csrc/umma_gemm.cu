@@ -1,0 +1,320 @@
+// Tensor-core (tcgen05 / TMEM / TMA) GEMMs of the LatentMoE layer, bf16 in,
+// fp32 accumulate.  One kernel serves every GEMM of the layer:
+//   grouped over experts: H = relu(z_perm U_e^T)^2, Y = H D_e^T   (report 5.6 step 6)
+//   dense:  z = x W_fc1^T, h_sh = relu(x W_su^T)^2,               (steps 5, 7)
+//           out = zc W_fc2^T + h_sh W_sd^T  (two K segments, one accumulator)
+//
+// Orientation: the MMA's M side is 128 weight rows (output columns) and its N
+// side is a tile of NT token rows ("swap AB"), so a decode step with a few
+// tokens per expert still fills the 128-row tensor-core tile and streams each
+// expert's weights exactly once.  Both operands are K-major, staged by TMA with
+// the 128-byte swizzle, 64 K-elements per pipeline stage.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring;
+// warp 1 allocates TMEM and one lane issues tcgen05.mma into one of two TMEM
+// accumulators; warps 2-5 drain the other accumulator (tcgen05.ld), apply the
+// epilogue and store.  Every wait is bounded: on timeout the kernel records
+// DEV_ERR_TIMEOUT, unwinds, waits for its own copies / MMAs and frees TMEM.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace lmoe {
+
+using namespace sm100;
+
+constexpr int kBM = 128;                  // weight rows per tile (MMA M)
+constexpr int kBK = 64;                   // K elements per stage (128 B of bf16)
+constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
+constexpr int kWTileBytes = kBM * kBK * 2;
+
+template <int NT, int STAGES>
+struct UmmaSmem {
+  static constexpr int kATileBytes = NT * kBK * 2;
+  static constexpr int kStageBytes = kWTileBytes + kATileBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
+};
+
+struct TileInfo {
+  int w_row0;      // first weight row (row of the weight tensor map)
+  int n0;          // first output column (weight row within the group)
+  int a_row0;      // first A row (token / pair) of the tile
+  int valid;       // A rows of the tile that belong to the group
+};
+
+template <int NT>
+__device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInfo& ti) {
+  const int nmb = (a.n_out + kBM - 1) / kBM;
+  int e = 0, base = 0, cnt = a.M, local = tile;
+  if (a.offsets) {
+    int lo = 0, hi = a.E;
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (a.tiles[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+    base = a.offsets[e];
+    cnt = a.offsets[e + 1] - base;
+    local = tile - a.tiles[e];
+  }
+  const int nnb = (cnt + NT - 1) / NT;
+  if (nnb == 0) return false;
+  const int mblk = local / nnb, nb = local - mblk * nnb;
+  if (mblk >= nmb) return false;
+  ti.n0 = mblk * kBM;
+  ti.w_row0 = e * a.w_group_rows + ti.n0;
+  ti.a_row0 = base + nb * NT;
+  ti.valid = min(NT, cnt - nb * NT);
+  return true;
+}
+
+__device__ __forceinline__ int total_tiles(const UmmaArgs& a) {
+  return a.offsets ? a.tiles[a.E] : a.dense_tiles;
+}
+
+template <typename TO>
+__device__ __forceinline__ void store_out(TO* p, float v) { store_val(p, v); }
+
+template <int NT, int STAGES, typename TO, bool RELU2>
+__global__ void __launch_bounds__(192, 1)
+umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
+                 const __grid_constant__ CUtensorMap amap0,
+                 const __grid_constant__ CUtensorMap wmap1,
+                 const __grid_constant__ CUtensorMap amap1, const UmmaArgs a) {
+  using S = UmmaSmem<NT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;       // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* mma_done = acc_empty + 2;        // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt0 = a.K0 / kBK, kt_all = kt0 + a.K1 / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&wmap0);
+    tma_prefetch_desc(&amap0);
+    if (a.K1 > 0) { tma_prefetch_desc(&wmap1); tma_prefetch_desc(&amap1); }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ntiles = total_tiles(a);
+
+  auto fail = [&](int where) {
+    atomicOr(a.err, DEV_ERR_TIMEOUT | (where << 8));
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        TileInfo ti;
+        if (!decode_tile<NT>(a, tile, ti)) continue;
+        for (int kt = 0; kt < kt_all; ++kt, ++it) {
+          const int s = it % STAGES;
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&empty[s], (round & 1) ^ 1)) { fail(1); break; }
+          if (*abort_flag) break;
+          uint8_t* st = smem + s * S::kStageBytes;
+          mbar_arrive_expect_tx(&full[s], S::kStageBytes);
+          const bool seg1 = kt >= kt0;
+          const int k0 = (seg1 ? kt - kt0 : kt) * kBK;
+          tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
+          tma_load_2d(st + kWTileBytes, seg1 ? &amap1 : &amap0, &full[s], k0, ti.a_row0);
+        }
+      }
+      // drain: every load this thread issued must land before the CTA exits
+      const uint32_t n = it < (uint32_t)STAGES ? it : (uint32_t)STAGES;
+      for (uint32_t j = 0; j < n; ++j) {
+        const uint32_t i = it - 1 - j;
+        if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1)) { fail(2); break; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, NT);
+      uint32_t it = 0, lt = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        TileInfo ti;
+        if (!decode_tile<NT>(a, tile, ti)) continue;
+        const uint32_t buf = lt & 1, use = lt >> 1;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(3); break; }
+        tc_fence_after();
+        const uint32_t d = tmem + buf * NT;
+        bool ok = true;
+        for (int kt = 0; kt < kt_all; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1)) { fail(4); ok = false; break; }
+          tc_fence_after();
+          const uint32_t wa = smem_u32(smem + s * S::kStageBytes);
+          const uint32_t aa = wa + kWTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+            mma_bf16_ss(d, sw128_desc(wa + kk * kUmmaK * 2), sw128_desc(aa + kk * kUmmaK * 2),
+                        idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);             // frees the stage when these MMAs finish
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+        ++lt;
+      }
+      mma_commit(mma_done);
+      if (!mbar_wait(mma_done, 0)) fail(5);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5 ----------------
+    const int q = warp & 3;                  // TMEM lane quarter this warp may read
+    TO* out = reinterpret_cast<TO*>(a.out);
+    uint32_t lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+      TileInfo ti;
+      if (!decode_tile<NT>(a, tile, ti)) continue;
+      const uint32_t buf = lt & 1, use = lt >> 1;
+      if (!mbar_wait(&acc_full[buf], use & 1)) { fail(6); break; }
+      tc_fence_after();
+      const int n = ti.n0 + 32 * q + lane;   // output column of this thread
+      const bool col_ok = n < a.n_out;
+#pragma unroll
+      for (int c = 0; c < NT / 8; ++c) {
+        uint32_t r[8];
+        tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, r);
+        tmem_ld_wait();
+        if (col_ok) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int row = c * 8 + j;
+            if (row < ti.valid) {
+              float v = __uint_as_float(r[j]);
+              if (RELU2) v = relu2(v);
+              store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      ++lt;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, S::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launches
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, K], box = box_rows x 64 elements, 128-B swizzle.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base || rows <= 0 || K <= 0 || (K % kBK) != 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int NT, int STAGES, typename TO, bool RELU2>
+static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
+  using S = UmmaSmem<NT, STAGES>;
+  auto kern = umma_gemm_kernel<NT, STAGES, TO, RELU2>;
+  static int configured = 0, sms = 0;
+  if (!configured) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    if (e != cudaSuccess) return e;
+    configured = 1;
+  }
+  int grid = L.max_tiles < sms ? L.max_tiles : sms;
+  if (grid < 1) grid = 1;
+  kern<<<grid, 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
+  return cudaGetLastError();
+}
+
+template <int NT, int STAGES>
+static cudaError_t umma_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
+  switch (L.epi) {
+    case UMMA_EPI_BF16: return umma_launch_t<NT, STAGES, __nv_bfloat16, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return umma_launch_t<NT, STAGES, __nv_bfloat16, true>(L, st);
+    case UMMA_EPI_F32: return umma_launch_t<NT, STAGES, float, false>(L, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st) {
+  switch (L.nt) {
+    case 16: return umma_launch_nt<16, 8>(L, st);
+    case 64: return umma_launch_nt<64, 8>(L, st);
+    case 256: return umma_launch_nt<256, 4>(L, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// z_perm[p, :] = z[perm[p] / k, :]  (16 bytes per thread)
+__global__ void gather_rows_kernel(const uint4* __restrict__ z, const int32_t* __restrict__ perm,
+                                   uint4* __restrict__ zp, long P, int k, int row_vecs) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= P * row_vecs) return;
+  const long p = i / row_vecs;
+  const int c = (int)(i - p * row_vecs);
+  zp[i] = z[(long)(perm[p] / k) * row_vecs + c];
+}
+
+void launch_gather_rows(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
+                        cudaStream_t st) {
+  const int rv = L * 2 / 16;
+  const long n = P * rv;
+  if (n == 0) return;
+  gather_rows_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)z, perm, (uint4*)zp, P, k, rv);
+}
+
+}  // namespace lmoe

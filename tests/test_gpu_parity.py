@@ -120,3 +120,20 @@ def test_host_entry_point_matches_device_entry_point(L):
     ih = torch.empty(TINY.T, TINY.k, dtype=torch.int32).pin_memory()
     lay.forward_host(xh, oh, ih)
     assert torch.equal(oh, out.cpu()) and torch.equal(ih, idx.cpu())
+
+
+@pytest.mark.parametrize("T", [1, 3, 64, 129, 300])
+def test_tiny_bf16_tensor_core_path(L, T):
+    """bf16 layers run on the tcgen05 GEMMs; T spans 16-, 64- and 256-row
+    token tiles and ragged tails."""
+    cfg = TINY.replace(dtype="bf16")
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    _assert_out(g[0], r["out"])
+
+
+def test_bf16_wide_tiles_and_many_experts(L):
+    cfg = TINY.replace(dtype="bf16", E=64, k=8, D=512, L=128, F=256, Fs=384, T=700)
+    lay, g, r = _run_full(L, cfg)
+    _assert_routing_exact(g, r)
+    _assert_out(g[0], r["out"])
