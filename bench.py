@@ -251,6 +251,9 @@ def run_ours(a):
     stage_ms = {k: statistics.median(s[k] for s in stages) for k in stages[0]}
     counts, _, _, _ = lay.routing(T)
     n_touched = int((counts > 0).sum().item())
+    lay.router_stats()
+    step()
+    exact_per_token = lay.router_stats() / T
 
     # end to end through the host entry point: pinned H2D of x, D2H of out
     xh = x.cpu().pin_memory()
@@ -317,6 +320,7 @@ def run_ours(a):
             "roofline": roof,
             "stages_ms": stage_ms,
             "experts_touched": n_touched,
+            "router_exact_logits_per_token": exact_per_token,
             "expert_weight_gbs": 2 * _expert_bytes(cfg, n_touched) /
                                  ((stage_ms["expert_up"] + stage_ms["expert_down"]) * 1e-3) / 1e9,
             "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,

@@ -178,6 +178,15 @@ moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
                              moe_dtype dtype, int32_t* topk_idx, float* topk_w,
                              void* stream);
 
+/* Router statistics since the last call (then reset), synchronous on `stream`:
+ * *exact_logits = number of (token, expert) logits the bf16 router recomputed
+ * in the defined fixed-order fp64 form.  bf16 layers compute all logits on the
+ * tensor cores and recompute exactly only the experts that a worst-case error
+ * bound cannot place clearly inside or outside the top-k (and every selected
+ * expert); fp32 layers evaluate every logit exactly and report 0. */
+moe_status moe_get_router_stats(moe_handle* handle, unsigned long long* exact_logits,
+                                void* stream);
+
 /* Drain `stream` and report (then clear) the device error word. */
 moe_status moe_sync(moe_handle* handle, void* stream);
 

@@ -58,6 +58,7 @@ SIGNATURES = [
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
     ("moe_route_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i,
                                _vp, _vp, _vp]),
+    ("moe_get_router_stats", _i, [_vp, _p(ctypes.c_ulonglong), _vp]),
     ("moe_sync", _i, [_vp, _vp]),
     ("moe_destroy", None, [_vp]),
     ("moe_status_string", ctypes.c_char_p, [_i]),
@@ -133,6 +134,12 @@ def moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts, top_k, r
     _check(_lib.moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts,
                                   top_k, rsf, dtype, topk_idx, topk_w, stream),
            "moe_route_noalloc")
+
+
+def moe_get_router_stats(h, stream) -> int:
+    v = ctypes.c_ulonglong(0)
+    _check(_lib.moe_get_router_stats(h, ctypes.byref(v), stream), "moe_get_router_stats")
+    return v.value
 
 
 def moe_sync(h, stream):

@@ -32,7 +32,10 @@ struct moe_handle {
   int last_T = 0;
   // tensor-core path (bf16): permuted latent rows and cached TMA maps
   void* z_perm = nullptr;
-  CUtensorMap wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
+  float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
+  uint32_t* cmask = nullptr;                     // [T, 32] candidate bits per token
+  unsigned long long* stats = nullptr;           // exactly recomputed logits
+  CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
   CUtensorMap am_zp[3], am_H[3], am_zc[3], am_hsh[3];   // token boxes of 16, 64, 256 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
   cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
@@ -88,7 +91,7 @@ int max_tiles(const moe_config& c, int T, int N) {
 // up / down, combine, G5 (fc2 + shared down) -- all tcgen05 GEMMs but the gather
 // and the combine.
 template <typename Mark>
-moe_status forward_umma(moe_handle* h, const void* hidden, int T, void* out,
+moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out,
                         const float* wts, Mark& mark, cudaStream_t s) {
   const moe_config& c = h->cfg;
   const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
@@ -104,7 +107,7 @@ moe_status forward_umma(moe_handle* h, const void* hidden, int T, void* out,
   g.args.M = T;
   g.nt = ntd;
   // step 5: z = x W_fc1^T, and the shared expert's up projection (both read x)
-  if (!make_tmap_bf16(&g.amap0, hidden, T, D, ntd)) return MOE_ERR_CUDA;
+  g.amap0 = xmap;
   g.wmap0 = h->wm_fc1;
   g.args.K0 = D; g.args.K1 = 0; g.args.n_out = L; g.args.ldo = L;
   g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
@@ -236,8 +239,16 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
       moe_destroy(h);
       return MOE_ERR_UNSUPPORTED;
     }
-    if (!dev_alloc(h, &h->z_perm, P * L * 2)) { moe_destroy(h); return MOE_ERR_OOM; }
-    bool m = make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
+    if (!dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
+        !dev_alloc(h, &h->cmask, T * 32 * 4) ||
+        !dev_alloc(h, &h->stats, 16)) {
+      moe_destroy(h);
+      return MOE_ERR_OOM;
+    }
+    launch_row_norms(h->w_gate, (int)E, (int)D, h->wnorm, s);
+    cudaMemsetAsync(h->stats, 0, 16, s);
+    bool m = make_tmap_bf16(&h->wm_gate, h->w_gate, E, D, 128) &&
+             make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
              make_tmap_bf16(&h->wm_su, h->w_su, Fs, D, 128) &&
              make_tmap_bf16(&h->wm_up, h->w_up, E * F, L, 128) &&
              make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128) &&
@@ -278,7 +289,20 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   mark(MOE_STAGE_ROUTER_LOGITS);
 
   // steps 1-4: logits, sigmoid, biased selection, weights; step 6 bookkeeping
-  launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
+  CUtensorMap xmap;
+  if (dt == MOE_BF16) {
+    // tensor-core logits; the certified selection below makes them exact
+    if (!make_tmap_bf16(&xmap, hidden, T, D, kNT[nt_index(T)])) return MOE_ERR_CUDA;
+    UmmaLaunch g{};
+    g.wmap0 = h->wm_gate; g.amap0 = xmap; g.nt = kNT[nt_index(T)];
+    g.args.err = h->err; g.args.E = 1; g.args.M = T;
+    g.args.K0 = D; g.args.n_out = E; g.args.ldo = E;
+    g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt);
+    g.args.out = h->logits; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
+    if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
+  }
   mark(MOE_STAGE_ROUTE);
   RouteArgs ra{};
   ra.logits = h->logits; ra.bias = h->bias; ra.T = T; ra.E = E; ra.k = k;
@@ -295,11 +319,18 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   }
   ra.tiles_up = h->tiles_up; ra.tiles_dn = h->tiles_dn;
   ra.err = h->err;
-  launch_route(ra, s);
+  ra.cmask = dt == MOE_BF16 ? h->cmask : nullptr;
+  if (dt == MOE_BF16) {
+    CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
+                h->stats};
+    launch_route_certified(ra, ca, s);
+  } else {
+    launch_route(ra, s);
+  }
   mark(MOE_STAGE_DENSE_IN);
 
   if (dt == MOE_BF16) {
-    moe_status us = forward_umma(h, hidden, T, out, wts, mark, s);
+    moe_status us = forward_umma(h, xmap, T, out, wts, mark, s);
     if (us != MOE_OK) return us;
   } else {
     // step 5 and the shared expert's up projection: both read x
@@ -404,6 +435,19 @@ moe_status moe_profile_read(moe_handle* h, float* stage_ms, int n) {
   for (int i = 0; i < n && i < MOE_NUM_STAGES; ++i)
     if (cudaEventElapsedTime(&stage_ms[i], h->ev[i], h->ev[i + 1]) != cudaSuccess)
       return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_get_router_stats(moe_handle* h, unsigned long long* exact_logits, void* stream) {
+  if (!h || !exact_logits) return MOE_ERR_INVALID_ARG;
+  *exact_logits = 0;
+  if (!h->stats) return MOE_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(exact_logits, h->stats, sizeof(unsigned long long),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemsetAsync(h->stats, 0, sizeof(unsigned long long), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

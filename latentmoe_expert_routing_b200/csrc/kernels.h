@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cuda_bf16.h>
+
 #include "latentmoe.h"
 
 namespace lmoe {
@@ -27,11 +29,23 @@ struct RouteArgs {
   int mt_dn, nc_dn;
   int32_t* tiles_dn;    // [E + 1]
   int* err;
+  uint32_t* cmask;           // [T, ceil(E/32)] candidate bits (certified router) or NULL
 };
 
 void launch_router_logits(const void* x, const void* wg, float* logits, int T,
                           int D, int E, moe_dtype dt, cudaStream_t st);
 void launch_route(const RouteArgs& a, cudaStream_t st);
+
+// Certified selection from tensor-core logits (RouteArgs::logits = fast logits)
+struct CertArgs {
+  const __nv_bfloat16* x;   // [T, D] hidden rows
+  const __nv_bfloat16* wg;  // [E, D] gate weight
+  const float* wnorm;       // [E] ||w_e||_2 rounded up
+  int D;
+  unsigned long long* stats;  // += number of exactly recomputed logits (or NULL)
+};
+void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
+void launch_row_norms(const void* w, int rows, int D, float* out, cudaStream_t st);
 
 // Row-streaming GEMMs:  out[m, n] = epi( sum_s sum_k A_s[m, k] * W_s[n, k] ).
 constexpr int kRowsPerWarp = 4;                  // weight rows per warp

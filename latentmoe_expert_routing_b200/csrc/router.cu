@@ -104,7 +104,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              int n_tok, int E, int k, float rsf,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
              int32_t* __restrict__ rank, int32_t* __restrict__ blkcnt, int nblk,
-             int* __restrict__ err) {
+             int* __restrict__ err, const uint32_t* __restrict__ cmask) {
   extern __shared__ uint32_t mask[];                 // [E]
   __shared__ float rsel[32][kMaxTopK];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -116,7 +116,10 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      if (e < E) {
+      // cmask (optional): only these experts can be in the top-k; their
+      // logits have been recomputed exactly
+      const bool cand = cmask == nullptr || ((cmask[(size_t)t * EPL + i] >> lane) & 1u);
+      if (e < E && cand) {
         s[i] = sigmoid_fixed(logits[(size_t)t * E + e]);
         c[i] = __fadd_rn(s[i], bias[e]);
       } else {
@@ -131,7 +134,8 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !(taken >> i & 1u) && (bi < 0 || ranks_above(c[i], e, bc, be))) {
+        if (e < E && c[i] != -INFINITY && !(taken >> i & 1u) &&
+            (bi < 0 || ranks_above(c[i], e, bc, be))) {
           bc = c[i]; be = e; bi = i;
         }
       }
@@ -286,7 +290,7 @@ template <int EPL>
 static void route_launch_epl(const RouteArgs& a, cudaStream_t st) {
   route_kernel<EPL><<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(
       a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w, a.rank,
-      a.blkcnt, a.nblk, a.err);
+      a.blkcnt, a.nblk, a.err, a.cmask);
 }
 
 void launch_route_select(const RouteArgs& a, cudaStream_t st) {
@@ -307,6 +311,179 @@ void launch_route(const RouteArgs& a, cudaStream_t st) {
   else if (epl <= 8) route_launch_epl<8>(a, st);
   else if (epl <= 16) route_launch_epl<16>(a, st);
   else route_launch_epl<32>(a, st);
+  route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
+                                        a.offsets, a.mt_up, a.nc_up, a.tiles_up,
+                                        a.mt_dn, a.nc_dn, a.tiles_dn);
+  const long P = (long)a.T * a.k;
+  route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
+      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+}
+
+}  // namespace lmoe
+
+namespace lmoe {
+
+// ---------------------------------------------------------------------------
+// Certified selection from tensor-core logits (bf16 layers).
+//
+// l~ (fp32 tensor-core accumulation of exact bf16 products) differs from the
+// defined logit l by at most Delta = g * ||x_t|| * ||w_e||, g = margin * K * 2^-23
+// / (1 - K * 2^-23): the worst-case bound of K-term floating-point summation
+// with unit roundoff 2^-23 (covers truncating adders) and Cauchy-Schwarz for
+// sum |x_k w_k|, times a safety margin.  The sigmoid has slope <= 1/4, so the
+// choice score c = s + bias lies within d_e = Delta/4 + eps of c~.  With
+// tau = the k-th largest lower bound c~ - d, every expert whose upper bound
+// c~ + d is below tau is beaten for sure by k others, so the true top-k lies in
+// C = { e : c~_e + d_e >= tau }.  The kernel recomputes the defined logit
+// (fixed-order fp64) for every e in C and selects among C exactly, giving the
+// same indices and weights as evaluating every expert exactly.
+// ---------------------------------------------------------------------------
+constexpr double kCertMargin = 2.0;
+constexpr double kCertEps = 0x1p-19;     // sigmoid/add rounding of c~, generous
+
+// Defined logit of (x row, w row): lane p sums partial p, shfl_down tree.
+__device__ __forceinline__ float exact_logit_warp(const __nv_bfloat16* __restrict__ xr,
+                                                  const __nv_bfloat16* __restrict__ wr,
+                                                  int D, int lane) {
+  double acc = 0.0;
+  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
+    float xv[8], wv[8];
+    load8(xr + k0, xv);
+    load8(wr + k0, wv);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc = fma((double)xv[r], (double)wv[r], acc);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+  return __double2float_rn(__shfl_sync(0xffffffffu, acc, 0));
+}
+
+// Bounds and candidates: one warp per token; lane l handles experts l+32i.
+// Writes cmask[t][i] bit l = expert l+32i is a candidate.
+template <int EPL>
+__global__ void __launch_bounds__(256)
+route_bounds_kernel(RouteArgs a, CertArgs ca) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int E = a.E, k = a.k, D = ca.D;
+  if (t >= a.T) return;
+  const __nv_bfloat16* xr = ca.x + (size_t)t * D;
+  float ss = 0.f;                                   // ||x_t||^2, inflated below
+  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
+    float xv[8];
+    load8(xr + k0, xv);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) ss = fmaf(xv[r], xv[r], ss);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const double u = 0x1p-23, Ku = D * u;
+  const double g = kCertMargin * Ku / (1.0 - Ku);
+  const double dscale = 0.25 * g * sqrt((double)ss) * (1.0 + 0x1p-10);
+  double c[EPL], d[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      c[i] = (double)__fadd_rn(sigmoid_fixed(a.logits[(size_t)t * E + e]), a.bias[e]);
+      d[i] = dscale * ca.wnorm[e] + kCertEps;
+    } else {
+      c[i] = -INFINITY;
+      d[i] = 0.0;
+    }
+  }
+  // tau = k-th largest lower bound c~ - d
+  uint32_t taken = 0u;
+  double tau = -INFINITY;
+  for (int j = 0; j < k; ++j) {
+    double best = -INFINITY;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !(taken >> i & 1u) && (bi < 0 || c[i] - d[i] > best)) {
+        best = c[i] - d[i];
+        bi = i;
+      }
+    }
+    double wv = best;
+    int wl = bi >= 0 ? lane : 32;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, wv, off);
+      const int ol = __shfl_xor_sync(0xffffffffu, wl, off);
+      if (ol < 32 && (wl == 32 || ov > wv || (ov == wv && ol < wl))) { wv = ov; wl = ol; }
+    }
+    const int wbi = __shfl_sync(0xffffffffu, bi, wl & 31);
+    if (lane == wl) taken |= 1u << wbi;
+    tau = wv;
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    const uint32_t b = __ballot_sync(0xffffffffu, e < E && c[i] + d[i] >= tau);
+    if (lane == 0) a.cmask[(size_t)t * EPL + i] = b;
+  }
+}
+
+// Exact logits of the candidates: one warp per (token, 32-expert word); the
+// defined fixed-order fp64 value overwrites the tensor-core logit in place.
+template <int EPL>
+__global__ void __launch_bounds__(256)
+route_exact_kernel(RouteArgs a, CertArgs ca) {
+  const int lane = threadIdx.x & 31;
+  const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (w >= (long)a.T * EPL) return;
+  const int t = (int)(w / EPL), i = (int)(w - (long)t * EPL);
+  uint32_t b = a.cmask[w];
+  if (lane == 0 && ca.stats && b) atomicAdd(ca.stats, (unsigned long long)__popc(b));
+  const __nv_bfloat16* xr = ca.x + (size_t)t * ca.D;
+  while (b) {
+    const int src = __ffs(b) - 1;
+    b &= b - 1;
+    const int e = src + 32 * i;
+    const float l = exact_logit_warp(xr, ca.wg + (size_t)e * ca.D, ca.D, lane);
+    if (lane == 0) const_cast<float*>(a.logits)[(size_t)t * a.E + e] = l;   // workspace
+  }
+}
+
+// ||w_e||_2 of each gate row, fp64 sum of squares, rounded up to fp32.
+__global__ void row_norms_kernel(const __nv_bfloat16* __restrict__ w, int rows, int D,
+                                 float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  double ss = 0.0;
+  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
+    float v[8];
+    load8(w + (size_t)r * D + k0, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) out[r] = __double2float_ru(sqrt(ss) * (1.0 + 0x1p-20));
+}
+
+void launch_row_norms(const void* w, int rows, int D, float* out, cudaStream_t st) {
+  row_norms_kernel<<<ceil_div(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)w, rows, D, out);
+}
+
+template <int EPL>
+static void route_cert_epl(const RouteArgs& a, const CertArgs& c, cudaStream_t st) {
+  route_bounds_kernel<EPL><<<ceil_div(a.T, 8), 256, 0, st>>>(a, c);
+  route_exact_kernel<EPL><<<ceil_div((long)a.T * EPL, 8), 256, 0, st>>>(a, c);
+  route_launch_epl<EPL>(a, st);
+}
+
+void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t st) {
+  const int epl = (a.E + 31) / 32;
+  if (epl <= 1) route_cert_epl<1>(a, c, st);
+  else if (epl <= 2) route_cert_epl<2>(a, c, st);
+  else if (epl <= 4) route_cert_epl<4>(a, c, st);
+  else if (epl <= 8) route_cert_epl<8>(a, c, st);
+  else if (epl <= 16) route_cert_epl<16>(a, c, st);
+  else route_cert_epl<32>(a, c, st);
   route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
                                         a.offsets, a.mt_up, a.nc_up, a.tiles_up,
                                         a.mt_dn, a.nc_dn, a.tiles_dn);

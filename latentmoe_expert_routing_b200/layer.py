@@ -83,6 +83,10 @@ class LatentMoE:
                           perm.data_ptr(), pos.data_ptr(), self.stream)
         return counts, offsets, perm[:T * k], pos[:T * k]
 
+    def router_stats(self) -> int:
+        """Exactly recomputed (token, expert) logits since the last call."""
+        return B.moe_get_router_stats(self.handle, self.stream)
+
     def sync(self):
         B.moe_sync(self.handle, self.stream)
 

@@ -42,6 +42,8 @@ def _check(cfg, ultra, sample_route, sample_out):
     counts, offsets, perm, pos = lay.routing(cfg.T)
     lay.sync()
     idx_h, w_h = idx.cpu().numpy(), np32(w)
+    exact = lay.router_stats()           # certified router: every selected + band
+    assert cfg.T * cfg.k <= exact <= cfg.T * cfg.E
     check_dispatch_properties(idx_h, counts.cpu().numpy(), offsets.cpu().numpy(),
                               perm.cpu().numpy(), pos.cpu().numpy(), cfg.E)
     rows = sample_route
