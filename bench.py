@@ -107,7 +107,10 @@ def _dist():
 
 
 def _expert_bytes(cfg, n_touched):
-    """Bytes of one expert matrix set actually streamed: dense bf16/fp32."""
+    """Bytes of one expert matrix per touched expert actually streamed: dense
+    bf16/fp32, or NVFP4 (4-bit codes + one E4M3 scale per 16 = 0.5625 B)."""
+    if cfg.expert_fmt != "dense":
+        return n_touched * cfg.F * cfg.L * 9 // 16
     es = 4 if cfg.dtype == "fp32" else 2
     return n_touched * cfg.F * cfg.L * es
 

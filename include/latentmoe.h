@@ -178,6 +178,20 @@ moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
                              moe_dtype dtype, int32_t* topk_idx, float* topk_w,
                              void* stream);
 
+/* NVFP4 quantisation (report section 8.1; NVFP4 format details) of n_mat
+ * row-major matrices w [n_mat, rows, K] (device, dtype), in 16-element blocks
+ * along K:
+ *   gscale[m]        = amax(w[m]) / (6 * 448)                      fp32
+ *   scales[m, r, b]  = E4M3(amax(block) / (6 * gscale[m]))  RNE, satfinite at 448
+ *   codes            = E2M1(w / (value(scale) * gscale[m])) RNE ties-to-even, sat. at 6
+ * with fp32 arithmetic before each encoding.  Outputs (device): codes
+ * [n_mat, rows, K/2] two per byte, the even element in the low nibble;
+ * scales [n_mat, rows, K/16]; gscale [n_mat].  K must be a multiple of 16.
+ * Uses a small temporary device buffer; synchronises `stream`.  moe_init runs
+ * the same quantiser on the experts of NVFP4 layers. */
+moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int rows, int K,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* stream);
+
 /* Router statistics since the last call (then reset), synchronous on `stream`:
  * *exact_logits = number of (token, expert) logits the bf16 router recomputed
  * in the defined fixed-order fp64 form.  bf16 layers compute all logits on the

@@ -58,6 +58,7 @@ SIGNATURES = [
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
     ("moe_route_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i,
                                _vp, _vp, _vp]),
+    ("moe_quantize_nvfp4", _i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     ("moe_get_router_stats", _i, [_vp, _p(ctypes.c_ulonglong), _vp]),
     ("moe_sync", _i, [_vp, _vp]),
     ("moe_destroy", None, [_vp]),
@@ -134,6 +135,11 @@ def moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts, top_k, r
     _check(_lib.moe_route_noalloc(hidden, w_gate, gate_bias, T, d_model, n_experts,
                                   top_k, rsf, dtype, topk_idx, topk_w, stream),
            "moe_route_noalloc")
+
+
+def moe_quantize_nvfp4(w, dtype, n_mat, rows, K, codes, scales, gscale, stream):
+    _check(_lib.moe_quantize_nvfp4(w, dtype, n_mat, rows, K, codes, scales, gscale, stream),
+           "moe_quantize_nvfp4")
 
 
 def moe_get_router_stats(h, stream) -> int:

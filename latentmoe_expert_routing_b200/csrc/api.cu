@@ -34,6 +34,9 @@ struct moe_handle {
   void* z_perm = nullptr;
   float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
   uint32_t* cmask = nullptr;                     // [T, 32] candidate bits per token
+  // NVFP4 experts: GEMM-layout records and per-expert global scales
+  uint8_t *rec_up = nullptr, *rec_dn = nullptr;
+  float *gs_up = nullptr, *gs_dn = nullptr;
   unsigned long long* stats = nullptr;           // exactly recomputed logits
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
   CUtensorMap am_zp[3], am_H[3], am_zc[3], am_hsh[3];   // token boxes of 16, 64, 256 rows
@@ -75,7 +78,10 @@ moe_status validate(const moe_config* c) {
   if (c->out_dtype != MOE_FP32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c->n_group != 1 || c->topk_group != 1) return MOE_ERR_UNSUPPORTED;
   if (c->n_experts > 1024 || c->top_k > 64) return MOE_ERR_UNSUPPORTED;
-  if (c->expert_fmt != MOE_EXPERT_DENSE) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_fmt != MOE_EXPERT_DENSE && c->expert_fmt != MOE_EXPERT_NVFP4_W4A16 &&
+      c->expert_fmt != MOE_EXPERT_NVFP4_W4A4)
+    return MOE_ERR_INVALID_ARG;
+  if (c->expert_fmt != MOE_EXPERT_DENSE && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
@@ -85,6 +91,36 @@ int max_tiles(const moe_config& c, int T, int N) {
   long P = (long)T * c.top_k;
   long t = (P / kMT + c.n_experts) * (long)ceil_div(N, kChunk);
   return t > 0x7fffffff ? 0x7fffffff : (int)t;
+}
+
+// NVFP4 experts: quantise up [E,F,L] and down [E,L,F] (plain layout, in
+// temporary buffers), then repack into the GEMM records the kernel streams.
+moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
+  const moe_config& c = h->cfg;
+  const size_t E = c.n_experts, F = c.d_ff, L = c.d_latent;
+  const size_t recs_up = E * ((F + 127) / 128) * (L / 64), recs_dn = E * ((L + 127) / 128) * (F / 64);
+  if (!dev_alloc(h, &h->rec_up, recs_up * 4608) || !dev_alloc(h, &h->rec_dn, recs_dn * 4608) ||
+      !dev_alloc(h, &h->gs_up, E * 4) || !dev_alloc(h, &h->gs_dn, E * 4))
+    return MOE_ERR_OOM;
+  uint8_t *codes = nullptr, *scales = nullptr;
+  unsigned* amax = nullptr;
+  const size_t n = E * F * L;
+  if (cudaMalloc(&codes, n / 2) != cudaSuccess || cudaMalloc(&scales, n / 16) != cudaSuccess ||
+      cudaMalloc(&amax, E * 4) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(codes); cudaFree(scales); cudaFree(amax);
+    return MOE_ERR_OOM;
+  }
+  cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, codes, scales,
+                                        h->gs_up, amax, s);
+  if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)F, (int)L, h->rec_up, s);
+  if (e == cudaSuccess)
+    e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, codes, scales, h->gs_dn,
+                              amax, s);
+  if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFree(codes); cudaFree(scales); cudaFree(amax);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // Tensor-core path for bf16 layers: G1 (fc1, shared up), row gather, grouped
@@ -111,7 +147,10 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   g.wmap0 = h->wm_fc1;
   g.args.K0 = D; g.args.K1 = 0; g.args.n_out = L; g.args.ldo = L;
   g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
-  g.args.out = h->z; g.epi = UMMA_EPI_BF16; g.max_tiles = g.args.dense_tiles;
+  const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
+  const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
+  g.args.out = h->z; g.epi = w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
+  g.max_tiles = g.args.dense_tiles;
   if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
   g.wmap0 = h->wm_su;
   g.args.n_out = Fs; g.args.ldo = Fs;
@@ -128,13 +167,16 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   u.nt = ntg;
   u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
-  u.args.tiles = h->tiles_up; u.args.out = h->H; u.epi = UMMA_EPI_BF16_RELU2;
+  u.args.tiles = h->tiles_up; u.args.out = h->H;
+  u.epi = w4a4 ? UMMA_EPI_BF16_RELU2_Q : UMMA_EPI_BF16_RELU2;
+  if (wq) { u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up; }
   u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
   if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_EXPERT_DOWN);
   u.wmap0 = h->wm_dn; u.amap0 = h->am_H[gi];
   u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
   u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
+  if (wq) { u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn; }
   u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
   if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_COMBINE);
@@ -260,6 +302,10 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
           make_tmap_bf16(&h->am_zc[i], h->zc, T, L, kNT[i]) &&
           make_tmap_bf16(&h->am_hsh[i], h->h_sh, T, Fs, kNT[i]);
     if (!m) { moe_destroy(h); return MOE_ERR_CUDA; }
+    if (c.expert_fmt != MOE_EXPERT_DENSE) {
+      moe_status q = quantize_experts(h, s);
+      if (q != MOE_OK) { moe_destroy(h); return q; }
+    }
   }
   if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess) {
@@ -436,6 +482,20 @@ moe_status moe_profile_read(moe_handle* h, float* stage_ms, int n) {
     if (cudaEventElapsedTime(&stage_ms[i], h->ev[i], h->ev[i + 1]) != cudaSuccess)
       return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int rows, int K,
+                              uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
+  if (!w || !codes || !scales || !gscale || n_mat <= 0 || rows <= 0 || K <= 0 || K % 16)
+    return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_BF16 && dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned* amax = nullptr;
+  if (cudaMalloc(&amax, (size_t)n_mat * 4) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_OOM; }
+  cudaError_t e = launch_quantize_nvfp4(w, dtype, n_mat, rows, K, codes, scales, gscale, amax, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFree(amax);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_get_router_stats(moe_handle* h, unsigned long long* exact_logits, void* stream) {

@@ -107,8 +107,13 @@ struct UmmaArgs {
   int dense_tiles;          // tile count (dense mode)
   void* out;
   int* err;
+  const uint8_t* wq;        // NVFP4 weight records (GEMM layout) or NULL: weights via wmap0
+  int wq_mblks;             // 128-row blocks per weight matrix (NVFP4)
+  const float* gscale;      // [E] per-group output scale (NVFP4 global scale) or NULL
 };
-enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2 };
+// epilogues; _Q variants round the output through NVFP4 in 16-column blocks
+enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2,
+               UMMA_EPI_BF16_Q = 3, UMMA_EPI_BF16_RELU2_Q = 4 };
 struct UmmaLaunch {
   CUtensorMap wmap0, amap0, wmap1, amap1;
   UmmaArgs args;
@@ -118,6 +123,11 @@ struct UmmaLaunch {
 };
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
+cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
+                                  uint8_t* codes, uint8_t* scales, float* gscale,
+                                  unsigned* amax_tmp, cudaStream_t st);
+cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
+                               int K, uint8_t* out, cudaStream_t st);
 void launch_gather_rows(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
                         cudaStream_t st);
 }  // namespace lmoe

@@ -1,0 +1,122 @@
+// NVFP4 weight quantiser (report section 8.1; NVFP4 format details): one FP32
+// global scale per matrix s_g = amax / (6 * 448), one E4M3 scale per 16
+// consecutive elements along K s_b = E4M3(amax_b / (6 s_g)), elements
+// q = E2M1(w / (value(s_b) * s_g)); all arithmetic before the encodings in fp32.
+//
+// Plain layout (C ABI): codes [n_mat, rows, K/2] (two per byte, even element in
+// the low nibble), scales [n_mat, rows, K/16], gscale [n_mat].
+// GEMM layout (library internal): per (matrix, 128-row block, 64-K stage) one
+// contiguous 4608-byte record: 128 rows x 32 code bytes, then 128 rows x 4
+// scale bytes; rows past the matrix are zero.
+#include "common.cuh"
+#include "kernels.h"
+#include "nvfp4.cuh"
+
+namespace lmoe {
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+
+// amax of each matrix (non-negative floats order like their bit patterns)
+template <typename T>
+__global__ void matrix_amax_kernel(const T* __restrict__ w, long per_mat, unsigned* __restrict__ amax) {
+  const int m = blockIdx.y;
+  const T* p = w + (size_t)m * per_mat;
+  float a = 0.f;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < per_mat; i += (long)gridDim.x * blockDim.x)
+    a = fmaxf(a, fabsf(to_f(p[i])));
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(&amax[m], __float_as_uint(a));
+}
+
+__global__ void global_scale_kernel(const unsigned* __restrict__ amax, float* __restrict__ gscale, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) gscale[i] = __fdiv_rn(__uint_as_float(amax[i]), 2688.0f);   // 6 * 448
+}
+
+// One thread per 16-element block.
+template <typename T>
+__global__ void quantize_blocks_kernel(const T* __restrict__ w, int n_mat, int rows, int K,
+                                       const float* __restrict__ gscale,
+                                       uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const long nb = (long)n_mat * rows * (K / 16);
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= nb) return;
+  const int m = (int)(b / ((long)rows * (K / 16)));
+  const float sg = gscale[m];
+  const T* p = w + b * 16;
+  float v[16], amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) { v[i] = to_f(p[i]); amax = fmaxf(amax, fabsf(v[i])); }
+  const float den = __fmul_rn(6.0f, sg);
+  const float ratio = den > 0.f ? __fdiv_rn(amax, den) : 0.f;
+  const uint32_t sb = e4m3_encode_pos(ratio);
+  const float scale = __fmul_rn(e4m3_value(sb), sg);
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = scale > 0.f ? e2m1_encode(__fdiv_rn(v[i], scale)) : 0u;
+    if (i < 8) lo |= q << (4 * i); else hi |= q << (4 * (i - 8));
+  }
+  *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
+  scales[b] = (uint8_t)sb;
+}
+
+// plain layout -> GEMM layout
+__global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                   int n_mat, int rows, int K, uint8_t* __restrict__ out) {
+  const int nmb = (rows + 127) / 128, nks = K / 64;
+  const long rec = (long)blockIdx.x;                 // one record per block, 128 threads = rows
+  if (rec >= (long)n_mat * nmb * nks) return;
+  const int ks = (int)(rec % nks);
+  const int mb = (int)((rec / nks) % nmb);
+  const int m = (int)(rec / ((long)nks * nmb));
+  const int r = threadIdx.x;
+  const int row = mb * 128 + r;
+  uint8_t* o = out + rec * 4608;
+  uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+  uint32_t s = 0;
+  if (row < rows) {
+    const uint8_t* cp = codes + ((size_t)m * rows + row) * (K / 2) + ks * 32;
+    c0 = *reinterpret_cast<const uint4*>(cp);
+    c1 = *reinterpret_cast<const uint4*>(cp + 16);
+    s = *reinterpret_cast<const uint32_t*>(scales + ((size_t)m * rows + row) * (K / 16) + ks * 4);
+  }
+  reinterpret_cast<uint4*>(o + r * 32)[0] = c0;
+  reinterpret_cast<uint4*>(o + r * 32)[1] = c1;
+  reinterpret_cast<uint32_t*>(o + 4096)[r] = s;
+}
+
+cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
+                                  uint8_t* codes, uint8_t* scales, float* gscale,
+                                  unsigned* amax_tmp, cudaStream_t st) {
+  const long per_mat = (long)rows * K;
+  cudaError_t e = cudaMemsetAsync(amax_tmp, 0, sizeof(unsigned) * n_mat, st);
+  if (e != cudaSuccess) return e;
+  dim3 g1(ceil_div(per_mat, 256 * 16) < 1024 ? ceil_div(per_mat, 256 * 16) : 1024, n_mat);
+  const long nb = (long)n_mat * rows * (K / 16);
+  if (dt == MOE_BF16) {
+    matrix_amax_kernel<<<g1, 256, 0, st>>>((const __nv_bfloat16*)w, per_mat, amax_tmp);
+    global_scale_kernel<<<ceil_div(n_mat, 256), 256, 0, st>>>(amax_tmp, gscale, n_mat);
+    quantize_blocks_kernel<<<ceil_div(nb, 256), 256, 0, st>>>((const __nv_bfloat16*)w, n_mat, rows, K,
+                                                              gscale, codes, scales);
+  } else {
+    matrix_amax_kernel<<<g1, 256, 0, st>>>((const float*)w, per_mat, amax_tmp);
+    global_scale_kernel<<<ceil_div(n_mat, 256), 256, 0, st>>>(amax_tmp, gscale, n_mat);
+    quantize_blocks_kernel<<<ceil_div(nb, 256), 256, 0, st>>>((const float*)w, n_mat, rows, K,
+                                                              gscale, codes, scales);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
+                               int K, uint8_t* out, cudaStream_t st) {
+  const long recs = (long)n_mat * ((rows + 127) / 128) * (K / 64);
+  repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, out);
+  return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -1,0 +1,53 @@
+// NVFP4 encoders and decoders shared by the quantiser and the GEMM kernels
+// (report section 8.1 / NVFP4 format details: E2M1 elements, E4M3 block
+// scales).  Round to nearest, ties to the even code, saturating; written as
+// plain comparisons and integer arithmetic so every device gives the same codes.
+#pragma once
+#include <stdint.h>
+
+namespace lmoe {
+
+// |y| -> E2M1 magnitude code 0..7 (0, .5, 1, 1.5, 2, 3, 4, 6); even codes own
+// their tie points; everything above 5 saturates to 6.
+__device__ __forceinline__ uint32_t e2m1_encode(float y) {
+  const float a = fabsf(y);
+  uint32_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return (y < 0.f && c != 0) ? (c | 8u) : c;
+}
+
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+  const float m = mag[code & 7u];
+  return (code & 8u) ? -m : m;
+}
+
+// Non-negative x -> E4M3 code (bias 7, subnormal step 2^-9), RNE, saturating at
+// 448 (code 0x7E).  Mantissa overflow carries into the exponent naturally.
+__device__ __forceinline__ uint32_t e4m3_encode_pos(float x) {
+  if (!(x > 0.f)) return 0u;
+  if (x >= 448.f) return 0x7Eu;
+  if (x < 0x1p-6f) return (uint32_t)rintf(x * 512.f);          // subnormal grid
+  int E;
+  const float f = frexpf(x, &E);                                 // x = f * 2^E, f in [.5,1)
+  const int e = E - 1;                                           // x = (2f) * 2^e
+  const uint32_t man = (uint32_t)rintf((2.f * f - 1.f) * 8.f);   // 0..8
+  const uint32_t code = ((uint32_t)(e + 7) << 3) + man;
+  return code > 0x7Eu ? 0x7Eu : code;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t ex = (code >> 3) & 15u, m = code & 7u;
+  const float v = ex == 0 ? (float)m * 0x1p-9f
+                          : __uint_as_float(((ex - 7u + 127u) << 23) | (m << 20));
+  return (code & 0x80u) ? -v : v;
+}
+
+}  // namespace lmoe

@@ -19,6 +19,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "nvfp4.cuh"
 #include "sm100.cuh"
 
 namespace lmoe {
@@ -30,16 +31,22 @@ constexpr int kBK = 64;                   // K elements per stage (128 B of bf16
 constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
 constexpr int kWTileBytes = kBM * kBK * 2;
 
-template <int NT, int STAGES>
+constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
+
+template <int NT, int STAGES, bool WQ = false>
 struct UmmaSmem {
   static constexpr int kATileBytes = NT * kBK * 2;
-  static constexpr int kStageBytes = kWTileBytes + kATileBytes;
+  static constexpr int kRawOffset = kWTileBytes + kATileBytes;    // NVFP4 record (WQ)
+  static constexpr int kStageBytes =
+      (kWTileBytes + kATileBytes + (WQ ? kWqRecordBytes : 0) + 1023) / 1024 * 1024;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
   static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
 };
 
 struct TileInfo {
+  int grp;         // group (expert) index, 0 in dense mode
+  int mblk;        // 128-row block of the weight matrix
   int w_row0;      // first weight row (row of the weight tensor map)
   int n0;          // first output column (weight row within the group)
   int a_row0;      // first A row (token / pair) of the tile
@@ -65,6 +72,8 @@ __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInf
   if (nnb == 0) return false;
   const int mblk = local / nnb, nb = local - mblk * nnb;
   if (mblk >= nmb) return false;
+  ti.grp = e;
+  ti.mblk = mblk;
   ti.n0 = mblk * kBM;
   ti.w_row0 = e * a.w_group_rows + ti.n0;
   ti.a_row0 = base + nb * NT;
@@ -79,19 +88,64 @@ __device__ __forceinline__ int total_tiles(const UmmaArgs& a) {
 template <typename TO>
 __device__ __forceinline__ void store_out(TO* p, float v) { store_val(p, v); }
 
-template <int NT, int STAGES, typename TO, bool RELU2>
-__global__ void __launch_bounds__(192, 1)
+// Bulk (non-tensor) copy of `bytes` contiguous bytes into shared memory,
+// completion signalled on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// NVFP4 record row r -> bf16 row r of the 128-byte-swizzled W tile: chunk c
+// (k = 8c..8c+7) lands at 16-byte slot c ^ (r & 7).  q * value(s_b) is exact in
+// bf16 (at most 6 significant bits); the global scale is applied later.
+__device__ __forceinline__ void dequant_row(const uint8_t* rec, uint8_t* wtile, int r) {
+  const uint4 c01[2] = {reinterpret_cast<const uint4*>(rec + r * 32)[0],
+                        reinterpret_cast<const uint4*>(rec + r * 32)[1]};
+  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(c01);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float s = e4m3_value((sc >> (8 * (c >> 1))) & 0xFFu);
+    const uint32_t q = cw[c];
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = e2m1_value((q >> (8 * i)) & 0xFu) * s;
+      const float hi = e2m1_value((q >> (8 * i + 4)) & 0xFu) * s;
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+      o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// NVFP4 round trip of v across the 16-lane block it belongs to (global scale
+// 1): s_b = E4M3(amax / 6), q = E2M1(v / value(s_b)), returns q * value(s_b).
+__device__ __forceinline__ float nvfp4_roundtrip16(float v) {
+  float amax = fabsf(v);
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
+  if (!(scale > 0.f)) return 0.f;
+  return __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v, scale))), scale);
+}
+
+template <int NT, int STAGES, typename TO, bool RELU2, bool WQ, bool QA>
+__global__ void __launch_bounds__(WQ ? 320 : 192, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
                  const __grid_constant__ CUtensorMap amap0,
                  const __grid_constant__ CUtensorMap wmap1,
                  const __grid_constant__ CUtensorMap amap1, const UmmaArgs a) {
-  using S = UmmaSmem<NT, STAGES>;
+  using S = UmmaSmem<NT, STAGES, WQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;       // [2]
+  uint64_t* ready = empty + STAGES;          // [STAGES] dequantised W tile written (WQ)
+  uint64_t* acc_full = ready + STAGES;       // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint64_t* mma_done = acc_empty + 2;        // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -101,13 +155,17 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
   const int kt0 = a.K0 / kBK, kt_all = kt0 + a.K1 / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&ready[s], 128);
+    }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&wmap0);
     tma_prefetch_desc(&amap0);
+    if (!WQ) tma_prefetch_desc(&wmap0);
     if (a.K1 > 0) { tma_prefetch_desc(&wmap1); tma_prefetch_desc(&amap1); }
   }
   if (warp == 1) {
@@ -138,10 +196,17 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
           if (!mbar_wait(&empty[s], (round & 1) ^ 1)) { fail(1); break; }
           if (*abort_flag) break;
           uint8_t* st = smem + s * S::kStageBytes;
-          mbar_arrive_expect_tx(&full[s], S::kStageBytes);
           const bool seg1 = kt >= kt0;
           const int k0 = (seg1 ? kt - kt0 : kt) * kBK;
-          tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
+          if (WQ) {
+            mbar_arrive_expect_tx(&full[s], S::kATileBytes + kWqRecordBytes);
+            const uint8_t* rec = a.wq + (((size_t)ti.grp * a.wq_mblks + ti.mblk) * kt_all + kt) *
+                                            (size_t)kWqRecordBytes;
+            bulk_load(st + S::kRawOffset, rec, kWqRecordBytes, &full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], kWTileBytes + S::kATileBytes);
+            tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
+          }
           tma_load_2d(st + kWTileBytes, seg1 ? &amap1 : &amap0, &full[s], k0, ti.a_row0);
         }
       }
@@ -167,7 +232,12 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         bool ok = true;
         for (int kt = 0; kt < kt_all; ++kt, ++it) {
           const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1)) { fail(4); ok = false; break; }
+          const uint32_t par = (it / STAGES) & 1;
+          if (!mbar_wait(&full[s], par) || (WQ && !mbar_wait(&ready[s], par))) {
+            fail(4);
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t wa = smem_u32(smem + s * S::kStageBytes);
           const uint32_t aa = wa + kWTileBytes;
@@ -184,7 +254,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) fail(5);
     }
-  } else {
+  } else if (warp < 6) {
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
     TO* out = reinterpret_cast<TO*>(a.out);
@@ -197,26 +267,45 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;   // output column of this thread
       const bool col_ok = n < a.n_out;
+      const float gs = a.gscale ? a.gscale[ti.grp] : 1.f;
 #pragma unroll
       for (int c = 0; c < NT / 8; ++c) {
         uint32_t r[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, r);
         tmem_ld_wait();
-        if (col_ok) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int row = c * 8 + j;
-            if (row < ti.valid) {
-              float v = __uint_as_float(r[j]);
-              if (RELU2) v = relu2(v);
-              store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
-            }
+        for (int j = 0; j < 8; ++j) {
+          const int row = c * 8 + j;
+          if (row < ti.valid) {              // uniform across the warp
+            float v = __uint_as_float(r[j]);
+            if (a.gscale) v = __fmul_rn(v, gs);
+            if (RELU2) v = relu2(v);
+            if (QA) v = nvfp4_roundtrip16(col_ok ? v : 0.f);
+            if (col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
       ++lt;
+    }
+  } else if (WQ) {
+    // ---------------- NVFP4 dequant: warps 6..9, one W row per thread ----------------
+    const int r = threadIdx.x - 192;
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+      TileInfo ti;
+      if (!decode_tile<NT>(a, tile, ti)) continue;
+      bool ok = true;
+      for (int kt = 0; kt < kt_all; ++kt, ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (it / STAGES) & 1)) { fail(7); ok = false; break; }
+        uint8_t* st = smem + s * S::kStageBytes;
+        dequant_row(st + S::kRawOffset, st, r);
+        fence_proxy_async();                 // generic-proxy writes -> tensor-core reads
+        mbar_arrive(&ready[s]);
+      }
+      if (!ok) break;
     }
   }
   tc_fence_before();
@@ -261,10 +350,10 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
          CUDA_SUCCESS;
 }
 
-template <int NT, int STAGES, typename TO, bool RELU2>
+template <int NT, int STAGES, typename TO, bool RELU2, bool WQ, bool QA>
 static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
-  using S = UmmaSmem<NT, STAGES>;
-  auto kern = umma_gemm_kernel<NT, STAGES, TO, RELU2>;
+  using S = UmmaSmem<NT, STAGES, WQ>;
+  auto kern = umma_gemm_kernel<NT, STAGES, TO, RELU2, WQ, QA>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -276,25 +365,36 @@ static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   }
   int grid = L.max_tiles < sms ? L.max_tiles : sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
+  kern<<<grid, WQ ? 320 : 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
   return cudaGetLastError();
 }
 
-template <int NT, int STAGES>
+template <int NT, int STAGES, bool WQ>
 static cudaError_t umma_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
   switch (L.epi) {
-    case UMMA_EPI_BF16: return umma_launch_t<NT, STAGES, __nv_bfloat16, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return umma_launch_t<NT, STAGES, __nv_bfloat16, true>(L, st);
-    case UMMA_EPI_F32: return umma_launch_t<NT, STAGES, float, false>(L, st);
+    case UMMA_EPI_BF16: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, WQ, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, WQ, false>(L, st);
+    case UMMA_EPI_F32: return umma_launch_t<NT, STAGES, float, false, WQ, false>(L, st);
+    case UMMA_EPI_BF16_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, WQ, true>(L, st);
+    case UMMA_EPI_BF16_RELU2_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, WQ, true>(L, st);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st) {
+  if (L.args.wq) {
+    if (L.args.K1 != 0) return cudaErrorInvalidValue;    // NVFP4 weights: one segment
+    switch (L.nt) {
+      case 16: return umma_launch_nt<16, 8, true>(L, st);
+      case 64: return umma_launch_nt<64, 6, true>(L, st);
+      case 256: return umma_launch_nt<256, 4, true>(L, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (L.nt) {
-    case 16: return umma_launch_nt<16, 8>(L, st);
-    case 64: return umma_launch_nt<64, 8>(L, st);
-    case 256: return umma_launch_nt<256, 4>(L, st);
+    case 16: return umma_launch_nt<16, 8, false>(L, st);
+    case 64: return umma_launch_nt<64, 8, false>(L, st);
+    case 256: return umma_launch_nt<256, 4, false>(L, st);
   }
   return cudaErrorInvalidValue;
 }

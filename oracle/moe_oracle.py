@@ -284,10 +284,20 @@ def _rne_grid_vec(ax: np.ndarray, values: np.ndarray) -> np.ndarray:
 
 
 def e2m1_encode_vec(x: np.ndarray) -> np.ndarray:
-    """Vector e2m1_encode -> uint8 codes."""
-    x = np.asarray(x, dtype=np.float64)
-    c = _rne_grid_vec(np.abs(x), np.array(_E2M1_POS_V))
-    return np.where((x < 0) & (c != 0), c | 8, c).astype(np.uint8)
+    """Vector e2m1_encode -> uint8 codes.  The nearest point of the grid
+    0, .5, 1, 1.5, 2, 3, 4, 6 with ties to the even code is the number of
+    midpoints below |x|, where a midpoint counts when |x| passes it strictly if
+    the code below it is even (.25, 1.25, 2.5, 5) and when |x| reaches it if the
+    code above it is even (.75, 1.75, 3.5)."""
+    x = np.asarray(x)
+    a = np.abs(x)
+    code = np.zeros(a.shape, dtype=np.uint8)
+    for t in (0.25, 1.25, 2.5, 5.0):
+        code += a > t
+    for t in (0.75, 1.75, 3.5):
+        code += a >= t
+    code |= ((x < 0) & (code != 0)).astype(np.uint8) << 3
+    return code
 
 
 def e4m3_encode_vec(x: np.ndarray) -> np.ndarray:

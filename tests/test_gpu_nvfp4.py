@@ -1,0 +1,109 @@
+"""NVFP4 on the GPU against the oracle (report section 8.1; NVFP4 format details).
+
+The quantiser's codes, block scales and global scales must equal the oracle's
+bit for bit on the same inputs; NVFP4 layers must route bit-exactly and match
+the oracle's emulated NVFP4 layer within rel-L2 5e-2."""
+import numpy as np
+import pytest
+import torch
+
+from latentmoe_expert_routing_b200 import inputs as I
+from oracle import moe_oracle as O
+from tests.gpu_common import (REL_L2_NVFP4, check_dispatch_properties, np32, oracle_rows,
+                              out_metrics)
+from tests.test_gpu_parity import _assert_routing_exact, _run_full
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from latentmoe_expert_routing_b200 import build
+    build.build()
+    from latentmoe_expert_routing_b200 import layer
+    return layer
+
+
+def _gpu_quantize(w):
+    from latentmoe_expert_routing_b200 import binding as B
+    n, rows, K = w.shape
+    codes = torch.empty(n, rows, K // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(n, rows, K // 16, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(n, dtype=torch.float32, device="cuda")
+    dt = B.MOE_BF16 if w.dtype == torch.bfloat16 else B.MOE_FP32
+    B.moe_quantize_nvfp4(w.data_ptr(), dt, n, rows, K, codes.data_ptr(), scales.data_ptr(),
+                         gs.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    return codes.cpu().numpy(), scales.cpu().numpy(), gs.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantizer_bit_exact(L, dtype):
+    g = torch.Generator().manual_seed(3)
+    w = (torch.randn(4, 192, 320, generator=g) * 0.05)
+    w[0, 0, :16] = 0.0                                   # all-zero block
+    w[1, 3, :16] = torch.tensor([6.0, 3.0, 2.5, 1.75, 1.25, 0.75, 0.25, -5.0,
+                                 -3.5, 0.5, 1.0, 1.5, 2.0, 4.0, -6.0, 0.0]) * 0.01
+    w[2] *= 100.0                                        # another global scale
+    w[3, 5, 16:32] = 1e-6                                # subnormal block scale region
+    w = w.to(dtype).cuda()
+    codes, scales, gs = _gpu_quantize(w)
+    wn = w.float().cpu().numpy()
+    for m in range(4):
+        sg = O.nvfp4_global_scale(wn[m])
+        q, sb = O.nvfp4_quantize(wn[m], sg)
+        assert gs[m].view(np.int32) == np.float32(sg).view(np.int32)
+        assert np.array_equal(scales[m], sb)
+        assert np.array_equal(codes[m], O.pack_e2m1(q))
+
+
+@pytest.mark.parametrize("fmt", ["w4a16", "w4a4"])
+@pytest.mark.parametrize("T", [3, 64, 200])
+def test_tiny_nvfp4_layer(L, fmt, T):
+    cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt=fmt)
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    rel, nmax, raw = out_metrics(g[0], r["out"])
+    assert rel <= REL_L2_NVFP4, (rel, nmax)
+
+
+@pytest.fixture(scope="module")
+def ultra_bf16_weights(L):
+    W = L.weights_for(I.CONFIGS["ultra_decode_bf16"])
+    yield W
+    del W
+    torch.cuda.empty_cache()
+
+
+def _ultra_check(L, W, cfg, route_rows, out_rows):
+    lay = L.layer_for(cfg, W, out_dtype="fp32")
+    x = I.hidden(cfg, "cuda")
+    out, idx, w = lay(x)
+    counts, offsets, perm, pos = lay.routing(cfg.T)
+    lay.sync()
+    idx_h = idx.cpu().numpy()
+    check_dispatch_properties(idx_h, counts.cpu().numpy(), offsets.cpu().numpy(),
+                              perm.cpu().numpy(), pos.cpu().numpy(), cfg.E)
+    l = O.router_logits(np32(x[route_rows]), np32(W["w_gate"]))
+    _, _, ridx, rw = O.route(l, np32(W["gate_bias"]), cfg.k, cfg.rsf)
+    assert np.array_equal(idx_h[route_rows], ridx)
+    assert np.array_equal(np32(w)[route_rows].view(np.int32), rw.view(np.int32))
+    r = oracle_rows(cfg, W, x, rows=out_rows)
+    rel, nmax, raw = out_metrics(out[out_rows], r["out"])
+    assert rel <= REL_L2_NVFP4, (rel, nmax)
+    lay.close()
+    return counts.cpu().numpy()
+
+
+def test_ultra_decode_w4a16(L, ultra_bf16_weights):
+    cfg = I.CONFIGS["ultra_decode_w4a16"]
+    _ultra_check(L, ultra_bf16_weights, cfg, list(range(cfg.T)), [7])
+
+
+def test_skewed_prefill_w4a4(L, ultra_bf16_weights):
+    cfg = I.CONFIGS["skewed_prefill_w4a4"]
+    W = dict(ultra_bf16_weights)
+    W["gate_bias"] = I.gate_bias(cfg, "cuda")          # Zipf profile
+    counts = _ultra_check(L, W, cfg, [0, 1, 5000, 16383] + list(range(100, 116)), [11])
+    assert O.max_violation(counts) > 20

@@ -321,3 +321,16 @@ def test_nvfp4_error_bound_and_scales():
 def test_pack_e2m1_low_nibble_first():
     c = np.array([[1, 2, 15, 0]], np.uint8)
     assert O.pack_e2m1(c).tolist() == [[0x21, 0x0F]]
+
+
+def test_e2m1_vector_encoder_matches_scalar_definition():
+    x = np.concatenate([np.linspace(-7, 7, 5601), np.array([0.25, 0.75, 1.25, 1.75, 2.5,
+                                                             3.5, 5.0, -0.25, -5.0, 0.0])])
+    assert [O.e2m1_encode(v) for v in x] == O.e2m1_encode_vec(x.astype(np.float32)).tolist()
+
+
+def test_e4m3_vector_encoder_matches_scalar_definition():
+    y = np.abs(np.random.RandomState(12).standard_normal(4000)) * np.logspace(-4, 3, 4000)
+    mids = [(O.e4m3_value(c) + O.e4m3_value(c + 1)) / 2 for c in range(0, 0x7E)]
+    y = np.concatenate([y, mids, [0.0, 448.0, 500.0]])
+    assert [O.e4m3_encode(v) for v in y] == O.e4m3_encode_vec(y).tolist()
