@@ -114,10 +114,12 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
   cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, codes, scales,
                                         h->gs_up, amax, s);
   if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)F, (int)L, h->rec_up, s);
+  if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_up, h->gs_up, (int)E, s);
   if (e == cudaSuccess)
     e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, codes, scales, h->gs_dn,
                               amax, s);
   if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, s);
+  if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   cudaFree(codes); cudaFree(scales); cudaFree(amax);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -126,6 +126,7 @@ cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
                                   uint8_t* codes, uint8_t* scales, float* gscale,
                                   unsigned* amax_tmp, cudaStream_t st);
+cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t st);
 cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
                                int K, uint8_t* out, cudaStream_t st);
 void launch_gather_rows(const void* z, const int32_t* perm, void* zp, long P, int k, int L,

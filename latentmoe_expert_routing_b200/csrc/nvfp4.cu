@@ -7,7 +7,10 @@
 // the low nibble), scales [n_mat, rows, K/16], gscale [n_mat].
 // GEMM layout (library internal): per (matrix, 128-row block, 64-K stage) one
 // contiguous 4608-byte record: 128 rows x 32 code bytes, then 128 rows x 4
-// scale bytes; rows past the matrix are zero.
+// scale bytes; rows past the matrix are zero.  Within a row, 32-bit word i holds
+// elements k = 8i..8i+7 with element 8i+2j in bits 4j..4j+3 and element
+// 8i+2j+1 in bits 16+4j..19+4j, so that one shift pair turns the word into a
+// bf16 pair (see the dequant in umma_gemm.cu).
 #include "common.cuh"
 #include "kernels.h"
 #include "nvfp4.cuh"
@@ -77,16 +80,24 @@ __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint
   const int r = threadIdx.x;
   const int row = mb * 128 + r;
   uint8_t* o = out + rec * 4608;
-  uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+  uint32_t wd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint32_t s = 0;
   if (row < rows) {
     const uint8_t* cp = codes + ((size_t)m * rows + row) * (K / 2) + ks * 32;
-    c0 = *reinterpret_cast<const uint4*>(cp);
-    c1 = *reinterpret_cast<const uint4*>(cp + 16);
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t b4 = *reinterpret_cast<const uint32_t*>(cp + 4 * i);   // bytes B0..B3
+      uint32_t w = 0;
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t bj = (b4 >> (8 * j)) & 0xFFu;
+        w |= (bj & 0xFu) << (4 * j);          // element 8i+2j
+        w |= (bj >> 4) << (16 + 4 * j);       // element 8i+2j+1
+      }
+      wd[i] = w;
+    }
     s = *reinterpret_cast<const uint32_t*>(scales + ((size_t)m * rows + row) * (K / 16) + ks * 4);
   }
-  reinterpret_cast<uint4*>(o + r * 32)[0] = c0;
-  reinterpret_cast<uint4*>(o + r * 32)[1] = c1;
+  reinterpret_cast<uint4*>(o + r * 32)[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  reinterpret_cast<uint4*>(o + r * 32)[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
   reinterpret_cast<uint32_t*>(o + 4096)[r] = s;
 }
 
@@ -109,6 +120,18 @@ cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int ro
     quantize_blocks_kernel<<<ceil_div(nb, 256), 256, 0, st>>>((const float*)w, n_mat, rows, K,
                                                               gscale, codes, scales);
   }
+  return cudaGetLastError();
+}
+
+// gs_gemm = s_g * 2^26: the dequantised tiles hold q * s_b * 2^-26 (section in
+// umma_gemm.cu), the epilogue multiplies the accumulator back.
+__global__ void gemm_gscale_kernel(const float* __restrict__ gs, float* __restrict__ out, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = gs[i] * 0x1p26f;
+}
+
+cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t st) {
+  gemm_gscale_kernel<<<ceil_div(n, 256), 256, 0, st>>>(gs, out, n);
   return cudaGetLastError();
 }
 

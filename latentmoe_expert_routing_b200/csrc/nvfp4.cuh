@@ -24,9 +24,10 @@ __device__ __forceinline__ uint32_t e2m1_encode(float y) {
 }
 
 __device__ __forceinline__ float e2m1_value(uint32_t code) {
-  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
-  const float m = mag[code & 7u];
-  return (code & 8u) ? -m : m;
+  // exponent bits e = code[2:1] (bias 1), mantissa bit m = code[0]; e = 0 is 0 or 0.5
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  const float mag = e == 0 ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
+  return (code & 8u) ? -mag : mag;
 }
 
 // Non-negative x -> E4M3 code (bias 7, subnormal step 2^-9), RNE, saturating at

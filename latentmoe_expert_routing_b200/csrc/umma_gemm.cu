@@ -97,27 +97,46 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// NVFP4 record row r -> bf16 row r of the 128-byte-swizzled W tile: chunk c
-// (k = 8c..8c+7) lands at 16-byte slot c ^ (r & 7).  q * value(s_b) is exact in
-// bf16 (at most 6 significant bits); the global scale is applied later.
-__device__ __forceinline__ void dequant_row(const uint8_t* rec, uint8_t* wtile, int r) {
-  const uint4 c01[2] = {reinterpret_cast<const uint4*>(rec + r * 32)[0],
-                        reinterpret_cast<const uint4*>(rec + r * 32)[1]};
+// NVFP4 record -> bf16 W tile.  Thread (r, half) expands chunks 4*half ..
+// 4*half+3 of row r (k = 8c..8c+7 each) into the 128-byte-swizzled tile: chunk c
+// lands at 16-byte slot c ^ (r & 7).  A record word holds the pair (8c+2j,
+// 8c+2j+1) at bits 4j and 16+4j; shifting the 3 magnitude bits of each code
+// into bf16 bits 6-8 (sign into bit 15) gives exactly q * 2^-126 (code 1 is the
+// bf16 subnormal 2^-127), and one bf16x2 multiply by value(s_b) * 2^100 gives
+// q * s_b * 2^-26 exactly (at most 6 significant bits, normal range).  The
+// epilogue multiplies the accumulator by s_g * 2^26.
+template <int J>
+__device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t x) {
+  constexpr int sa = 6 - 4 * J, sb = 12 - 4 * J;
+  const uint32_t a = sa >= 0 ? (x << sa) : (x >> -sa);
+  const uint32_t b = x << sb;
+  return (a & 0x01C001C0u) | (b & 0x80008000u);
+}
+
+__device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile, int r, int half) {
+  const uint4 cw = reinterpret_cast<const uint4*>(rec + r * 32)[half];
   const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
-  const uint32_t* cw = reinterpret_cast<const uint32_t*>(c01);
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float s = e4m3_value((sc >> (8 * (c >> 1))) & 0xFFu);
-    const uint32_t q = cw[c];
-    uint32_t o[4];
+  for (int b = 0; b < 2; ++b) {
+    const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
+    const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
+    const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float lo = e2m1_value((q >> (8 * i)) & 0xFu) * s;
-      const float hi = e2m1_value((q >> (8 * i + 4)) & 0xFu) * s;
-      const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
-      o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 4 * half + 2 * b + cc;
+      const uint32_t x = words[2 * b + cc];
+      uint32_t o[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
+                       e2m1_pair_bits<3>(x)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
+        v = __hmul2(v, s2);
+        o[j] = *reinterpret_cast<uint32_t*>(&v);
+      }
+      *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -133,7 +152,7 @@ __device__ __forceinline__ float nvfp4_roundtrip16(float v) {
 }
 
 template <int NT, int STAGES, typename TO, bool RELU2, bool WQ, bool QA>
-__global__ void __launch_bounds__(WQ ? 320 : 192, 1)
+__global__ void __launch_bounds__(WQ ? 448 : 192, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
                  const __grid_constant__ CUtensorMap amap0,
                  const __grid_constant__ CUtensorMap wmap1,
@@ -158,7 +177,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&ready[s], 128);
+      mbar_init(&ready[s], 256);
     }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     mbar_init(mma_done, 1);
@@ -290,8 +309,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       ++lt;
     }
   } else if (WQ) {
-    // ---------------- NVFP4 dequant: warps 6..9, one W row per thread ----------------
-    const int r = threadIdx.x - 192;
+    // ---------------- NVFP4 dequant: warps 6..13, half a W row per thread ----------------
+    const int r = (threadIdx.x - 192) >> 1, half = (threadIdx.x - 192) & 1;
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
       TileInfo ti;
@@ -301,7 +320,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         const int s = it % STAGES;
         if (!mbar_wait(&full[s], (it / STAGES) & 1)) { fail(7); ok = false; break; }
         uint8_t* st = smem + s * S::kStageBytes;
-        dequant_row(st + S::kRawOffset, st, r);
+        dequant_half(st + S::kRawOffset, st, r, half);
         fence_proxy_async();                 // generic-proxy writes -> tensor-core reads
         mbar_arrive(&ready[s]);
       }
@@ -365,7 +384,7 @@ static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   }
   int grid = L.max_tiles < sms ? L.max_tiles : sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, WQ ? 320 : 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
+  kern<<<grid, WQ ? 448 : 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
   return cudaGetLastError();
 }
 

@@ -66,6 +66,10 @@ def test_tiny_nvfp4_layer(L, fmt, T):
     _assert_routing_exact(g, r)
     rel, nmax, raw = out_metrics(g[0], r["out"])
     assert rel <= REL_L2_NVFP4, (rel, nmax)
+    if fmt == "w4a16":
+        # same weights as the oracle's emulated path: only accumulation order and
+        # bf16 activation rounding differ, so the error stays at the bf16 level
+        assert rel <= 1e-2, rel
 
 
 @pytest.fixture(scope="module")
