@@ -123,6 +123,7 @@ struct UmmaLaunch {
 };
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
+cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
                                   uint8_t* codes, uint8_t* scales, float* gscale,
                                   unsigned* amax_tmp, cudaStream_t st);

@@ -36,11 +36,12 @@ __device__ __forceinline__ uint32_t e4m3_encode_pos(float x) {
   if (!(x > 0.f)) return 0u;
   if (x >= 448.f) return 0x7Eu;
   if (x < 0x1p-6f) return (uint32_t)rintf(x * 512.f);          // subnormal grid
-  int E;
-  const float f = frexpf(x, &E);                                 // x = f * 2^E, f in [.5,1)
-  const int e = E - 1;                                           // x = (2f) * 2^e
-  const uint32_t man = (uint32_t)rintf((2.f * f - 1.f) * 8.f);   // 0..8
-  const uint32_t code = ((uint32_t)(e + 7) << 3) + man;
+  // normal: keep 3 of the 23 fp32 mantissa bits, round half to even at bit 20
+  const uint32_t b = __float_as_uint(x);
+  const uint32_t e = (b >> 23) - 120u;                           // (E - 127) + 7, in 1..15
+  const uint32_t m = b & 0x7FFFFFu;
+  const uint32_t r = m + 0x7FFFFu + ((m >> 20) & 1u);
+  const uint32_t code = (e << 3) + (r >> 20);                    // carry moves into the exponent
   return code > 0x7Eu ? 0x7Eu : code;
 }
 

@@ -46,14 +46,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, giving up after about
-// a second.  Returns false on timeout (the caller records it and unwinds).
-constexpr uint32_t kWaitSpinLimit = 1u << 22;
+// two seconds of SM clock.  try_wait itself suspends the thread for a short,
+// hardware-chosen time, so the loop polls without sleeping (a sleep here would
+// add its wake-up granularity to every pipeline hand-off).  Returns false on
+// timeout (the caller records it and unwinds).
+constexpr long long kWaitCycles = 4000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (i >= 64) __nanosleep(256);
+    if (clock64() - t0 > kWaitCycles) return false;
   }
-  return false;
+}
+
+// Same bound, for waits that normally last a whole tile (the epilogue waiting for
+// an accumulator): back off with short sleeps so the polling warps leave issue
+// slots to the producer and MMA threads of the same SM.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(64);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
 }
 
 // ---- TMA -------------------------------------------------------------------

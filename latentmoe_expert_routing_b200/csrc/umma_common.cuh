@@ -1,0 +1,140 @@
+// Helpers shared by the tensor-core GEMM kernels (umma_gemm.cu, umma_nvfp4.cu):
+// tile decoding over a device-side tile list, NVFP4 dequantisation into
+// swizzled bf16 tiles, the NVFP4 activation round trip of the W4A4 epilogue.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "nvfp4.cuh"
+#include "sm100.cuh"
+
+namespace lmoe {
+
+using namespace sm100;
+
+constexpr int kBM = 128;                  // weight rows per tile (MMA M)
+constexpr int kBK = 64;                   // K elements per stage (128 B of bf16)
+constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
+constexpr int kWTileBytes = kBM * kBK * 2;
+
+constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
+
+template <int NT, int STAGES>
+struct UmmaSmem {
+  static constexpr int kATileBytes = NT * kBK * 2;
+  static constexpr int kStageBytes = kWTileBytes + kATileBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
+  static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
+};
+
+struct TileInfo {
+  int grp;         // group (expert) index, 0 in dense mode
+  int mblk;        // 128-row block of the weight matrix
+  int w_row0;      // first weight row (row of the weight tensor map)
+  int n0;          // first output column (weight row within the group)
+  int a_row0;      // first A row (token / pair) of the tile
+  int valid;       // A rows of the tile that belong to the group
+};
+
+template <int NT>
+__device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInfo& ti) {
+  const int nmb = (a.n_out + kBM - 1) / kBM;
+  int e = 0, base = 0, cnt = a.M, local = tile;
+  if (a.offsets) {
+    int lo = 0, hi = a.E;
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (a.tiles[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+    base = a.offsets[e];
+    cnt = a.offsets[e + 1] - base;
+    local = tile - a.tiles[e];
+  }
+  const int nnb = (cnt + NT - 1) / NT;
+  if (nnb == 0) return false;
+  const int mblk = local / nnb, nb = local - mblk * nnb;
+  if (mblk >= nmb) return false;
+  ti.grp = e;
+  ti.mblk = mblk;
+  ti.n0 = mblk * kBM;
+  ti.w_row0 = e * a.w_group_rows + ti.n0;
+  ti.a_row0 = base + nb * NT;
+  ti.valid = min(NT, cnt - nb * NT);
+  return true;
+}
+
+__device__ __forceinline__ int total_tiles(const UmmaArgs& a) {
+  return a.offsets ? a.tiles[a.E] : a.dense_tiles;
+}
+
+template <typename TO>
+__device__ __forceinline__ void store_out(TO* p, float v) { store_val(p, v); }
+
+// Bulk (non-tensor) copy of `bytes` contiguous bytes into shared memory,
+// completion signalled on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// NVFP4 record -> bf16 W tile.  Thread (r, half) expands chunks 4*half ..
+// 4*half+3 of row r (k = 8c..8c+7 each) into the 128-byte-swizzled tile: chunk c
+// lands at 16-byte slot c ^ (r & 7).  A record word holds the pair (8c+2j,
+// 8c+2j+1) at bits 4j and 16+4j; shifting the 3 magnitude bits of each code
+// into bf16 bits 6-8 (sign into bit 15) gives exactly q * 2^-126 (code 1 is the
+// bf16 subnormal 2^-127), and one bf16x2 multiply by value(s_b) * 2^100 gives
+// q * s_b * 2^-26 exactly (at most 6 significant bits, normal range).  The
+// epilogue multiplies the accumulator by s_g * 2^26.
+template <int J>
+__device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t x) {
+  constexpr int sa = 6 - 4 * J, sb = 12 - 4 * J;
+  const uint32_t a = sa >= 0 ? (x << sa) : (x >> -sa);
+  const uint32_t b = x << sb;
+  return (a & 0x01C001C0u) | (b & 0x80008000u);
+}
+
+__device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile, int r, int half) {
+  const uint4 cw = reinterpret_cast<const uint4*>(rec + r * 32)[half];
+  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
+    const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
+    const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 4 * half + 2 * b + cc;
+      const uint32_t x = words[2 * b + cc];
+      uint32_t o[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
+                       e2m1_pair_bits<3>(x)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
+        v = __hmul2(v, s2);
+        o[j] = *reinterpret_cast<uint32_t*>(&v);
+      }
+      *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// NVFP4 round trip of v across the 16-lane block it belongs to (global scale
+// 1): s_b = E4M3(amax / 6), q = E2M1(v / value(s_b)), returns q * value(s_b).
+__device__ __forceinline__ float nvfp4_roundtrip16(float v) {
+  float amax = fabsf(v);
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
+  if (!(scale > 0.f)) return 0.f;
+  return __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v, scale))), scale);
+}
+
+
+}  // namespace lmoe

@@ -17,154 +17,23 @@
 // DEV_ERR_TIMEOUT, unwinds, waits for its own copies / MMAs and frees TMEM.
 #include <cuda.h>
 
-#include "common.cuh"
-#include "kernels.h"
-#include "nvfp4.cuh"
-#include "sm100.cuh"
+#include "umma_common.cuh"
 
 namespace lmoe {
 
-using namespace sm100;
-
-constexpr int kBM = 128;                  // weight rows per tile (MMA M)
-constexpr int kBK = 64;                   // K elements per stage (128 B of bf16)
-constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
-constexpr int kWTileBytes = kBM * kBK * 2;
-
-constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
-
-template <int NT, int STAGES, bool WQ = false>
-struct UmmaSmem {
-  static constexpr int kATileBytes = NT * kBK * 2;
-  static constexpr int kRawOffset = kWTileBytes + kATileBytes;    // NVFP4 record (WQ)
-  static constexpr int kStageBytes =
-      (kWTileBytes + kATileBytes + (WQ ? kWqRecordBytes : 0) + 1023) / 1024 * 1024;
-  static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
-  static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
-};
-
-struct TileInfo {
-  int grp;         // group (expert) index, 0 in dense mode
-  int mblk;        // 128-row block of the weight matrix
-  int w_row0;      // first weight row (row of the weight tensor map)
-  int n0;          // first output column (weight row within the group)
-  int a_row0;      // first A row (token / pair) of the tile
-  int valid;       // A rows of the tile that belong to the group
-};
-
-template <int NT>
-__device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInfo& ti) {
-  const int nmb = (a.n_out + kBM - 1) / kBM;
-  int e = 0, base = 0, cnt = a.M, local = tile;
-  if (a.offsets) {
-    int lo = 0, hi = a.E;
-    while (hi - lo > 1) {
-      int mid = (lo + hi) >> 1;
-      if (a.tiles[mid] <= tile) lo = mid; else hi = mid;
-    }
-    e = lo;
-    base = a.offsets[e];
-    cnt = a.offsets[e + 1] - base;
-    local = tile - a.tiles[e];
-  }
-  const int nnb = (cnt + NT - 1) / NT;
-  if (nnb == 0) return false;
-  const int mblk = local / nnb, nb = local - mblk * nnb;
-  if (mblk >= nmb) return false;
-  ti.grp = e;
-  ti.mblk = mblk;
-  ti.n0 = mblk * kBM;
-  ti.w_row0 = e * a.w_group_rows + ti.n0;
-  ti.a_row0 = base + nb * NT;
-  ti.valid = min(NT, cnt - nb * NT);
-  return true;
-}
-
-__device__ __forceinline__ int total_tiles(const UmmaArgs& a) {
-  return a.offsets ? a.tiles[a.E] : a.dense_tiles;
-}
-
-template <typename TO>
-__device__ __forceinline__ void store_out(TO* p, float v) { store_val(p, v); }
-
-// Bulk (non-tensor) copy of `bytes` contiguous bytes into shared memory,
-// completion signalled on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// NVFP4 record -> bf16 W tile.  Thread (r, half) expands chunks 4*half ..
-// 4*half+3 of row r (k = 8c..8c+7 each) into the 128-byte-swizzled tile: chunk c
-// lands at 16-byte slot c ^ (r & 7).  A record word holds the pair (8c+2j,
-// 8c+2j+1) at bits 4j and 16+4j; shifting the 3 magnitude bits of each code
-// into bf16 bits 6-8 (sign into bit 15) gives exactly q * 2^-126 (code 1 is the
-// bf16 subnormal 2^-127), and one bf16x2 multiply by value(s_b) * 2^100 gives
-// q * s_b * 2^-26 exactly (at most 6 significant bits, normal range).  The
-// epilogue multiplies the accumulator by s_g * 2^26.
-template <int J>
-__device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t x) {
-  constexpr int sa = 6 - 4 * J, sb = 12 - 4 * J;
-  const uint32_t a = sa >= 0 ? (x << sa) : (x >> -sa);
-  const uint32_t b = x << sb;
-  return (a & 0x01C001C0u) | (b & 0x80008000u);
-}
-
-__device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile, int r, int half) {
-  const uint4 cw = reinterpret_cast<const uint4*>(rec + r * 32)[half];
-  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
-  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
-    const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
-    const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 4 * half + 2 * b + cc;
-      const uint32_t x = words[2 * b + cc];
-      uint32_t o[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
-                       e2m1_pair_bits<3>(x)};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
-        v = __hmul2(v, s2);
-        o[j] = *reinterpret_cast<uint32_t*>(&v);
-      }
-      *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) =
-          make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-}
-
-// NVFP4 round trip of v across the 16-lane block it belongs to (global scale
-// 1): s_b = E4M3(amax / 6), q = E2M1(v / value(s_b)), returns q * value(s_b).
-__device__ __forceinline__ float nvfp4_roundtrip16(float v) {
-  float amax = fabsf(v);
-#pragma unroll
-  for (int off = 1; off < 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
-  if (!(scale > 0.f)) return 0.f;
-  return __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v, scale))), scale);
-}
-
-template <int NT, int STAGES, typename TO, bool RELU2, bool WQ, bool QA>
-__global__ void __launch_bounds__(WQ ? 448 : 192, 1)
+template <int NT, int STAGES, typename TO, bool RELU2, bool QA>
+__global__ void __launch_bounds__(192, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
                  const __grid_constant__ CUtensorMap amap0,
                  const __grid_constant__ CUtensorMap wmap1,
                  const __grid_constant__ CUtensorMap amap1, const UmmaArgs a) {
-  using S = UmmaSmem<NT, STAGES, WQ>;
+  using S = UmmaSmem<NT, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset);
   uint64_t* empty = full + STAGES;
-  uint64_t* ready = empty + STAGES;          // [STAGES] dequantised W tile written (WQ)
-  uint64_t* acc_full = ready + STAGES;       // [2]
+  uint64_t* acc_full = empty + STAGES;       // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
   uint64_t* mma_done = acc_empty + 2;        // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -177,14 +46,13 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&ready[s], 256);
     }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&amap0);
-    if (!WQ) tma_prefetch_desc(&wmap0);
+    tma_prefetch_desc(&wmap0);
     if (a.K1 > 0) { tma_prefetch_desc(&wmap1); tma_prefetch_desc(&amap1); }
   }
   if (warp == 1) {
@@ -217,15 +85,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
           uint8_t* st = smem + s * S::kStageBytes;
           const bool seg1 = kt >= kt0;
           const int k0 = (seg1 ? kt - kt0 : kt) * kBK;
-          if (WQ) {
-            mbar_arrive_expect_tx(&full[s], S::kATileBytes + kWqRecordBytes);
-            const uint8_t* rec = a.wq + (((size_t)ti.grp * a.wq_mblks + ti.mblk) * kt_all + kt) *
-                                            (size_t)kWqRecordBytes;
-            bulk_load(st + S::kRawOffset, rec, kWqRecordBytes, &full[s]);
-          } else {
-            mbar_arrive_expect_tx(&full[s], kWTileBytes + S::kATileBytes);
-            tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
-          }
+          mbar_arrive_expect_tx(&full[s], kWTileBytes + S::kATileBytes);
+          tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
           tma_load_2d(st + kWTileBytes, seg1 ? &amap1 : &amap0, &full[s], k0, ti.a_row0);
         }
       }
@@ -252,7 +113,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         for (int kt = 0; kt < kt_all; ++kt, ++it) {
           const int s = it % STAGES;
           const uint32_t par = (it / STAGES) & 1;
-          if (!mbar_wait(&full[s], par) || (WQ && !mbar_wait(&ready[s], par))) {
+          if (!mbar_wait(&full[s], par)) {
             fail(4);
             ok = false;
             break;
@@ -273,7 +134,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) fail(5);
     }
-  } else if (warp < 6) {
+  } else {
     // ---------------- epilogue: warps 2..5 ----------------
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
     TO* out = reinterpret_cast<TO*>(a.out);
@@ -282,7 +143,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       TileInfo ti;
       if (!decode_tile<NT>(a, tile, ti)) continue;
       const uint32_t buf = lt & 1, use = lt >> 1;
-      if (!mbar_wait(&acc_full[buf], use & 1)) { fail(6); break; }
+      if (!mbar_wait_backoff(&acc_full[buf], use & 1)) { fail(6); break; }
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;   // output column of this thread
       const bool col_ok = n < a.n_out;
@@ -307,24 +168,6 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
       ++lt;
-    }
-  } else if (WQ) {
-    // ---------------- NVFP4 dequant: warps 6..13, half a W row per thread ----------------
-    const int r = (threadIdx.x - 192) >> 1, half = (threadIdx.x - 192) & 1;
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-      TileInfo ti;
-      if (!decode_tile<NT>(a, tile, ti)) continue;
-      bool ok = true;
-      for (int kt = 0; kt < kt_all; ++kt, ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&full[s], (it / STAGES) & 1)) { fail(7); ok = false; break; }
-        uint8_t* st = smem + s * S::kStageBytes;
-        dequant_half(st + S::kRawOffset, st, r, half);
-        fence_proxy_async();                 // generic-proxy writes -> tensor-core reads
-        mbar_arrive(&ready[s]);
-      }
-      if (!ok) break;
     }
   }
   tc_fence_before();
@@ -369,10 +212,10 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
          CUDA_SUCCESS;
 }
 
-template <int NT, int STAGES, typename TO, bool RELU2, bool WQ, bool QA>
+template <int NT, int STAGES, typename TO, bool RELU2, bool QA>
 static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
-  using S = UmmaSmem<NT, STAGES, WQ>;
-  auto kern = umma_gemm_kernel<NT, STAGES, TO, RELU2, WQ, QA>;
+  using S = UmmaSmem<NT, STAGES>;
+  auto kern = umma_gemm_kernel<NT, STAGES, TO, RELU2, QA>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -384,36 +227,28 @@ static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   }
   int grid = L.max_tiles < sms ? L.max_tiles : sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, WQ ? 448 : 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
+  kern<<<grid, 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
   return cudaGetLastError();
 }
 
-template <int NT, int STAGES, bool WQ>
+template <int NT, int STAGES>
 static cudaError_t umma_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
   switch (L.epi) {
-    case UMMA_EPI_BF16: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, WQ, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, WQ, false>(L, st);
-    case UMMA_EPI_F32: return umma_launch_t<NT, STAGES, float, false, WQ, false>(L, st);
-    case UMMA_EPI_BF16_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, WQ, true>(L, st);
-    case UMMA_EPI_BF16_RELU2_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, WQ, true>(L, st);
+    case UMMA_EPI_BF16: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, false>(L, st);
+    case UMMA_EPI_F32: return umma_launch_t<NT, STAGES, float, false, false>(L, st);
+    case UMMA_EPI_BF16_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, false, true>(L, st);
+    case UMMA_EPI_BF16_RELU2_Q: return umma_launch_t<NT, STAGES, __nv_bfloat16, true, true>(L, st);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st) {
-  if (L.args.wq) {
-    if (L.args.K1 != 0) return cudaErrorInvalidValue;    // NVFP4 weights: one segment
-    switch (L.nt) {
-      case 16: return umma_launch_nt<16, 8, true>(L, st);
-      case 64: return umma_launch_nt<64, 6, true>(L, st);
-      case 256: return umma_launch_nt<256, 4, true>(L, st);
-    }
-    return cudaErrorInvalidValue;
-  }
+  if (L.args.wq) return launch_umma_wq(L, st);           // NVFP4 weights: umma_nvfp4.cu
   switch (L.nt) {
-    case 16: return umma_launch_nt<16, 8, false>(L, st);
-    case 64: return umma_launch_nt<64, 8, false>(L, st);
-    case 256: return umma_launch_nt<256, 4, false>(L, st);
+    case 16: return umma_launch_nt<16, 8>(L, st);
+    case 64: return umma_launch_nt<64, 8>(L, st);
+    case 256: return umma_launch_nt<256, 4>(L, st);
   }
   return cudaErrorInvalidValue;
 }
