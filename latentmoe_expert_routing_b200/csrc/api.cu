@@ -36,6 +36,7 @@ struct moe_handle {
   uint32_t* cmask = nullptr;                     // [T, 32] candidate bits per token
   // NVFP4 experts: GEMM-layout records and per-expert global scales
   uint8_t *rec_up = nullptr, *rec_dn = nullptr;
+  CUtensorMap rm_up[3], rm_dn[3];                // record maps, batches of 1, 2, 4
   float *gs_up = nullptr, *gs_dn = nullptr;
   unsigned long long* stats = nullptr;           // exactly recomputed logits
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
@@ -120,6 +121,10 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
                               amax, s);
   if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, s);
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+    if (!make_tmap_records(&h->rm_up[i], h->rec_up, (long)recs_up, 1 << i) ||
+        !make_tmap_records(&h->rm_dn[i], h->rec_dn, (long)recs_dn, 1 << i))
+      e = cudaErrorInvalidValue;
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   cudaFree(codes); cudaFree(scales); cudaFree(amax);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -171,14 +176,21 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
   u.args.tiles = h->tiles_up; u.args.out = h->H;
   u.epi = w4a4 ? UMMA_EPI_BF16_RELU2_Q : UMMA_EPI_BF16_RELU2;
-  if (wq) { u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up; }
+  auto batch_idx = [](int kt) { return kt % 4 == 0 ? 2 : (kt % 2 == 0 ? 1 : 0); };
+  if (wq) {
+    u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up;
+    u.wqmap = h->rm_up[batch_idx(L / 64)];
+  }
   u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
   if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_EXPERT_DOWN);
   u.wmap0 = h->wm_dn; u.amap0 = h->am_H[gi];
   u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
   u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
-  if (wq) { u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn; }
+  if (wq) {
+    u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn;
+    u.wqmap = h->rm_dn[batch_idx(F / 64)];
+  }
   u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
   if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_COMBINE);

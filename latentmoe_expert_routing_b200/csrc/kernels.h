@@ -116,12 +116,15 @@ enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2,
                UMMA_EPI_BF16_Q = 3, UMMA_EPI_BF16_RELU2_Q = 4 };
 struct UmmaLaunch {
   CUtensorMap wmap0, amap0, wmap1, amap1;
+  CUtensorMap wqmap;        // NVFP4 records as [records][36][128 B] (see make_tmap_records)
   UmmaArgs args;
   int nt;                   // token rows per tile: 16, 64 or 256
   UmmaEpi epi;
   int max_tiles;            // upper bound of the tile count (grid clamp)
 };
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
+// NVFP4 GEMM records (4608 B each) as a 3-D uint8 tensor, box = `batch` records
+bool make_tmap_records(CUtensorMap* map, const void* base, long n_records, int batch);
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,

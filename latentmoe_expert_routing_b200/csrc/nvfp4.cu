@@ -6,8 +6,9 @@
 // Plain layout (C ABI): codes [n_mat, rows, K/2] (two per byte, even element in
 // the low nibble), scales [n_mat, rows, K/16], gscale [n_mat].
 // GEMM layout (library internal): per (matrix, 128-row block, 64-K stage) one
-// contiguous 4608-byte record: 128 rows x 32 code bytes, then 128 rows x 4
-// scale bytes; rows past the matrix are zero.  Within a row, 32-bit word i holds
+// contiguous 4608-byte record: codes as [half 0..1][row 0..127][16 bytes] (row r's
+// elements 32h..32h+31 at h*2048 + r*16), then 128 rows x 4 scale bytes; rows
+// past the matrix are zero.  Within a row, 32-bit word i holds
 // elements k = 8i..8i+7 with element 8i+2j in bits 4j..4j+3 and element
 // 8i+2j+1 in bits 16+4j..19+4j, so that one shift pair turns the word into a
 // bf16 pair (see the dequant in umma_gemm.cu).
@@ -96,8 +97,8 @@ __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint
     }
     s = *reinterpret_cast<const uint32_t*>(scales + ((size_t)m * rows + row) * (K / 16) + ks * 4);
   }
-  reinterpret_cast<uint4*>(o + r * 32)[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-  reinterpret_cast<uint4*>(o + r * 32)[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+  *reinterpret_cast<uint4*>(o + r * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  *reinterpret_cast<uint4*>(o + 2048 + r * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
   reinterpret_cast<uint32_t*>(o + 4096)[r] = s;
 }
 

@@ -17,6 +17,7 @@ constexpr int kBM = 128;                  // weight rows per tile (MMA M)
 constexpr int kBK = 64;                   // K elements per stage (128 B of bf16)
 constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
 constexpr int kWTileBytes = kBM * kBK * 2;
+constexpr int kTableBytes = 2 * 4 * 1025 + 16;     // tiles[E+1], offsets[E+1], E <= 1024
 
 constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
 
@@ -25,7 +26,8 @@ struct UmmaSmem {
   static constexpr int kATileBytes = NT * kBK * 2;
   static constexpr int kStageBytes = kWTileBytes + kATileBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int kTableOffset = kBarOffset + 256;
+  static constexpr int kBytes = kTableOffset + kTableBytes + 1024;   // + alignment slack
   static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
 };
 
@@ -38,20 +40,33 @@ struct TileInfo {
   int valid;       // A rows of the tile that belong to the group
 };
 
+// Grouped mode reads the tile and A-row offset tables from shared memory
+// (copied once per CTA by load_tables): the binary search then costs a few
+// shared loads instead of dependent trips to L2 on every tile.
+
+__device__ __forceinline__ void load_tables(const UmmaArgs& a, int32_t* s_tiles, int32_t* s_off) {
+  if (!a.offsets) return;
+  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) {
+    s_tiles[i] = a.tiles[i];
+    s_off[i] = a.offsets[i];
+  }
+}
+
 template <int NT>
-__device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInfo& ti) {
+__device__ __forceinline__ bool decode_tile(const UmmaArgs& a, const int32_t* s_tiles,
+                                            const int32_t* s_off, int tile, TileInfo& ti) {
   const int nmb = (a.n_out + kBM - 1) / kBM;
   int e = 0, base = 0, cnt = a.M, local = tile;
   if (a.offsets) {
     int lo = 0, hi = a.E;
     while (hi - lo > 1) {
       int mid = (lo + hi) >> 1;
-      if (a.tiles[mid] <= tile) lo = mid; else hi = mid;
+      if (s_tiles[mid] <= tile) lo = mid; else hi = mid;
     }
     e = lo;
-    base = a.offsets[e];
-    cnt = a.offsets[e + 1] - base;
-    local = tile - a.tiles[e];
+    base = s_off[e];
+    cnt = s_off[e + 1] - base;
+    local = tile - s_tiles[e];
   }
   const int nnb = (cnt + NT - 1) / NT;
   if (nnb == 0) return false;
@@ -66,8 +81,8 @@ __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, int tile, TileInf
   return true;
 }
 
-__device__ __forceinline__ int total_tiles(const UmmaArgs& a) {
-  return a.offsets ? a.tiles[a.E] : a.dense_tiles;
+__device__ __forceinline__ int total_tiles(const UmmaArgs& a, const int32_t* s_tiles) {
+  return a.offsets ? s_tiles[a.E] : a.dense_tiles;
 }
 
 template <typename TO>
@@ -82,7 +97,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// NVFP4 record -> bf16 W tile.  Thread (r, half) expands chunks 4*half ..
+// NVFP4 record -> bf16 W tile.  Record codes are half-major ([half][row][16 B]),
+// so a warp expanding 32 consecutive rows of one half reads 512 contiguous
+// bytes and its swizzled stores hit every bank evenly.
+// Thread (r, half) expands chunks 4*half ..
 // 4*half+3 of row r (k = 8c..8c+7 each) into the 128-byte-swizzled tile: chunk c
 // lands at 16-byte slot c ^ (r & 7).  A record word holds the pair (8c+2j,
 // 8c+2j+1) at bits 4j and 16+4j; shifting the 3 magnitude bits of each code
@@ -99,7 +117,7 @@ __device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t x) {
 }
 
 __device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile, int r, int half) {
-  const uint4 cw = reinterpret_cast<const uint4*>(rec + r * 32)[half];
+  const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
   const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
   const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll

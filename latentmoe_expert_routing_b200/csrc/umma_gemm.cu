@@ -38,6 +38,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
   uint64_t* mma_done = acc_empty + 2;        // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_tiles = reinterpret_cast<int32_t*>(smem + S::kTableOffset);
+  int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt0 = a.K0 / kBK, kt_all = kt0 + a.K1 / kBK;
@@ -59,11 +61,12 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     tmem_alloc(tmem_slot, S::kTmemCols);
     tmem_relinquish();
   }
+  load_tables(a, s_tiles, s_off);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ntiles = total_tiles(a);
+  const int ntiles = total_tiles(a, s_tiles);
 
   auto fail = [&](int where) {
     atomicOr(a.err, DEV_ERR_TIMEOUT | (where << 8));
@@ -73,22 +76,22 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t it = 0, st = 0, pe = 1;           // slot, parity to wait for (fresh: passes)
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
-        if (!decode_tile<NT>(a, tile, ti)) continue;
+        if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
+        bool ok = true;
         for (int kt = 0; kt < kt_all; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t round = it / STAGES;
-          if (!mbar_wait(&empty[s], (round & 1) ^ 1)) { fail(1); break; }
-          if (*abort_flag) break;
-          uint8_t* st = smem + s * S::kStageBytes;
+          if (!mbar_wait(&empty[st], pe)) { fail(1); ok = false; break; }
+          uint8_t* sp = smem + st * S::kStageBytes;
+          mbar_arrive_expect_tx(&full[st], kWTileBytes + S::kATileBytes);
           const bool seg1 = kt >= kt0;
           const int k0 = (seg1 ? kt - kt0 : kt) * kBK;
-          mbar_arrive_expect_tx(&full[s], kWTileBytes + S::kATileBytes);
-          tma_load_2d(st, seg1 ? &wmap1 : &wmap0, &full[s], k0, ti.w_row0);
-          tma_load_2d(st + kWTileBytes, seg1 ? &amap1 : &amap0, &full[s], k0, ti.a_row0);
+          tma_load_2d(sp, seg1 ? &wmap1 : &wmap0, &full[st], k0, ti.w_row0);
+          tma_load_2d(sp + kWTileBytes, seg1 ? &amap1 : &amap0, &full[st], k0, ti.a_row0);
+          if (++st == STAGES) { st = 0; pe ^= 1; }
         }
+        if (!ok) break;
       }
       // drain: every load this thread issued must land before the CTA exits
       const uint32_t n = it < (uint32_t)STAGES ? it : (uint32_t)STAGES;
@@ -99,33 +102,31 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // One thread; the loop is kept short (incremental slot and parity,
+    // descriptors advanced by constants) because its length sets the step rate.
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, NT);
-      uint32_t it = 0, lt = 0;
+      const uint64_t desc0 = sw128_desc(smem_u32(smem));
+      uint32_t st = 0, pf = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
-        if (!decode_tile<NT>(a, tile, ti)) continue;
+        if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         const uint32_t buf = lt & 1, use = lt >> 1;
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(3); break; }
         tc_fence_after();
         const uint32_t d = tmem + buf * NT;
         bool ok = true;
-        for (int kt = 0; kt < kt_all; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t par = (it / STAGES) & 1;
-          if (!mbar_wait(&full[s], par)) {
-            fail(4);
-            ok = false;
-            break;
-          }
+        for (int kt = 0; kt < kt_all; ++kt) {
+          if (!mbar_wait(&full[st], pf)) { fail(4); ok = false; break; }
           tc_fence_after();
-          const uint32_t wa = smem_u32(smem + s * S::kStageBytes);
-          const uint32_t aa = wa + kWTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-            mma_bf16_ss(d, sw128_desc(wa + kk * kUmmaK * 2), sw128_desc(aa + kk * kUmmaK * 2),
-                        idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[s]);             // frees the stage when these MMAs finish
+          const uint64_t wd = desc0 + (uint64_t)(st * (S::kStageBytes >> 4));
+          const uint64_t ad = wd + (uint64_t)(kWTileBytes >> 4);
+          mma_bf16_ss(d, wd, ad, idesc, kt > 0 ? 1u : 0u);
+          mma_bf16_ss(d, wd + 2, ad + 2, idesc, 1u);
+          mma_bf16_ss(d, wd + 4, ad + 4, idesc, 1u);
+          mma_bf16_ss(d, wd + 6, ad + 6, idesc, 1u);
+          mma_commit(&empty[st]);            // frees the stage when these MMAs finish
+          if (++st == STAGES) { st = 0; pf ^= 1; }
         }
         if (!ok) break;
         mma_commit(&acc_full[buf]);
@@ -141,7 +142,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     uint32_t lt = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
       TileInfo ti;
-      if (!decode_tile<NT>(a, tile, ti)) continue;
+      if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
       const uint32_t buf = lt & 1, use = lt >> 1;
       if (!mbar_wait_backoff(&acc_full[buf], use & 1)) { fail(6); break; }
       tc_fence_after();
@@ -210,6 +211,18 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+bool make_tmap_records(CUtensorMap* map, const void* base, long n_records, int batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base || n_records <= 0 || batch < 1 || batch > 4) return false;
+  cuuint64_t dims[3] = {128, 36, (cuuint64_t)n_records};
+  cuuint64_t strides[2] = {128, 4608};
+  cuuint32_t box[3] = {128, 36, (cuuint32_t)batch};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int NT, int STAGES, typename TO, bool RELU2, bool QA>
