@@ -136,6 +136,23 @@ def _oracle_sample(cfg, W, x, n_tok):
     return n_tok / dt, dt
 
 
+def _measured_traffic(cfg, n_touched):
+    """DRAM bytes per grouped-GEMM launch from the committed ncu capture, scaled
+    by touched experts; None when the kernel sources changed since the capture
+    or the workload is not the dense-bf16 decode the capture covers."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "umma_gemm_traffic.json")
+    if cfg.dtype != "bf16" or cfg.expert_fmt != "dense" or not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256()
+    for f in d["source_files"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != d["source_sha256"]:
+        return None
+    return d["dram_bytes_per_touched_expert"] * n_touched
+
+
 def _cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -305,7 +322,8 @@ def run_ours(a):
                 "peak_source": f"{src} (sustained bf16)", "flops_per_launch": fl}
     else:
         roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": hbm,
-                "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": _measured_traffic(cfg, n_touched),
                 "peak_source": src, "bytes_per_launch": (b_up + b_dn) / 2}
     if rank == 0:
         clk_s = clk.summary()
