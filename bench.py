@@ -100,10 +100,8 @@ class Clocks:
 
 
 def _dist():
-    rank = int(os.environ.get("RANK", 0))
-    world = int(os.environ.get("WORLD_SIZE", 1))
-    local = int(os.environ.get("LOCAL_RANK", 0))
-    return rank, world, local
+    from latentmoe_expert_routing_b200 import dist as D
+    return D.env_ranks()
 
 
 def _expert_bytes(cfg, n_touched):
@@ -210,13 +208,10 @@ def _weights(cfg, dev):
 
 def run_ours(a):
     import torch
-    import torch.distributed as dist
+    from latentmoe_expert_routing_b200 import dist as D
     rank, world, local = _dist()
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+    D.init("nccl", 300, torch.device("cuda", local))
     from latentmoe_expert_routing_b200 import binding as B
     from latentmoe_expert_routing_b200 import inputs as I
     from latentmoe_expert_routing_b200 import layer as LY
@@ -235,9 +230,7 @@ def run_ours(a):
     def step():
         lay(x, out, idx, wts)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = D.barrier
 
     clk = Clocks(local).__enter__()          # sampling from warm-up on: GPU under load
     for _ in range(max(a.warmup, 3)):
@@ -255,11 +248,7 @@ def run_ours(a):
     clk.__exit__()
     barrier()
     lay.sync()
-    ms = e0.elapsed_time(e1) / a.steps
-    ms_t = torch.tensor([ms], device="cuda")
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = D.max_over_ranks(e0.elapsed_time(e1) / a.steps, "cuda")
 
     # per-stage durations (CUDA events recorded by the library on this stream)
     B.moe_profile_enable(lay.handle, 1)
@@ -287,10 +276,7 @@ def run_ours(a):
         lay.forward_host(xh, oh)
     h1.record(st)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([h0.elapsed_time(h1) / a.steps], device="cuda")
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = D.max_over_ranks(h0.elapsed_time(h1) / a.steps, "cuda")
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -328,7 +314,7 @@ def run_ours(a):
     if rank == 0:
         clk_s = clk.summary()
         line = {
-            "metric": METRIC, "value": world * T / (ms_max * 1e-3), "unit": UNIT,
+            "metric": METRIC, "value": D.job_throughput(T, world, ms_max * 1e-3), "unit": UNIT,
             "n_gpus": world, "steps": a.steps, "warmup": max(a.warmup, 3),
             "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
@@ -347,16 +333,14 @@ def run_ours(a):
             "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,
             "clocks": clk_s,
             "gpu_launches": 10 * a.steps,
-            "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
+            "e2e": {"value": D.job_throughput(T, world, e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": T * cfg.D * es,
                     "d2h_bytes_per_step": T * cfg.D * es},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
     del lay
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    D.finish()
     return 0
 
 

@@ -201,6 +201,13 @@ moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int row
 moe_status moe_get_router_stats(moe_handle* handle, unsigned long long* exact_logits,
                                 void* stream);
 
+/* Self-test of device-side failure reporting: launches one bounded wait on a
+ * device flag that nothing sets.  The wait gives up after `microseconds`
+ * (at most 1 s) and records a timeout in the device error word, so the next
+ * moe_sync() returns MOE_ERR_TIMEOUT; the context stays usable.  Every
+ * pipeline wait inside the library's kernels is bounded the same way. */
+moe_status moe_selftest_wait_timeout(moe_handle* handle, int microseconds, void* stream);
+
 /* Drain `stream` and report (then clear) the device error word. */
 moe_status moe_sync(moe_handle* handle, void* stream);
 

@@ -60,6 +60,7 @@ SIGNATURES = [
                                _vp, _vp, _vp]),
     ("moe_quantize_nvfp4", _i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     ("moe_get_router_stats", _i, [_vp, _p(ctypes.c_ulonglong), _vp]),
+    ("moe_selftest_wait_timeout", _i, [_vp, _i, _vp]),
     ("moe_sync", _i, [_vp, _vp]),
     ("moe_destroy", None, [_vp]),
     ("moe_status_string", ctypes.c_char_p, [_i]),

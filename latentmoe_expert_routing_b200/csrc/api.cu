@@ -33,6 +33,9 @@ struct moe_handle {
   // tensor-core path (bf16): permuted latent rows and cached TMA maps
   void* z_perm = nullptr;
   float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
+  float* splitws = nullptr;                      // split-K partials of the dense GEMMs
+  size_t splitws_elems = 0;
+  int sms = 148;
   uint32_t* cmask = nullptr;                     // [T, 32] candidate bits per token
   // NVFP4 experts: GEMM-layout records and per-expert global scales
   uint8_t *rec_up = nullptr, *rec_dn = nullptr;
@@ -47,7 +50,48 @@ struct moe_handle {
 
 namespace {
 
+// Self-test: one bounded wait on a device flag that nothing sets.  The wait
+// gives up after `cycles` SM clocks and records DEV_ERR_TIMEOUT in the error
+// word, the same way the GEMM pipelines report a wait that ran out.
+__global__ void selftest_wait_kernel(const volatile int* flag, long long cycles, int* err) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const long long t0 = clock64();
+  while (*flag == 0) {
+    if (clock64() - t0 > cycles) {
+      atomicOr(err, DEV_ERR_TIMEOUT);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
 const int kNT[3] = {16, 64, 256};
+const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K partials
+
+// Dense tensor-core GEMM with split-K when its output tiles cannot fill the
+// SMs (decode-sized T): slices write fp32 partials, a fixed-order reduce applies
+// the epilogue.  g.args.{K0,K1,n_out,ldo,M,out}, g.nt, g.epi and the maps are set.
+moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s) {
+  const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
+  const int steps = (g.args.K0 + g.args.K1) / 64;
+  int S = 1;
+  while (tiles * S < h->sms && steps % (2 * S) == 0 && steps / (2 * S) >= 2 &&
+         (size_t)(2 * S) * g.args.M * g.args.n_out <= h->splitws_elems)
+    S *= 2;
+  g.args.ksplit = S;
+  g.args.dense_tiles = tiles * S;
+  g.max_tiles = tiles * S;
+  if (S == 1) return launch_umma(g, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const UmmaEpi epi = g.epi;
+  void* out = g.args.out;
+  g.epi = UMMA_EPI_F32;
+  g.args.out = h->splitws;
+  g.args.ldo = g.args.n_out;
+  g.args.split_stride = (long)g.args.M * g.args.n_out;
+  if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_split_reduce(h->splitws, S, g.args.M, g.args.n_out, out, epi, s) == cudaSuccess
+             ? MOE_OK : MOE_ERR_CUDA;
+}
 
 int nt_index(long rows_per_group) { return rows_per_group <= 16 ? 0 : rows_per_group <= 64 ? 1 : 2; }
 
@@ -143,6 +187,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   const int di = nt_index(T), gi = nt_index(P / E);
   const int ntd = kNT[di], ntg = kNT[gi];
   cudaError_t e;
+  moe_status st;
 
   UmmaLaunch g{};
   g.args.err = h->err;
@@ -158,12 +203,12 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
   g.args.out = h->z; g.epi = w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
   g.max_tiles = g.args.dense_tiles;
-  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
   g.wmap0 = h->wm_su;
   g.args.n_out = Fs; g.args.ldo = Fs;
   g.args.dense_tiles = ceil_div(Fs, 128) * ceil_div(T, ntd);
   g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
-  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
   mark(MOE_STAGE_EXPERT_UP);
 
   // step 6: routed experts on permuted latent rows (grouped by expert)
@@ -204,7 +249,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   g.args.dense_tiles = ceil_div(D, 128) * ceil_div(T, ntd);
   g.args.out = out; g.epi = c.out_dtype == MOE_BF16 ? UMMA_EPI_BF16 : UMMA_EPI_F32;
   g.max_tiles = g.args.dense_tiles;
-  if ((e = launch_umma(g, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
   return MOE_OK;
 }
 
@@ -295,7 +340,10 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
       moe_destroy(h);
       return MOE_ERR_UNSUPPORTED;
     }
-    if (!dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
+    cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+    h->splitws_elems = kSplitWsElems;
+    if (!dev_alloc(h, &h->splitws, h->splitws_elems * 4) ||
+        !dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
         !dev_alloc(h, &h->cmask, T * 32 * 4) ||
         !dev_alloc(h, &h->stats, 16)) {
       moe_destroy(h);
@@ -359,7 +407,8 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
     g.args.K0 = D; g.args.n_out = E; g.args.ldo = E;
     g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt);
     g.args.out = h->logits; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
-    if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+    moe_status ls = launch_dense_umma(h, g, s);
+    if (ls != MOE_OK) return ls;
   } else {
     launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
   }
@@ -383,7 +432,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
                 h->stats};
-    launch_route_certified(ra, ca, s);
+    launch_route_fused(ra, ca, s);
   } else {
     launch_route(ra, s);
   }
@@ -523,6 +572,19 @@ moe_status moe_get_router_stats(moe_handle* h, unsigned long long* exact_logits,
       cudaStreamSynchronize(s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(moe_handle* h, int microseconds, void* stream) {
+  if (!h || microseconds < 0 || microseconds > 1000000) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  int* flag = h->err + 1;                        // second word of the error block: stays 0
+  if (cudaMemsetAsync(flag, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  int dev = 0, khz = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+  const long long cycles = (long long)khz * 1000LL / 1000000LL * microseconds;
+  selftest_wait_kernel<<<1, 32, 0, s>>>(flag, cycles, h->err);
+  return cuda_status(cudaGetLastError());
 }
 
 moe_status moe_sync(moe_handle* h, void* stream) {

@@ -45,6 +45,7 @@ struct CertArgs {
   unsigned long long* stats;  // += number of exactly recomputed logits (or NULL)
 };
 void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
+void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
 void launch_row_norms(const void* w, int rows, int D, float* out, cudaStream_t st);
 
 // Row-streaming GEMMs:  out[m, n] = epi( sum_s sum_k A_s[m, k] * W_s[n, k] ).
@@ -110,6 +111,9 @@ struct UmmaArgs {
   const uint8_t* wq;        // NVFP4 weight records (GEMM layout) or NULL: weights via wmap0
   int wq_mblks;             // 128-row blocks per weight matrix (NVFP4)
   const float* gscale;      // [E] per-group output scale (NVFP4 global scale) or NULL
+  int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
+                            // fp32 partials out[slice][row][n] (slice stride below)
+  long split_stride;        // elements between slices of the partial output
 };
 // epilogues; _Q variants round the output through NVFP4 in 16-column blocks
 enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2,
@@ -126,6 +130,9 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
 // NVFP4 GEMM records (4608 B each) as a 3-D uint8 tensor, box = `batch` records
 bool make_tmap_records(CUtensorMap* map, const void* base, long n_records, int batch);
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
+// out[r][n] = epi(sum_s ws[s][r][n]) for s = 0..S-1 in order (split-K reduce)
+cudaError_t launch_split_reduce(const float* ws, int S, int M, int N, void* out, UmmaEpi epi,
+                                cudaStream_t st);
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
                                   uint8_t* codes, uint8_t* scales, float* gscale,

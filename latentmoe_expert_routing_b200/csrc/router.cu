@@ -53,7 +53,7 @@ router_logits_kernel(const T* __restrict__ x, const T* __restrict__ wg,
 }
 
 // ---------------------------------------------------------------------------
-// exp in fp64 from IEEE +, *, rint and scalbn only: a = n ln2 + r with a
+// exp in fp64 from IEEE +, *, rint and an exact power-of-two multiply: a = n ln2 + r with a
 // two-part (Cody-Waite) ln 2 whose high part has 32 significant bits, then the
 // degree-13 Taylor polynomial of exp(r) by Horner.  The explicit _rn
 // intrinsics keep the compiler from contracting a*b+c into an FMA, so the
@@ -73,7 +73,9 @@ __device__ __forceinline__ double exp_fixed(double a) {
   double p = c[13];
 #pragma unroll
   for (int i = 12; i >= 0; --i) p = __dadd_rn(__dmul_rn(p, r), c[i]);
-  return scalbn(p, (int)n);
+  // p * 2^n with 2^n built from its exponent bits: |n| <= 116 keeps both 2^n and
+  // the product normal, so the multiply is exact (the same value scalbn gives)
+  return __dmul_rn(p, __longlong_as_double((long long)((int)n + 1023) << 52));
 }
 
 __device__ __forceinline__ float sigmoid_fixed(float l) {
@@ -345,8 +347,30 @@ constexpr double kCertEps = 0x1p-19;     // sigmoid/add rounding of c~, generous
 __device__ __forceinline__ float exact_logit_warp(const __nv_bfloat16* __restrict__ xr,
                                                   const __nv_bfloat16* __restrict__ wr,
                                                   int D, int lane) {
+  // Loads are issued four iterations ahead of the additions (memory-level
+  // parallelism); the additions keep the defined order (k ascending per lane).
   double acc = 0.0;
-  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
+  int k0 = 8 * lane;
+  for (; k0 + 3 * 256 < D; k0 += 4 * 256) {
+    uint4 xu[4], wu[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      xu[u] = *reinterpret_cast<const uint4*>(xr + k0 + u * 256);
+      wu[u] = __ldg(reinterpret_cast<const uint4*>(wr + k0 + u * 256));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xu[u]);
+      const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wu[u]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 xf = __bfloat1622float2(xh[q]), wf = __bfloat1622float2(wh[q]);
+        acc = fma((double)xf.x, (double)wf.x, acc);
+        acc = fma((double)xf.y, (double)wf.y, acc);
+      }
+    }
+  }
+  for (; k0 < D; k0 += 256) {
     float xv[8], wv[8];
     load8(xr + k0, xv);
     load8(wr + k0, wv);
@@ -484,6 +508,155 @@ void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t 
   else if (epl <= 8) route_cert_epl<8>(a, c, st);
   else if (epl <= 16) route_cert_epl<16>(a, c, st);
   else route_cert_epl<32>(a, c, st);
+  route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
+                                        a.offsets, a.mt_up, a.nc_up, a.tiles_up,
+                                        a.mt_dn, a.nc_dn, a.tiles_dn);
+  const long P = (long)a.T * a.k;
+  route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
+      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+}
+
+}  // namespace lmoe
+
+namespace lmoe {
+
+// ---------------------------------------------------------------------------
+// Certified router, fused: one CTA per token, thread e <-> expert e.
+//   1. ||x_t||, choice-score intervals [c~ - d, c~ + d] from the tensor-core logit
+//   2. tau = k-th largest lower bound: bitwise search over order-preserving keys
+//      of the lower bounds rounded down to fp32 (rounding down can only lower
+//      tau, which only adds candidates), one __syncthreads_count per bit
+//   3. candidates (upper bound >= tau) get the defined fixed-order fp64 logit,
+//      computed by the CTA's warps in parallel
+//   4. exact rank among candidates by counting (score desc, index asc); slot j =
+//      rank j; weights from the raw scores summed in slot order
+// Ranks within 32-token blocks for the grouping come from route_ranks_kernel.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t f32_order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float f32_from_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__global__ void __launch_bounds__(1024)
+route_fused_kernel(RouteArgs a, CertArgs ca) {
+  __shared__ float s_red[32];
+  __shared__ int s_cand[1024];
+  __shared__ float s_s[1024], s_c[1024];
+  __shared__ float s_rsel[kMaxTopK];
+  __shared__ int s_nc;
+  const int t = blockIdx.x, e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int E = a.E, k = a.k, D = ca.D, nw = blockDim.x >> 5;
+  const __nv_bfloat16* xr = ca.x + (size_t)t * D;
+
+  // 1. ||x_t||^2 (fp32 partial sums, inflated below) and the score intervals
+  float ss = 0.f;
+  for (int k0 = 8 * e; k0 < D; k0 += 8 * blockDim.x) {
+    float xv[8];
+    load8(xr + k0, xv);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) ss = fmaf(xv[r], xv[r], ss);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (lane == 0) s_red[warp] = ss;
+  if (e == 0) s_nc = 0;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < nw; ++w) tot += s_red[w];
+  const double u = 0x1p-23, Ku = D * u;
+  const double g = kCertMargin * Ku / (1.0 - Ku);
+  const double dscale = 0.25 * g * sqrt((double)tot) * (1.0 + 0x1p-9);
+  double cu = -INFINITY, lo = -INFINITY;
+  if (e < E) {
+    const double c = (double)__fadd_rn(sigmoid_fixed(a.logits[(size_t)t * E + e]), a.bias[e]);
+    const double d = dscale * ca.wnorm[e] + kCertEps;
+    cu = c + d;
+    lo = c - d;
+  }
+  // 2. tau: the largest key K with #{lower-bound keys >= K} >= k
+  const uint32_t key = e < E ? f32_order_key(__double2float_rd(lo)) : 0u;
+  uint32_t K = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t trial = K | (1u << bit);
+    if (__syncthreads_count(key >= trial) >= k) K = trial;
+  }
+  const double tau = (double)f32_from_key(K);
+  // 3. candidates, compacted, then exact logits (one warp per candidate)
+  const bool cand = e < E && cu >= tau;
+  const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+  int base = 0;
+  if (lane == 0 && bal) base = atomicAdd(&s_nc, __popc(bal));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  if (cand) s_cand[base + __popc(bal & ((1u << lane) - 1u))] = e;
+  __syncthreads();
+  const int nc = s_nc;
+  for (int i = warp; i < nc; i += nw) {
+    const int ce = s_cand[i];
+    const float l = exact_logit_warp(xr, ca.wg + (size_t)ce * D, D, lane);
+    if (lane == 0) {
+      const float sv = sigmoid_fixed(l);
+      s_s[ce] = sv;
+      s_c[ce] = __fadd_rn(sv, a.bias[ce]);
+    }
+  }
+  __syncthreads();
+  // 4. exact ranks among the candidates
+  if (cand) {
+    const float c = s_c[e];
+    int rank = 0;
+    for (int i = 0; i < nc; ++i) {
+      const int o = s_cand[i];
+      const float oc = s_c[o];
+      rank += (oc > c || (oc == c && o < e)) ? 1 : 0;
+    }
+    if (rank < k) {
+      a.topk_idx[(size_t)t * k + rank] = e;
+      s_rsel[rank] = s_s[e];
+    }
+  }
+  __syncthreads();
+  if (e == 0) {
+    float S = 0.f;
+    for (int j = 0; j < k; ++j) S = __fadd_rn(S, s_rsel[j]);
+    s_red[0] = __fadd_rn(S, 1e-20f);
+    if (ca.stats) atomicAdd(ca.stats, (unsigned long long)nc);
+  }
+  __syncthreads();
+  if (e < k) a.topk_w[(size_t)t * k + e] = __fmul_rn(__fdiv_rn(s_rsel[e], s_red[0]), a.rsf);
+}
+
+// Ranks of each token among its 32-token block's tokens that chose the same
+// expert, and per-block expert counts, from the selected indices.
+__global__ void __launch_bounds__(1024)
+route_ranks_kernel(RouteArgs a) {
+  extern __shared__ uint32_t mask[];                 // [E]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * 32 + warp;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) mask[e] = 0u;
+  __syncthreads();
+  if (t < a.T)
+    for (int j = lane; j < a.k; j += 32) {
+      const int e = a.topk_idx[(size_t)t * a.k + j];
+      if (e < 0 || e >= a.E) { atomicOr(a.err, DEV_ERR_INDEX); continue; }
+      atomicOr(&mask[e], 1u << warp);
+    }
+  __syncthreads();
+  if (t < a.T)
+    for (int j = lane; j < a.k; j += 32) {
+      const int e = a.topk_idx[(size_t)t * a.k + j];
+      if (e >= 0 && e < a.E) a.rank[(size_t)t * a.k + j] = __popc(mask[e] & ((1u << warp) - 1u));
+    }
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x)
+    a.blkcnt[(size_t)e * a.nblk + blockIdx.x] = __popc(mask[e]);
+}
+
+void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st) {
+  const int threads = ((a.E + 31) / 32) * 32;
+  route_fused_kernel<<<a.T, threads, 0, st>>>(a, c);
+  route_ranks_kernel<<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(a);
   route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
                                         a.offsets, a.mt_up, a.nc_up, a.tiles_up,
                                         a.mt_dn, a.nc_dn, a.tiles_dn);

@@ -38,6 +38,8 @@ struct TileInfo {
   int n0;          // first output column (weight row within the group)
   int a_row0;      // first A row (token / pair) of the tile
   int valid;       // A rows of the tile that belong to the group
+  int kb, ke;      // K steps [kb, ke) of this tile (split-K slice)
+  int slice;       // split-K slice index (0 without split)
 };
 
 // Grouped mode reads the tile and A-row offset tables from shared memory
@@ -56,6 +58,12 @@ template <int NT>
 __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, const int32_t* s_tiles,
                                             const int32_t* s_off, int tile, TileInfo& ti) {
   const int nmb = (a.n_out + kBM - 1) / kBM;
+  const int S = a.offsets ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
+  const int kt_all = (a.K0 + a.K1) / kBK;
+  ti.slice = tile % S;
+  ti.kb = ti.slice * (kt_all / S);
+  ti.ke = ti.kb + kt_all / S;
+  tile /= S;
   int e = 0, base = 0, cnt = a.M, local = tile;
   if (a.offsets) {
     int lo = 0, hi = a.E;

@@ -42,7 +42,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt0 = a.K0 / kBK, kt_all = kt0 + a.K1 / kBK;
+  const int kt0 = a.K0 / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -81,7 +81,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
-        for (int kt = 0; kt < kt_all; ++kt, ++it) {
+        for (int kt = ti.kb; kt < ti.ke; ++kt, ++it) {
           if (!mbar_wait(&empty[st], pe)) { fail(1); ok = false; break; }
           uint8_t* sp = smem + st * S::kStageBytes;
           mbar_arrive_expect_tx(&full[st], kWTileBytes + S::kATileBytes);
@@ -116,12 +116,12 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         tc_fence_after();
         const uint32_t d = tmem + buf * NT;
         bool ok = true;
-        for (int kt = 0; kt < kt_all; ++kt) {
+        for (int kt = ti.kb; kt < ti.ke; ++kt) {
           if (!mbar_wait(&full[st], pf)) { fail(4); ok = false; break; }
           tc_fence_after();
           const uint64_t wd = desc0 + (uint64_t)(st * (S::kStageBytes >> 4));
           const uint64_t ad = wd + (uint64_t)(kWTileBytes >> 4);
-          mma_bf16_ss(d, wd, ad, idesc, kt > 0 ? 1u : 0u);
+          mma_bf16_ss(d, wd, ad, idesc, kt > ti.kb ? 1u : 0u);
           mma_bf16_ss(d, wd + 2, ad + 2, idesc, 1u);
           mma_bf16_ss(d, wd + 4, ad + 4, idesc, 1u);
           mma_bf16_ss(d, wd + 6, ad + 6, idesc, 1u);
@@ -162,7 +162,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
             if (a.gscale) v = __fmul_rn(v, gs);
             if (RELU2) v = relu2(v);
             if (QA) v = nvfp4_roundtrip16(col_ok ? v : 0.f);
-            if (col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
+            if (col_ok)
+              store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
           }
         }
       }
@@ -264,6 +265,59 @@ cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st) {
     case 256: return umma_launch_nt<256, 4>(L, st);
   }
   return cudaErrorInvalidValue;
+}
+
+// Split-K reduce: one thread per 16 consecutive output columns of a row, slices
+// summed in order (deterministic), then the epilogue of the unsplit GEMM.
+template <typename TO, bool RELU2, bool QA>
+__global__ void split_reduce_kernel(const float* __restrict__ ws, int S, int M, int N,
+                                    TO* __restrict__ out) {
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nb = N / 16;
+  if (b >= (long)M * nb) return;
+  const int r = (int)(b / nb), c0 = (int)(b - (long)r * nb) * 16;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(ws + ((size_t)s * M + r) * N + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t = p[q];
+      v[4 * q] += t.x; v[4 * q + 1] += t.y; v[4 * q + 2] += t.z; v[4 * q + 3] += t.w;
+    }
+  }
+  if (RELU2) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = relu2(v[i]);
+  }
+  if (QA) {                                    // NVFP4 round trip of the 16-column block
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      v[i] = scale > 0.f ? __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v[i], scale))), scale) : 0.f;
+  }
+  TO* o = out + (size_t)r * N + c0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) store_out(o + i, v[i]);
+}
+
+cudaError_t launch_split_reduce(const float* ws, int S, int M, int N, void* out, UmmaEpi epi,
+                                cudaStream_t st) {
+  if (N % 16) return cudaErrorInvalidValue;
+  const long n = (long)M * (N / 16);
+  const int g = ceil_div(n, 256);
+  switch (epi) {
+    case UMMA_EPI_BF16: split_reduce_kernel<__nv_bfloat16, false, false><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
+    case UMMA_EPI_BF16_RELU2: split_reduce_kernel<__nv_bfloat16, true, false><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
+    case UMMA_EPI_F32: split_reduce_kernel<float, false, false><<<g, 256, 0, st>>>(ws, S, M, N, (float*)out); break;
+    case UMMA_EPI_BF16_Q: split_reduce_kernel<__nv_bfloat16, false, true><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
+    case UMMA_EPI_BF16_RELU2_Q: split_reduce_kernel<__nv_bfloat16, true, true><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
+  }
+  return cudaGetLastError();
 }
 
 // z_perm[p, :] = z[perm[p] / k, :]  (16 bytes per thread)
