@@ -37,6 +37,8 @@ def _args():
     ap.add_argument("--config", default="ultra_decode_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step eagerly instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -236,6 +238,16 @@ def run_ours(a):
     for _ in range(max(a.warmup, 3)):
         step()
     lay.sync()
+    eager_step = step
+    graph = None
+    if not a.no_graph:
+        # the whole forward (every library launch) captured once, replayed per step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        step = graph.replay
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -250,6 +262,7 @@ def run_ours(a):
     lay.sync()
     ms_max = D.max_over_ranks(e0.elapsed_time(e1) / a.steps, "cuda")
 
+    step = eager_step
     # per-stage durations (CUDA events recorded by the library on this stream)
     B.moe_profile_enable(lay.handle, 1)
     stages = []
@@ -322,6 +335,7 @@ def run_ours(a):
                        "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
                        "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
                        "parallelism": f"replicas{world}",
+                       "cuda_graph": graph is not None,
                        "l2": "no flush: each step streams the touched experts' weights "
                              f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
             "roofline": roof,
@@ -339,6 +353,7 @@ def run_ours(a):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line))
+    del graph
     del lay
     D.finish()
     return 0

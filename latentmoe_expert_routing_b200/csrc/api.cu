@@ -74,10 +74,17 @@ const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K part
 moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s) {
   const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
   const int steps = (g.args.K0 + g.args.K1) / 64;
+  // Pick the K split with the least modelled time: waves of the persistent grid
+  // times (steps per slice + a fixed per-tile cost of about two steps).
   int S = 1;
-  while (tiles * S < h->sms && steps % (2 * S) == 0 && steps / (2 * S) >= 2 &&
-         (size_t)(2 * S) * g.args.M * g.args.n_out <= h->splitws_elems)
-    S *= 2;
+  double best = 1e30;
+  for (int c = 1; c <= 64 && c <= steps; ++c) {
+    if (steps % c || (c > 1 && steps / c < 2)) continue;
+    if (c > 1 && (size_t)c * g.args.M * g.args.n_out > h->splitws_elems) continue;
+    const int waves = ceil_div((long)tiles * c, h->sms);
+    const double cost = waves * (steps / (double)c + 2.0) + (c > 1 ? 1.0 : 0.0);
+    if (cost < best - 1e-9) { best = cost; S = c; }
+  }
   g.args.ksplit = S;
   g.args.dense_tiles = tiles * S;
   g.max_tiles = tiles * S;
