@@ -43,7 +43,7 @@ struct moe_handle {
   float *gs_up = nullptr, *gs_dn = nullptr;
   unsigned long long* stats = nullptr;           // exactly recomputed logits
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
-  CUtensorMap am_zp[3], am_H[3], am_zc[3], am_hsh[3];   // token boxes of 16, 64, 256 rows
+  CUtensorMap am_zp[4], am_H[4], am_zc[4], am_hsh[4];   // token boxes of 16, 64, 256, 128 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
   cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
 };
@@ -65,7 +65,7 @@ __global__ void selftest_wait_kernel(const volatile int* flag, long long cycles,
   }
 }
 
-const int kNT[3] = {16, 64, 256};
+const int kNT[4] = {16, 64, 256, 128};
 const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K partials
 
 // Dense tensor-core GEMM with split-K when its output tiles cannot fill the
@@ -101,6 +101,13 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s) {
 }
 
 int nt_index(long rows_per_group) { return rows_per_group <= 16 ? 0 : rows_per_group <= 64 ? 1 : 2; }
+
+// Token rows per grouped-GEMM tile: NVFP4 experts keep their dequantised
+// weights in TMEM next to the accumulators, so their widest tile is 128 rows.
+int grouped_nt_index(const moe_config& c, long P) {
+  const int i = nt_index(P / c.n_experts);
+  return (c.expert_fmt != MOE_EXPERT_DENSE && i == 2) ? 3 : i;
+}
 
 size_t dt_size(moe_dtype d) { return d == MOE_BF16 ? 2 : 4; }
 
@@ -191,7 +198,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
   const int F = c.d_ff, Fs = c.d_ff_shared;
   const long P = (long)T * k;
-  const int di = nt_index(T), gi = nt_index(P / E);
+  const int di = nt_index(T), gi = grouped_nt_index(c, P);
   const int ntd = kNT[di], ntg = kNT[gi];
   cudaError_t e;
   moe_status st;
@@ -365,7 +372,7 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
              make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128) &&
              make_tmap_bf16(&h->wm_fc2, h->w_fc2, D, L, 128) &&
              make_tmap_bf16(&h->wm_sd, h->w_sd, D, Fs, 128);
-    for (int i = 0; i < 3 && m; ++i)
+    for (int i = 0; i < 4 && m; ++i)
       m = make_tmap_bf16(&h->am_zp[i], h->z_perm, P, L, kNT[i]) &&
           make_tmap_bf16(&h->am_H[i], h->H, P, F, kNT[i]) &&
           make_tmap_bf16(&h->am_zc[i], h->zc, T, L, kNT[i]) &&
@@ -426,7 +433,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
   ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
   if (dt == MOE_BF16) {           // tensor-core tiles: 128 weight rows x NT pairs
-    const int nt = kNT[nt_index((long)T * k / E)];
+    const int nt = kNT[grouped_nt_index(c, (long)T * k)];
     ra.mt_up = nt; ra.nc_up = ceil_div(F, 128);
     ra.mt_dn = nt; ra.nc_dn = ceil_div(L, 128);
   } else {

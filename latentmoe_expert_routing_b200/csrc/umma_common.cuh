@@ -151,6 +151,36 @@ __device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile,
   }
 }
 
+// NVFP4 record row r (both halves, k = 0..63) -> 32 packed bf16x2 words in k
+// order, each exactly q * s_b * 2^-26 (see dequant_half).
+__device__ __forceinline__ void dequant_row_regs(const uint8_t* rec, int r, uint32_t (&o)[32]) {
+  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
+      const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
+      const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const uint32_t x = words[2 * b + cc];
+        const int c = 4 * half + 2 * b + cc;            // chunk: k = 8c .. 8c+7
+        uint32_t p[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
+                         e2m1_pair_bits<3>(x)};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&p[j]);
+          v = __hmul2(v, s2);
+          o[4 * c + j] = *reinterpret_cast<uint32_t*>(&v);
+        }
+      }
+    }
+  }
+}
+
 // NVFP4 round trip of v across the 16-lane block it belongs to (global scale
 // 1): s_b = E4M3(amax / 6), q = E2M1(v / value(s_b)), returns q * value(s_b).
 __device__ __forceinline__ float nvfp4_roundtrip16(float v) {

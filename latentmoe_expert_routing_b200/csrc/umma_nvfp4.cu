@@ -2,22 +2,24 @@
 // NVFP4 format details; section 5.6 step 6).  Same tiling and orientation as
 // umma_gemm_kernel (128 weight rows x NT token rows, bf16 kind::f16 MMA into a
 // double-buffered TMEM accumulator); the weights arrive as 4608-byte NVFP4
-// records and are expanded to exact bf16 tiles in shared memory.
+// records and are expanded to exact bf16 rows directly in tensor memory, from
+// where the MMA reads its A operand ("TS" form).
 //
-// A record carries 3.5x fewer HBM bytes than the bf16 tile it becomes, so at the
-// HBM rate a pipeline step lasts only ~200 cycles.  Three rings, each deep
-// enough for its own latency, decouple the steps: records (RAW, HBM latency),
-// activation tiles (SA, TMA latency) and dequantised bf16 W tiles (SW, the
-// dequant -> MMA -> release loop).
+// A 64-K slice of NVFP4 weights is only 4.6 KB, while the single issuing thread
+// pays ~100 cycles per barrier wait and ~60-100 per commit or MMA on a loaded
+// SM; so a pipeline step is a batch of KS = 4 slices (K = 256, 16 MMAs per
+// wait/commit pair).  The dequantised W tiles live in TMEM (slots of 32*KS
+// columns next to the accumulators), which leaves shared memory for the record
+// batches (covering HBM latency) and the activation tiles.
 //
 // Warps (640 threads):
-//   0      record producer (1-D bulk copies into the raw ring)
+//   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
-//   2      activation producer (TMA tiles into the stage ring)
+//   2      activation producer (TMA tiles into the A ring)
 //   3      idle
 //   4-7    epilogue group 0 (even 8-column chunks of the accumulator)
-//   8-15   dequant: raw record -> swizzled bf16 W tile; four groups of two warps
-//          expand four pipeline steps concurrently (two rows per thread)
+//   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
+//          alternate steps; each thread expands one 64-element weight row
 //   16-19  epilogue group 1 (odd chunks)
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
@@ -27,35 +29,39 @@
 
 namespace lmoe {
 
-template <int NT, int SW, int SA, int RAW>
+constexpr int kMaxKS = 4;                    // 64-K slices per pipeline step
+
+template <int NT, int SA, int RAW>
 struct WqSmem {
-  static constexpr int kATileBytes = NT * kBK * 2;                     // multiple of 1024
-  static constexpr int kAOffset = SW * kWTileBytes;
-  static constexpr int kRawOffset = kAOffset + SA * kATileBytes;
-  static constexpr int kBarOffset = kRawOffset + RAW * kWqRecordBytes;
-  static constexpr int kTableOffset = kBarOffset + 1024;
+  static constexpr int kATileBytes = NT * kBK * 2;                     // one 64-K slice, multiple of 1024
+  static constexpr int kASlotBytes = kMaxKS * kATileBytes;             // one step
+  static constexpr int kRawSlotBytes = kMaxKS * kWqRecordBytes;        // one step's records
+  static constexpr int kRawOffset = SA * kASlotBytes;
+  static constexpr int kBarOffset = kRawOffset + RAW * kRawSlotBytes;
+  static constexpr int kTableOffset = kBarOffset + 1024;               // 128 barrier slots
   static constexpr int kBytes = kTableOffset + kTableBytes + 1024;     // + alignment
-  static constexpr uint32_t kTmemCols = 2 * NT < 32 ? 32 : 2 * NT;
+  static constexpr int kWCol0 = 2 * NT;                                // W slots after the accumulators
+  static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
 };
 
 constexpr int kWqThreads = 640;
-constexpr int kDqGroups = 4;                 // dequant groups working on different steps
-constexpr int kDqGroupThreads = 64;
+constexpr int kDqGroups = 2;                 // dequant groups working on alternate steps
+constexpr int kDqGroupThreads = 128;
 
-template <int NT, int SW, int SA, int RAW, typename TO, bool RELU2, bool QA>
+template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA>
 __global__ void __launch_bounds__(kWqThreads, 1)
 umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wqmap,
                const UmmaArgs a) {
-  using S = WqSmem<NT, SW, SA, RAW>;
+  using S = WqSmem<NT, SA, RAW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset); // A tile landed
   uint64_t* a_empty = a_full + SA;                                      // A slot free (MMA done)
-  uint64_t* w_ready = a_empty + SA;                                     // W tile written
-  uint64_t* w_empty = w_ready + SW;                                     // W slot free (MMA done)
-  uint64_t* raw_full = w_empty + SW;                                    // record landed
-  uint64_t* raw_empty = raw_full + RAW;                                 // record consumed
+  uint64_t* w_ready = a_empty + SA;                                     // W slot written (TMEM)
+  uint64_t* w_empty = w_ready + S::kMaxSW;                              // W slot free (MMA done)
+  uint64_t* raw_full = w_empty + S::kMaxSW;                             // record batch landed
+  uint64_t* raw_empty = raw_full + RAW;                                 // record batch consumed
   uint64_t* acc_full = raw_empty + RAW;                                 // [2]
   uint64_t* acc_empty = acc_full + 2;                                   // [2]
   uint64_t* mma_done = acc_empty + 2;
@@ -66,15 +72,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt_all = a.K0 / kBK;
-  // records move in batches of G consecutive steps (one bulk copy each); every
-  // tile has a multiple of G steps, so a batch never spans two tiles
-  const int G = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
-  const int NG = RAW / G;
+  // a step is KS consecutive 64-K slices (one record batch, one TMA); every
+  // tile has a multiple of KS slices
+  const int KS = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
+  const int nsteps = kt_all / KS;
+  const int SW = (512 - S::kWCol0) / (32 * KS);                        // W slots of 32*KS columns
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
     for (int s = 0; s < SW; ++s) { mbar_init(&w_ready[s], kDqGroupThreads); mbar_init(&w_empty[s], 1); }
-    for (int r = 0; r < RAW / G; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], G * kDqGroupThreads); }
+    for (int r = 0; r < RAW; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], kDqGroupThreads); }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 256); }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -83,7 +90,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     tma_prefetch_desc(&wqmap);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, S::kTmemCols);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   load_tables(a, s_tiles, s_off);
@@ -101,41 +108,42 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   if (warp == 0) {
     // ---------------- record producer ----------------
     if (lane == 0) {
-      uint32_t it = 0, gi = 0, pr = 1;           // batch slot, parity to wait for
+      uint32_t it = 0, rs = 0, pr = 1;           // step, slot, parity to wait for
       uint8_t* const raw0 = smem + S::kRawOffset;
-      const uint32_t bytes = G * kWqRecordBytes;
+      const uint32_t bytes = KS * kWqRecordBytes;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         int rec = (ti.grp * a.wq_mblks + ti.mblk) * kt_all;     // first record of the tile
         bool ok = true;
-        for (int kt = 0; kt < kt_all; kt += G, it += G, rec += G) {
-          if (!mbar_wait(&raw_empty[gi], pr)) { fail(11); ok = false; break; }
-          mbar_arrive_expect_tx(&raw_full[gi], bytes);
-          tma_load_3d(raw0 + gi * bytes, &wqmap, &raw_full[gi], 0, 0, rec);
-          if (++gi == (uint32_t)NG) { gi = 0; pr ^= 1; }
+        for (int st = 0; st < nsteps; ++st, ++it, rec += KS) {
+          if (!mbar_wait(&raw_empty[rs], pr)) { fail(11); ok = false; break; }
+          mbar_arrive_expect_tx(&raw_full[rs], bytes);
+          tma_load_3d(raw0 + rs * S::kRawSlotBytes, &wqmap, &raw_full[rs], 0, 0, rec);
+          if (++rs == (uint32_t)RAW) { rs = 0; pr ^= 1; }
         }
         if (!ok) break;
       }
-      const uint32_t nb = it / G, n = nb < (uint32_t)NG ? nb : (uint32_t)NG;
+      const uint32_t n = it < (uint32_t)RAW ? it : (uint32_t)RAW;
       for (uint32_t j = 0; j < n; ++j) {
-        const uint32_t i = nb - 1 - j;
-        if (!mbar_wait(&raw_full[i % NG], (i / NG) & 1)) { fail(12); break; }
+        const uint32_t i = it - 1 - j;
+        if (!mbar_wait(&raw_full[i % RAW], (i / RAW) & 1)) { fail(12); break; }
       }
     }
   } else if (warp == 2) {
     // ---------------- activation producer ----------------
     if (lane == 0) {
       uint32_t it = 0, sa = 0, pa = 1;
-      uint8_t* const a0 = smem + S::kAOffset;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
-        for (int kt = 0; kt < kt_all; ++kt, ++it) {
+        for (int st = 0; st < nsteps; ++st, ++it) {
           if (!mbar_wait(&a_empty[sa], pa)) { fail(13); ok = false; break; }
-          mbar_arrive_expect_tx(&a_full[sa], S::kATileBytes);
-          tma_load_2d(a0 + sa * S::kATileBytes, &amap, &a_full[sa], kt * kBK, ti.a_row0);
+          mbar_arrive_expect_tx(&a_full[sa], KS * S::kATileBytes);
+          uint8_t* dst = smem + sa * S::kASlotBytes;
+          for (int ks = 0; ks < KS; ++ks)
+            tma_load_2d(dst + ks * S::kATileBytes, &amap, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
           if (++sa == SA) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
@@ -147,13 +155,10 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // One thread; the loop is kept short (incremental slots and parities,
-    // descriptors advanced by constants) because its length sets the step rate.
+    // ---------------- MMA issuer (A from TMEM, B from shared memory) ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, NT);
-      const uint64_t wdesc0 = sw128_desc(smem_u32(smem));
-      const uint64_t adesc0 = sw128_desc(smem_u32(smem + S::kAOffset));
+      const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
       uint32_t sa = 0, pa = 0, sw = 0, pw = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
@@ -163,15 +168,17 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         tc_fence_after();
         const uint32_t d = tmem + buf * NT;
         bool ok = true;
-        for (int kt = 0; kt < kt_all; ++kt) {
+        for (int st = 0; st < nsteps; ++st) {
           if (!mbar_wait(&a_full[sa], pa) || !mbar_wait(&w_ready[sw], pw)) { fail(16); ok = false; break; }
           tc_fence_after();
-          const uint64_t wd = wdesc0 + (uint64_t)(sw * (kWTileBytes >> 4));
-          const uint64_t ad = adesc0 + (uint64_t)(sa * (S::kATileBytes >> 4));
-          mma_bf16_ss(d, wd, ad, idesc, kt > 0 ? 1u : 0u);
-          mma_bf16_ss(d, wd + 2, ad + 2, idesc, 1u);
-          mma_bf16_ss(d, wd + 4, ad + 4, idesc, 1u);
-          mma_bf16_ss(d, wd + 6, ad + 6, idesc, 1u);
+          uint32_t wt = tmem + S::kWCol0 + sw * 32 * KS;
+          uint64_t bd = bdesc0 + (uint64_t)(sa * (S::kASlotBytes >> 4));
+          for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
+            mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
+            mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
+            mma_bf16_ts(d, wt + 16, bd + 4, idesc, 1u);
+            mma_bf16_ts(d, wt + 24, bd + 6, idesc, 1u);
+          }
           mma_commit(&a_empty[sa]);          // both slots free once these MMAs finish
           mma_commit(&w_empty[sw]);
           if (++sa == SA) { sa = 0; pa ^= 1; }
@@ -185,29 +192,30 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       if (!mbar_wait(mma_done, 0)) fail(17);
     }
   } else if (warp >= 8 && warp < 16) {
-    // ---------------- dequant: 4 groups of 2 warps, group g owns steps it % 4 == g ----------------
-    const int t = threadIdx.x - 256;
-    const int g = t / kDqGroupThreads, gt = t % kDqGroupThreads;   // 64 threads, 2 rows each
+    // ---------------- dequant: records -> TMEM W slots ----------------
+    const int g = (warp - 8) >> 2, q = warp & 3;
+    const int r = 32 * q + lane;                 // weight row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + S::kWCol0;
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
       TileInfo ti;
       if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
       bool ok = true;
-      for (int kt = 0; kt < kt_all; ++kt, ++it) {
+      for (int st = 0; st < nsteps; ++st, ++it) {
         if ((int)(it % kDqGroups) != g) continue;
         const int sw = it % SW, rr = it % RAW;
-        const uint32_t bi = it / G;                  // batch of this step
-        if (!mbar_wait(&raw_full[bi % NG], (bi / NG) & 1) ||
-            !mbar_wait(&w_empty[sw], ((it / SW) & 1) ^ 1)) { fail(18); ok = false; break; }
-        const uint8_t* rec = smem + S::kRawOffset + rr * kWqRecordBytes;
-        uint8_t* wt = smem + sw * kWTileBytes;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {                // unit = (half, row); warps take 32 rows
-          const int u = q * kDqGroupThreads + gt;
-          dequant_half(rec, wt, u & 127, u >> 7);
+        if (!mbar_wait_sleep(&raw_full[rr], (it / RAW) & 1) ||
+            !mbar_wait_sleep(&w_empty[sw], ((it / SW) & 1) ^ 1)) { fail(18); ok = false; break; }
+        tc_fence_after();
+        const uint8_t* rec = smem + S::kRawOffset + rr * S::kRawSlotBytes;
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t o[32];
+          dequant_row_regs(rec + ks * kWqRecordBytes, r, o);
+          tmem_st32(lane_base + sw * 32 * KS + ks * 32, o);
         }
-        fence_proxy_async();                 // generic-proxy writes -> tensor-core reads
-        mbar_arrive(&raw_empty[bi % NG]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&raw_empty[rr]);
         mbar_arrive(&w_ready[sw]);
       }
       if (!ok) break;
@@ -222,7 +230,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       TileInfo ti;
       if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
       const uint32_t buf = lt & 1, use = lt >> 1;
-      if (!mbar_wait_backoff(&acc_full[buf], use & 1)) { fail(19); break; }
+      if (!mbar_wait_sleep(&acc_full[buf], use & 1)) { fail(19); break; }
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
@@ -252,19 +260,22 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, S::kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-template <int NT, int SW, int SA, int RAW, typename TO, bool RELU2, bool QA>
+template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA>
 static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
-  using S = WqSmem<NT, SW, SA, RAW>;
+  using S = WqSmem<NT, SA, RAW>;
   static_assert(S::kBytes <= 232448, "shared memory budget");
   // dequant groups work on up to kDqGroups steps at once: each ring needs at
   // least that many slots, or a waiter could target a phase two ahead (parity alias)
-  static_assert(SW >= kDqGroups && RAW >= kDqGroups, "ring too shallow for the dequant groups");
-  static_assert(RAW % 4 == 0 && RAW / 4 >= 2, "record ring holds whole batches of 1, 2 or 4");
-  auto kern = umma_wq_kernel<NT, SW, SA, RAW, TO, RELU2, QA>;
+  // dequant groups work on up to kDqGroups steps at once: each ring needs at
+  // least that many slots, or a waiter could target a phase two ahead (parity alias)
+  static_assert((512 - S::kWCol0) / (32 * kMaxKS) >= kDqGroups && RAW >= kDqGroups && SA >= 2,
+                "ring too shallow for the dequant groups");
+  static_assert(2 * SA + 2 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
+  auto kern = umma_wq_kernel<NT, SA, RAW, TO, RELU2, QA>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -280,42 +291,24 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NT, int SW, int SA, int RAW>
+template <int NT, int SA, int RAW>
 static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
   switch (L.epi) {
-    case UMMA_EPI_BF16: return wq_launch_t<NT, SW, SA, RAW, __nv_bfloat16, false, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, SW, SA, RAW, __nv_bfloat16, true, false>(L, st);
-    case UMMA_EPI_F32: return wq_launch_t<NT, SW, SA, RAW, float, false, false>(L, st);
-    case UMMA_EPI_BF16_Q: return wq_launch_t<NT, SW, SA, RAW, __nv_bfloat16, false, true>(L, st);
-    case UMMA_EPI_BF16_RELU2_Q: return wq_launch_t<NT, SW, SA, RAW, __nv_bfloat16, true, true>(L, st);
+    case UMMA_EPI_BF16: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, false>(L, st);
+    case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false>(L, st);
+    case UMMA_EPI_BF16_Q: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, true>(L, st);
+    case UMMA_EPI_BF16_RELU2_Q: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, true>(L, st);
   }
   return cudaErrorInvalidValue;
 }
 
-// Ring split for 16-token tiles (weight-streaming decode).  LMOE_WQ16_RINGS
-// selects an alternative split for tuning: 0 = default.
-static int wq16_variant() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("LMOE_WQ16_RINGS");
-    v = e ? atoi(e) : 0;
-  }
-  return v;
-}
-
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st) {
   if (L.args.K1 != 0 || !L.args.wq) return cudaErrorInvalidValue;
-  if (L.nt == 16) {
-    switch (wq16_variant()) {
-      case 1: return wq_launch_nt<16, 4, 8, 24>(L, st);     // 64 + 16 + 110 KB
-      case 2: return wq_launch_nt<16, 4, 8, 28>(L, st);     // 64 + 16 + 129 KB
-      default: break;
-    }
-  }
   switch (L.nt) {
-    case 16: return wq_launch_nt<16, 5, 16, 20>(L, st);     // 80 + 32 + 92 KB
-    case 64: return wq_launch_nt<64, 5, 12, 8>(L, st);      // 80 + 96 + 37 KB
-    case 256: return wq_launch_nt<256, 4, 3, 8>(L, st);     // 64 + 96 + 37 KB
+    case 16: return wq_launch_nt<16, 6, 8>(L, st);          // A 48 KB + records 147 KB
+    case 64: return wq_launch_nt<64, 3, 6>(L, st);          // A 96 KB + records 110 KB
+    case 128: return wq_launch_nt<128, 2, 4>(L, st);        // A 128 KB + records 74 KB
   }
   return cudaErrorInvalidValue;
 }
