@@ -33,6 +33,7 @@ struct moe_handle {
   // tensor-core path (bf16): permuted latent rows and cached TMA maps
   void* z_perm = nullptr;
   float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
+  float* wstat = nullptr;                        // max / min nonzero |w_gate[e]|
   float* splitws = nullptr;                      // split-K partials of the dense GEMMs
   size_t splitws_elems = 0;
   int sms = 148;
@@ -358,12 +359,13 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
     h->splitws_elems = kSplitWsElems;
     if (!dev_alloc(h, &h->splitws, h->splitws_elems * 4) ||
         !dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
+        !dev_alloc(h, &h->wstat, E * 8) ||
         !dev_alloc(h, &h->cmask, T * 32 * 4) ||
         !dev_alloc(h, &h->stats, 16)) {
       moe_destroy(h);
       return MOE_ERR_OOM;
     }
-    launch_row_norms(h->w_gate, (int)E, (int)D, h->wnorm, s);
+    launch_row_norms(h->w_gate, (int)E, (int)D, h->wnorm, h->wstat, s);
     cudaMemsetAsync(h->stats, 0, 16, s);
     bool m = make_tmap_bf16(&h->wm_gate, h->w_gate, E, D, 128) &&
              make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
@@ -445,7 +447,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.cmask = dt == MOE_BF16 ? h->cmask : nullptr;
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
-                h->stats};
+                h->stats, h->wstat};
     launch_route_fused(ra, ca, s);
   } else {
     launch_route(ra, s);

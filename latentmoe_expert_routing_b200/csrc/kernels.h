@@ -43,10 +43,10 @@ struct CertArgs {
   const float* wnorm;       // [E] ||w_e||_2 rounded up
   int D;
   unsigned long long* stats;  // += number of exactly recomputed logits (or NULL)
+  const float* wstat;       // [E][2] max |w_e|, min nonzero |w_e| (or NULL: double path)
 };
-void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
 void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
-void launch_row_norms(const void* w, int rows, int D, float* out, cudaStream_t st);
+void launch_row_norms(const void* w, int rows, int D, float* out, float* stat, cudaStream_t st);
 
 // Row-streaming GEMMs:  out[m, n] = epi( sum_s sum_k A_s[m, k] * W_s[n, k] ).
 constexpr int kRowsPerWarp = 4;                  // weight rows per warp

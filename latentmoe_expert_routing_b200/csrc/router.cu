@@ -382,138 +382,85 @@ __device__ __forceinline__ float exact_logit_warp(const __nv_bfloat16* __restric
   return __double2float_rn(__shfl_sync(0xffffffffu, acc, 0));
 }
 
-// Bounds and candidates: one warp per token; lane l handles experts l+32i.
-// Writes cmask[t][i] bit l = expert l+32i is a candidate.
-template <int EPL>
-__global__ void __launch_bounds__(256)
-route_bounds_kernel(RouteArgs a, CertArgs ca) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int E = a.E, k = a.k, D = ca.D;
-  if (t >= a.T) return;
-  const __nv_bfloat16* xr = ca.x + (size_t)t * D;
-  float ss = 0.f;                                   // ||x_t||^2, inflated below
-  for (int k0 = 8 * lane; k0 < D; k0 += 256) {
-    float xv[8];
-    load8(xr + k0, xv);
+// The same defined logit when every product x_k * w_k is exact in fp32 (two bf16
+// significands give at most 16 bits; exact for |product| in [2^-134, 2^127) or
+// zero): one fp32 multiply and one conversion per element instead of two.
+__device__ __forceinline__ float exact_logit_warp_f32prod(const __nv_bfloat16* __restrict__ xr,
+                                                          const __nv_bfloat16* __restrict__ wr,
+                                                          int D, int lane) {
+  double acc = 0.0;
+  int k0 = 8 * lane;
+  for (; k0 + 3 * 256 < D; k0 += 4 * 256) {
+    uint4 xu[4], wu[4];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) ss = fmaf(xv[r], xv[r], ss);
-  }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  const double u = 0x1p-23, Ku = D * u;
-  const double g = kCertMargin * Ku / (1.0 - Ku);
-  const double dscale = 0.25 * g * sqrt((double)ss) * (1.0 + 0x1p-10);
-  double c[EPL], d[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) {
-      c[i] = (double)__fadd_rn(sigmoid_fixed(a.logits[(size_t)t * E + e]), a.bias[e]);
-      d[i] = dscale * ca.wnorm[e] + kCertEps;
-    } else {
-      c[i] = -INFINITY;
-      d[i] = 0.0;
+    for (int u = 0; u < 4; ++u) {
+      xu[u] = *reinterpret_cast<const uint4*>(xr + k0 + u * 256);
+      wu[u] = __ldg(reinterpret_cast<const uint4*>(wr + k0 + u * 256));
     }
-  }
-  // tau = k-th largest lower bound c~ - d
-  uint32_t taken = 0u;
-  double tau = -INFINITY;
-  for (int j = 0; j < k; ++j) {
-    double best = -INFINITY;
-    int bi = -1;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken >> i & 1u) && (bi < 0 || c[i] - d[i] > best)) {
-        best = c[i] - d[i];
-        bi = i;
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xu[u]);
+      const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wu[u]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 xf = __bfloat1622float2(xh[q]), wf = __bfloat1622float2(wh[q]);
+        acc = __dadd_rn(acc, (double)__fmul_rn(xf.x, wf.x));
+        acc = __dadd_rn(acc, (double)__fmul_rn(xf.y, wf.y));
       }
     }
-    double wv = best;
-    int wl = bi >= 0 ? lane : 32;
+  }
+  for (; k0 < D; k0 += 256) {
+    float xv[8], wv[8];
+    load8(xr + k0, xv);
+    load8(wr + k0, wv);
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const double ov = __shfl_xor_sync(0xffffffffu, wv, off);
-      const int ol = __shfl_xor_sync(0xffffffffu, wl, off);
-      if (ol < 32 && (wl == 32 || ov > wv || (ov == wv && ol < wl))) { wv = ov; wl = ol; }
-    }
-    const int wbi = __shfl_sync(0xffffffffu, bi, wl & 31);
-    if (lane == wl) taken |= 1u << wbi;
-    tau = wv;
+    for (int r = 0; r < 8; ++r) acc = __dadd_rn(acc, (double)__fmul_rn(xv[r], wv[r]));
   }
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    const uint32_t b = __ballot_sync(0xffffffffu, e < E && c[i] + d[i] >= tau);
-    if (lane == 0) a.cmask[(size_t)t * EPL + i] = b;
-  }
+  for (int off = 16; off >= 1; off >>= 1) acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+  return __double2float_rn(__shfl_sync(0xffffffffu, acc, 0));
 }
 
-// Exact logits of the candidates: one warp per (token, 32-expert word); the
-// defined fixed-order fp64 value overwrites the tensor-core logit in place.
-template <int EPL>
-__global__ void __launch_bounds__(256)
-route_exact_kernel(RouteArgs a, CertArgs ca) {
-  const int lane = threadIdx.x & 31;
-  const long w = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (w >= (long)a.T * EPL) return;
-  const int t = (int)(w / EPL), i = (int)(w - (long)t * EPL);
-  uint32_t b = a.cmask[w];
-  if (lane == 0 && ca.stats && b) atomicAdd(ca.stats, (unsigned long long)__popc(b));
-  const __nv_bfloat16* xr = ca.x + (size_t)t * ca.D;
-  while (b) {
-    const int src = __ffs(b) - 1;
-    b &= b - 1;
-    const int e = src + 32 * i;
-    const float l = exact_logit_warp(xr, ca.wg + (size_t)e * ca.D, ca.D, lane);
-    if (lane == 0) const_cast<float*>(a.logits)[(size_t)t * a.E + e] = l;   // workspace
-  }
+// products of a row with magnitudes in [lo_a, hi_a] and one in [lo_b, hi_b] are
+// all exact in fp32 (zeros are exact anyway)
+__device__ __forceinline__ bool products_exact_f32(float hi_a, float lo_a, float hi_b, float lo_b) {
+  return (double)hi_a * (double)hi_b < 0x1p127 && (double)lo_a * (double)lo_b >= 0x1p-134;
 }
 
-// ||w_e||_2 of each gate row, fp64 sum of squares, rounded up to fp32.
+// ||w_e||_2 of each gate row (fp64 sum of squares, rounded up to fp32), and
+// the row's largest and smallest nonzero magnitudes (stat[2e], stat[2e+1]).
 __global__ void row_norms_kernel(const __nv_bfloat16* __restrict__ w, int rows, int D,
-                                 float* __restrict__ out) {
+                                 float* __restrict__ out, float* __restrict__ stat) {
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= rows) return;
   double ss = 0.0;
+  float mx = 0.f, mn = INFINITY;
   for (int k0 = 8 * lane; k0 < D; k0 += 256) {
     float v[8];
     load8(w + (size_t)r * D + k0, v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
+    for (int i = 0; i < 8; ++i) {
+      ss = fma((double)v[i], (double)v[i], ss);
+      const float av = fabsf(v[i]);
+      mx = fmaxf(mx, av);
+      if (av > 0.f) mn = fminf(mn, av);
+    }
   }
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if (lane == 0) out[r] = __double2float_ru(sqrt(ss) * (1.0 + 0x1p-20));
+  for (int off = 16; off >= 1; off >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  if (lane == 0) {
+    out[r] = __double2float_ru(sqrt(ss) * (1.0 + 0x1p-20));
+    if (stat) { stat[2 * r] = mx; stat[2 * r + 1] = mn; }
+  }
 }
 
-void launch_row_norms(const void* w, int rows, int D, float* out, cudaStream_t st) {
-  row_norms_kernel<<<ceil_div(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)w, rows, D, out);
-}
-
-template <int EPL>
-static void route_cert_epl(const RouteArgs& a, const CertArgs& c, cudaStream_t st) {
-  route_bounds_kernel<EPL><<<ceil_div(a.T, 8), 256, 0, st>>>(a, c);
-  route_exact_kernel<EPL><<<ceil_div((long)a.T * EPL, 8), 256, 0, st>>>(a, c);
-  route_launch_epl<EPL>(a, st);
-}
-
-void launch_route_certified(const RouteArgs& a, const CertArgs& c, cudaStream_t st) {
-  const int epl = (a.E + 31) / 32;
-  if (epl <= 1) route_cert_epl<1>(a, c, st);
-  else if (epl <= 2) route_cert_epl<2>(a, c, st);
-  else if (epl <= 4) route_cert_epl<4>(a, c, st);
-  else if (epl <= 8) route_cert_epl<8>(a, c, st);
-  else if (epl <= 16) route_cert_epl<16>(a, c, st);
-  else route_cert_epl<32>(a, c, st);
-  route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
-                                        a.offsets, a.mt_up, a.nc_up, a.tiles_up,
-                                        a.mt_dn, a.nc_dn, a.tiles_dn);
-  const long P = (long)a.T * a.k;
-  route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
-      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+void launch_row_norms(const void* w, int rows, int D, float* out, float* stat, cudaStream_t st) {
+  row_norms_kernel<<<ceil_div(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)w, rows, D, out, stat);
 }
 
 }  // namespace lmoe
@@ -551,21 +498,36 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
   const int E = a.E, k = a.k, D = ca.D, nw = blockDim.x >> 5;
   const __nv_bfloat16* xr = ca.x + (size_t)t * D;
 
-  // 1. ||x_t||^2 (fp32 partial sums, inflated below) and the score intervals
-  float ss = 0.f;
+  // 1. ||x_t||^2 (fp32 partial sums, inflated below), max |x|, min nonzero |x|,
+  //    and the score intervals
+  __shared__ float s_mx[32], s_mn[32];
+  float ss = 0.f, mx = 0.f, mn = INFINITY;
   for (int k0 = 8 * e; k0 < D; k0 += 8 * blockDim.x) {
     float xv[8];
     load8(xr + k0, xv);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) ss = fmaf(xv[r], xv[r], ss);
+    for (int r = 0; r < 8; ++r) {
+      ss = fmaf(xv[r], xv[r], ss);
+      const float ax = fabsf(xv[r]);
+      mx = fmaxf(mx, ax);
+      if (ax > 0.f) mn = fminf(mn, ax);
+    }
   }
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if (lane == 0) s_red[warp] = ss;
+  for (int off = 16; off >= 1; off >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  if (lane == 0) { s_red[warp] = ss; s_mx[warp] = mx; s_mn[warp] = mn; }
   if (e == 0) s_nc = 0;
   __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < nw; ++w) tot += s_red[w];
+  float tot = 0.f, xmax = 0.f, xmin = INFINITY;
+  for (int w = 0; w < nw; ++w) {
+    tot += s_red[w];
+    xmax = fmaxf(xmax, s_mx[w]);
+    xmin = fminf(xmin, s_mn[w]);
+  }
   const double u = 0x1p-23, Ku = D * u;
   const double g = kCertMargin * Ku / (1.0 - Ku);
   const double dscale = 0.25 * g * sqrt((double)tot) * (1.0 + 0x1p-9);
@@ -595,7 +557,10 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
   const int nc = s_nc;
   for (int i = warp; i < nc; i += nw) {
     const int ce = s_cand[i];
-    const float l = exact_logit_warp(xr, ca.wg + (size_t)ce * D, D, lane);
+    const bool fast = ca.wstat &&
+        products_exact_f32(xmax, xmin, ca.wstat[2 * ce], ca.wstat[2 * ce + 1]);
+    const float l = fast ? exact_logit_warp_f32prod(xr, ca.wg + (size_t)ce * D, D, lane)
+                         : exact_logit_warp(xr, ca.wg + (size_t)ce * D, D, lane);
     if (lane == 0) {
       const float sv = sigmoid_fixed(l);
       s_s[ce] = sv;
