@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "latentmoe.h"
+#include "umma_common.cuh"
 
 using namespace lmoe;
 
@@ -236,7 +237,10 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
   u.args.tiles = h->tiles_up; u.args.out = h->H;
   u.epi = w4a4 ? UMMA_EPI_BF16_RELU2_Q : UMMA_EPI_BF16_RELU2;
-  auto batch_idx = [](int kt) { return kt % 4 == 0 ? 2 : (kt % 2 == 0 ? 1 : 0); };
+  auto batch_idx = [ntg](int kt) {      // record map box = slices per step of the kernel
+    const int ks = wq_slices_per_step(kt, ntg);
+    return ks == 4 ? 2 : (ks == 2 ? 1 : 0);
+  };
   if (wq) {
     u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up;
     u.wqmap = h->rm_up[batch_idx(L / 64)];

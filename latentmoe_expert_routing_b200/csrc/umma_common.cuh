@@ -19,7 +19,17 @@ constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
 constexpr int kWTileBytes = kBM * kBK * 2;
 constexpr int kTableBytes = 2 * 4 * 1025 + 16;     // tiles[E+1], offsets[E+1], E <= 1024
 
-constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
+constexpr int kWqRecordBytes = 4608;
+
+// 64-K slices per pipeline step of the NVFP4 kernel: up to 4 dividing the
+// tile's K, and few enough that TMEM (512 columns) holds a W slot of 32*KS
+// columns per dequant group (two) next to the two accumulators (2*nt columns).
+// The host picks the record TMA box with the same rule.
+__host__ __device__ inline int wq_slices_per_step(int kt_all, int nt) {
+  int ks = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
+  while (ks > 1 && (512 - 2 * nt) / (32 * ks) < 2) ks >>= 1;
+  return ks;
+}      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
 
 template <int NT, int STAGES>
 struct UmmaSmem {
@@ -178,6 +188,24 @@ __device__ __forceinline__ void dequant_row_regs(const uint8_t* rec, int r, uint
         }
       }
     }
+  }
+}
+
+// NVFP4 round trip of 8 rows at once (v[j] = this lane's column of row j): the
+// same arithmetic as nvfp4_roundtrip16, written so the 8 rows' shuffles,
+// divisions and encodes are independent (instruction-level parallelism).
+__device__ __forceinline__ void nvfp4_roundtrip16x8(float (&v)[8]) {
+  float amax[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) amax[j] = fabsf(v[j]);
+#pragma unroll
+  for (int off = 1; off < 16; off <<= 1)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax[j] = fmaxf(amax[j], __shfl_xor_sync(0xffffffffu, amax[j], off));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax[j], 6.0f)));
+    v[j] = scale > 0.f ? __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v[j], scale))), scale) : 0.f;
   }
 }
 

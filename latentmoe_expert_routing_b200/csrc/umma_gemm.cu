@@ -154,17 +154,21 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         uint32_t r[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, r);
         tmem_ld_wait();
+        if (c * 8 >= ti.valid) continue;     // uniform across the warp
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[j] = __uint_as_float(r[j]);
+          if (a.gscale) v[j] = __fmul_rn(v[j], gs);
+          if (RELU2) v[j] = relu2(v[j]);
+          if (!col_ok) v[j] = 0.f;
+        }
+        if (QA) nvfp4_roundtrip16x8(v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int row = c * 8 + j;
-          if (row < ti.valid) {              // uniform across the warp
-            float v = __uint_as_float(r[j]);
-            if (a.gscale) v = __fmul_rn(v, gs);
-            if (RELU2) v = relu2(v);
-            if (QA) v = nvfp4_roundtrip16(col_ok ? v : 0.f);
-            if (col_ok)
-              store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
-          }
+          if (row < ti.valid && col_ok)
+            store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
         }
       }
       tc_fence_before();

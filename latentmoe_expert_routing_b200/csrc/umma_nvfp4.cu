@@ -19,7 +19,7 @@
 //   3      idle
 //   4-7    epilogue group 0 (even 8-column chunks of the accumulator)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
-//          alternate steps; each thread expands one 64-element weight row
+//          alternate steps; each thread expands its weight row's slices
 //   16-19  epilogue group 1 (odd chunks)
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
@@ -45,8 +45,14 @@ struct WqSmem {
 };
 
 constexpr int kWqThreads = 640;
-constexpr int kDqGroups = 2;                 // dequant groups working on alternate steps
+constexpr int kDqGroups = 2;                 // dequant groups taking alternate steps
 constexpr int kDqGroupThreads = 128;
+
+// dequant group of a warp (four warps per group, one per TMEM lane quarter):
+// warps 8-15 form groups 0-1; -1 for other roles
+__device__ __forceinline__ int dq_group(int warp) {
+  return (warp >= 8 && warp < 16) ? (warp - 8) >> 2 : -1;
+}
 
 template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA>
 __global__ void __launch_bounds__(kWqThreads, 1)
@@ -74,7 +80,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   const int kt_all = a.K0 / kBK;
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
   // tile has a multiple of KS slices
-  const int KS = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
+  const int KS = wq_slices_per_step(kt_all, NT);
   const int nsteps = kt_all / KS;
   const int SW = (512 - S::kWCol0) / (32 * KS);                        // W slots of 32*KS columns
 
@@ -191,9 +197,9 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       mma_commit(mma_done);
       if (!mbar_wait(mma_done, 0)) fail(17);
     }
-  } else if (warp >= 8 && warp < 16) {
+  } else if (dq_group(warp) >= 0) {
     // ---------------- dequant: records -> TMEM W slots ----------------
-    const int g = (warp - 8) >> 2, q = warp & 3;
+    const int g = dq_group(warp), q = warp & 3;
     const int r = 32 * q + lane;                 // weight row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + S::kWCol0;
     uint32_t it = 0;
@@ -220,7 +226,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       }
       if (!ok) break;
     }
-  } else if ((warp >= 4 && warp < 8) || warp >= 16) {
+  } else if ((warp >= 4 && warp < 8) || (warp >= 16 && warp < 20)) {
     // ---------------- epilogue (two groups split the accumulator's chunks) ----------------
     const int q = warp & 3;
     const int grp = warp >= 16 ? 1 : 0;
@@ -240,15 +246,18 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         uint32_t rg[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, rg);
         tmem_ld_wait();
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[j] = __fmul_rn(__uint_as_float(rg[j]), gs);
+          if (RELU2) v[j] = relu2(v[j]);
+          if (!col_ok) v[j] = 0.f;
+        }
+        if (QA) nvfp4_roundtrip16x8(v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int row = c * 8 + j;
-          if (row < ti.valid) {
-            float v = __fmul_rn(__uint_as_float(rg[j]), gs);
-            if (RELU2) v = relu2(v);
-            if (QA) v = nvfp4_roundtrip16(col_ok ? v : 0.f);
-            if (col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v);
-          }
+          if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
         }
       }
       tc_fence_before();
@@ -272,7 +281,7 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   // least that many slots, or a waiter could target a phase two ahead (parity alias)
   // dequant groups work on up to kDqGroups steps at once: each ring needs at
   // least that many slots, or a waiter could target a phase two ahead (parity alias)
-  static_assert((512 - S::kWCol0) / (32 * kMaxKS) >= kDqGroups && RAW >= kDqGroups && SA >= 2,
+  static_assert((512 - S::kWCol0) / 32 >= kDqGroups && RAW >= kDqGroups && SA >= 2,
                 "ring too shallow for the dequant groups");
   static_assert(2 * SA + 2 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
   auto kern = umma_wq_kernel<NT, SA, RAW, TO, RELU2, QA>;
