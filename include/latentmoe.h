@@ -208,6 +208,19 @@ moe_status moe_get_router_stats(moe_handle* handle, unsigned long long* exact_lo
  * pipeline wait inside the library's kernels is bounded the same way. */
 moe_status moe_selftest_wait_timeout(moe_handle* handle, int microseconds, void* stream);
 
+/* Self-test of the hardware NVFP4 conversions the W4A4 path relies on
+ * (NVFP4 format details: E2M1 elements, E4M3 block scales): on the current
+ * device, compares (1) the E2M1 round trip of every finite fp32 value by the
+ * hardware conversion (round to nearest, ties to even, saturating) with the
+ * library's encoder written from the format definition, as values (-0 == +0);
+ * (2) the hardware E2M1 -> fp16 expansion of all 256 code pairs and (3) the
+ * hardware E4M3 -> fp16 expansion of all 65536 scale pairs with the format's
+ * values.  Writes the number of disagreements (0 expected) to
+ * *mismatches_host and synchronises `stream`.  MOE_ERR_INVALID_ARG for a NULL
+ * pointer; MOE_ERR_OOM when the device counter cannot be allocated;
+ * MOE_ERR_CUDA on a launch or copy failure. */
+moe_status moe_selftest_nvfp4_convert(unsigned long long* mismatches_host, void* stream);
+
 /* Drain `stream` and report (then clear) the device error word. */
 moe_status moe_sync(moe_handle* handle, void* stream);
 

@@ -61,6 +61,7 @@ SIGNATURES = [
     ("moe_quantize_nvfp4", _i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     ("moe_get_router_stats", _i, [_vp, _p(ctypes.c_ulonglong), _vp]),
     ("moe_selftest_wait_timeout", _i, [_vp, _i, _vp]),
+    ("moe_selftest_nvfp4_convert", _i, [_vp, _vp]),
     ("moe_sync", _i, [_vp, _vp]),
     ("moe_destroy", None, [_vp]),
     ("moe_status_string", ctypes.c_char_p, [_i]),
@@ -146,6 +147,12 @@ def moe_quantize_nvfp4(w, dtype, n_mat, rows, K, codes, scales, gscale, stream):
 def moe_get_router_stats(h, stream) -> int:
     v = ctypes.c_ulonglong(0)
     _check(_lib.moe_get_router_stats(h, ctypes.byref(v), stream), "moe_get_router_stats")
+    return v.value
+
+
+def moe_selftest_nvfp4_convert(stream) -> int:
+    v = ctypes.c_ulonglong(0)
+    _check(_lib.moe_selftest_nvfp4_convert(ctypes.byref(v), stream), "moe_selftest_nvfp4_convert")
     return v.value
 
 

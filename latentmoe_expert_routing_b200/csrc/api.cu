@@ -172,14 +172,18 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
     cudaFree(codes); cudaFree(scales); cudaFree(amax);
     return MOE_ERR_OOM;
   }
+  // W4A4 streams fp16 operands: its records keep the plain nibble order
+  const int natural = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
   cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, codes, scales,
                                         h->gs_up, amax, s);
-  if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)F, (int)L, h->rec_up, s);
+  if (e == cudaSuccess)
+    e = launch_repack_gemm(codes, scales, (int)E, (int)F, (int)L, h->rec_up, natural, s);
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_up, h->gs_up, (int)E, s);
   if (e == cudaSuccess)
     e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, codes, scales, h->gs_dn,
                               amax, s);
-  if (e == cudaSuccess) e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, s);
+  if (e == cudaSuccess)
+    e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, natural, s);
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
   for (int i = 0; i < 3 && e == cudaSuccess; ++i)
     if (!make_tmap_records(&h->rm_up[i], h->rec_up, (long)recs_up, 1 << i) ||
@@ -228,15 +232,18 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   mark(MOE_STAGE_EXPERT_UP);
 
   // step 6: routed experts on permuted latent rows (grouped by expert)
-  launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
+  // (W4A4: z holds NVFP4 round-trip values, exact in fp16, the experts' operand type)
+  if (w4a4) launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, s);
+  else launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
   UmmaLaunch u{};
+  u.a_f16 = w4a4;
   u.args.err = h->err;
   u.args.E = E; u.args.offsets = h->offsets;
   u.nt = ntg;
   u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
   u.args.tiles = h->tiles_up; u.args.out = h->H;
-  u.epi = w4a4 ? UMMA_EPI_BF16_RELU2_Q : UMMA_EPI_BF16_RELU2;
+  u.epi = w4a4 ? UMMA_EPI_F16_RELU2_Q : UMMA_EPI_BF16_RELU2;
   auto batch_idx = [ntg](int kt) {      // record map box = slices per step of the kernel
     const int ks = wq_slices_per_step(kt, ntg);
     return ks == 4 ? 2 : (ks == 2 ? 1 : 0);
@@ -605,6 +612,19 @@ moe_status moe_selftest_wait_timeout(moe_handle* h, int microseconds, void* stre
   const long long cycles = (long long)khz * 1000LL / 1000000LL * microseconds;
   selftest_wait_kernel<<<1, 32, 0, s>>>(flag, cycles, h->err);
   return cuda_status(cudaGetLastError());
+}
+
+moe_status moe_selftest_nvfp4_convert(unsigned long long* mismatches_host, void* stream) {
+  if (!mismatches_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned long long* bad = nullptr;
+  if (cudaMalloc(&bad, sizeof(*bad)) != cudaSuccess) { cudaGetLastError(); return MOE_ERR_OOM; }
+  cudaError_t e = cudaMemsetAsync(bad, 0, sizeof(*bad), s);
+  if (e == cudaSuccess) e = launch_nvfp4_convert_check(bad, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(mismatches_host, bad, sizeof(*bad), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  cudaFree(bad);
+  return cuda_status(e);
 }
 
 moe_status moe_sync(moe_handle* h, void* stream) {

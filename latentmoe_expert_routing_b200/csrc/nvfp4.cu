@@ -11,7 +11,11 @@
 // past the matrix are zero.  Within a row, 32-bit word i holds
 // elements k = 8i..8i+7 with element 8i+2j in bits 4j..4j+3 and element
 // 8i+2j+1 in bits 16+4j..19+4j, so that one shift pair turns the word into a
-// bf16 pair (see the dequant in umma_gemm.cu).
+// bf16 pair (see the dequant in umma_common.cuh).  The W4A4 layout ("natural")
+// keeps the plain byte order instead (element 2i in the low nibble of byte i),
+// which the hardware E2M1 -> f16x2 conversion reads directly.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "nvfp4.cuh"
@@ -71,7 +75,8 @@ __global__ void quantize_blocks_kernel(const T* __restrict__ w, int n_mat, int r
 
 // plain layout -> GEMM layout
 __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                   int n_mat, int rows, int K, uint8_t* __restrict__ out) {
+                                   int n_mat, int rows, int K, int natural,
+                                   uint8_t* __restrict__ out) {
   const int nmb = (rows + 127) / 128, nks = K / 64;
   const long rec = (long)blockIdx.x;                 // one record per block, 128 threads = rows
   if (rec >= (long)n_mat * nmb * nks) return;
@@ -87,6 +92,7 @@ __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint
     const uint8_t* cp = codes + ((size_t)m * rows + row) * (K / 2) + ks * 32;
     for (int i = 0; i < 8; ++i) {
       const uint32_t b4 = *reinterpret_cast<const uint32_t*>(cp + 4 * i);   // bytes B0..B3
+      if (natural) { wd[i] = b4; continue; }
       uint32_t w = 0;
       for (int j = 0; j < 4; ++j) {
         const uint32_t bj = (b4 >> (8 * j)) & 0xFFu;
@@ -137,10 +143,74 @@ cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t 
 }
 
 cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
-                               int K, uint8_t* out, cudaStream_t st) {
+                               int K, uint8_t* out, int natural, cudaStream_t st) {
   const long recs = (long)n_mat * ((rows + 127) / 128) * (K / 64);
-  repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, out);
+  repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, natural, out);
   return cudaGetLastError();
+}
+
+// ---- self-test of the hardware conversions against the format definition ----
+// grid-stride over all 2^32 fp32 bit patterns (two per step, the pair the
+// hardware converts together), then all E2M1 bytes and E4M3 pairs.
+__global__ void nvfp4_convert_check_kernel(unsigned long long* bad) {
+  const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const uint64_t nth = (uint64_t)gridDim.x * blockDim.x;
+  unsigned long long n = 0;
+  for (uint64_t i = tid; i < (1ull << 31); i += nth) {
+    const uint32_t b0 = (uint32_t)(2 * i), b1 = b0 + 1;
+    const float y0 = __uint_as_float(b0), y1 = __uint_as_float(b1);
+    const uint32_t h = e2m1_round_f16x2(y0, y1);
+    const float r0 = __low2float(*reinterpret_cast<const __half2*>(&h));
+    const float r1 = __high2float(*reinterpret_cast<const __half2*>(&h));
+    if (!isnan(y0) && r0 != e2m1_value(e2m1_encode(y0))) ++n;
+    if (!isnan(y1) && r1 != e2m1_value(e2m1_encode(y1))) ++n;
+  }
+  if (tid < 256) {                        // E2M1 byte -> f16x2
+    uint32_t h[4];
+    e2m1x8_to_f16x2((uint32_t)tid, h);    // byte 0 = tid, bytes 1..3 = 0
+    const __half2 p = *reinterpret_cast<const __half2*>(&h[0]);
+    if (__low2float(p) != e2m1_value((uint32_t)tid & 15u)) ++n;
+    if (__high2float(p) != e2m1_value((uint32_t)tid >> 4)) ++n;
+  }
+  for (uint64_t i = tid; i < 65536; i += nth) {   // E4M3 pair -> f16x2 (finite codes)
+    const uint32_t c0 = (uint32_t)i & 0xFFu, c1 = (uint32_t)i >> 8;
+    const uint32_t h = e4m3x2_to_f16x2((uint32_t)i);
+    const __half2 p = *reinterpret_cast<const __half2*>(&h);
+    if ((c0 & 0x7Fu) != 0x7Fu && __low2float(p) != e4m3_value(c0)) ++n;
+    if ((c1 & 0x7Fu) != 0x7Fu && __high2float(p) != e4m3_value(c1)) ++n;
+  }
+  if (n) atomicAdd(bad, n);
+}
+
+cudaError_t launch_nvfp4_convert_check(unsigned long long* bad, cudaStream_t st) {
+  nvfp4_convert_check_kernel<<<4 * 148, 256, 0, st>>>(bad);
+  return cudaGetLastError();
+}
+
+// one thread per 8 elements of a permuted row
+__global__ void gather_rows_f16_kernel(const uint4* __restrict__ z, const int32_t* __restrict__ perm,
+                                       uint4* __restrict__ zp, long P, int k, int row_vecs) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= P * row_vecs) return;
+  const long p = i / row_vecs;
+  const int c = (int)(i - p * row_vecs);
+  const uint4 u = z[(long)(perm[p] / k) * row_vecs + c];
+  uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+    const __half2 h = __floats2half2_rn(f.x, f.y);
+    w[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  zp[i] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+void launch_gather_rows_f16(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
+                            cudaStream_t st) {
+  const int rv = L / 8;
+  const long n = P * rv;
+  if (n == 0) return;
+  gather_rows_f16_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)z, perm, (uint4*)zp, P, k, rv);
 }
 
 }  // namespace lmoe

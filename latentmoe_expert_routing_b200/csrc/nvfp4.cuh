@@ -52,4 +52,42 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return (code & 0x80u) ? -v : v;
 }
 
+// ---- hardware conversions (sm_100a) for the fp16 operand path --------------
+// Every E2M1 value and every E4M3 value is exactly an fp16 number, and so is
+// any product q * s_b of the two (at most 6 significant bits, magnitudes in
+// [2^-10, 2688], inside fp16's normal range), so these conversions and one
+// f16x2 multiply give exact dequantised values.
+
+// One 32-bit word of eight E2M1 codes, element 2i in the low nibble of byte i
+// -> four f16x2 words (element 2i in the low half of word i).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t x, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(x));
+}
+
+// Two E4M3 codes (the low byte first) -> f16x2 of their values.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t d;
+  const unsigned short t = (unsigned short)(two & 0xFFFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(t));
+  return d;
+}
+
+// E2M1 round trip of two fp32 values (round to nearest, ties to the even
+// code, saturating at 6: the same decisions as e2m1_encode) -> f16x2 of the
+// rounded values, y0 in the low half.
+__device__ __forceinline__ uint32_t e2m1_round_f16x2(float y0, float y1) {
+  uint32_t d;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(d) : "f"(y0), "f"(y1));
+  return d;
+}
+
 }  // namespace lmoe

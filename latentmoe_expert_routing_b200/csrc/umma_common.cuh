@@ -3,6 +3,7 @@
 // swizzled bf16 tiles, the NVFP4 activation round trip of the W4A4 epilogue.
 #pragma once
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -191,34 +192,56 @@ __device__ __forceinline__ void dequant_row_regs(const uint8_t* rec, int r, uint
   }
 }
 
-// NVFP4 round trip of 8 rows at once (v[j] = this lane's column of row j): the
-// same arithmetic as nvfp4_roundtrip16, written so the 8 rows' shuffles,
-// divisions and encodes are independent (instruction-level parallelism).
-__device__ __forceinline__ void nvfp4_roundtrip16x8(float (&v)[8]) {
-  float amax[8];
+// NVFP4 round trip (global scale 1) of this lane's 8 token values within the
+// 16-lane block of rows it belongs to, as f16x2 pairs (tokens 2p, 2p+1 in
+// h[p]; exact, q * s_b being an fp16 number): over the block, amax = max |v|,
+// s_b = E4M3(amax / 6) (fp32 division, nearest-even encode), then per value
+// q = E2M1(v / value(s_b)) (fp32 division; the E2M1 rounding is the hardware
+// conversion, which decides as e2m1_encode does) and the result q * s_b.  The 8 block maxima are reduced by halving exchanges (xor 8,
+// 4, 2, 1), after which lanes 2t and 2t+1 of the block hold token t's maximum;
+// they compute its scale once and the other lanes read it by shuffle.  Zero
+// numerators skip the division (0 / s = 0), whose slow path they would take.
+__device__ __forceinline__ void nvfp4_roundtrip16x8_h(const float (&v)[8], uint32_t (&h)[4]) {
+  const int lane = threadIdx.x & 31;
+  const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+  float m4[4], m2[2];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) amax[j] = fabsf(v[j]);
+  for (int i = 0; i < 4; ++i) {          // keep tokens 4*b3 + i, send the other four
+    const float lo = fabsf(v[i]), hi = fabsf(v[i + 4]);
+    m4[i] = fmaxf(b3 ? hi : lo, __shfl_xor_sync(0xffffffffu, b3 ? lo : hi, 8));
+  }
 #pragma unroll
-  for (int off = 1; off < 16; off <<= 1)
+  for (int i = 0; i < 2; ++i)            // tokens 4*b3 + 2*b2 + i
+    m2[i] = fmaxf(b2 ? m4[i + 2] : m4[i], __shfl_xor_sync(0xffffffffu, b2 ? m4[i] : m4[i + 2], 4));
+  float m1 = fmaxf(b1 ? m2[1] : m2[0], __shfl_xor_sync(0xffffffffu, b1 ? m2[0] : m2[1], 2));
+  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));   // token 4*b3 + 2*b2 + b1
+  const float s = m1 > 0.f ? e4m3_value(e4m3_encode_pos(__fdiv_rn(m1, 6.0f))) : 0.f;
+  const int base = lane & 16;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) amax[j] = fmaxf(amax[j], __shfl_xor_sync(0xffffffffu, amax[j], off));
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax[j], 6.0f)));
-    v[j] = scale > 0.f ? __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v[j], scale))), scale) : 0.f;
+  for (int p = 0; p < 4; ++p) {
+    const float s0 = __shfl_sync(0xffffffffu, s, base | (4 * p));
+    const float s1 = __shfl_sync(0xffffffffu, s, base | (4 * p + 2));
+    const float x0 = v[2 * p], x1 = v[2 * p + 1];
+    const float y0 = (x0 != 0.f && s0 > 0.f) ? __fdiv_rn(x0, s0) : 0.f;
+    const float y1 = (x1 != 0.f && s1 > 0.f) ? __fdiv_rn(x1, s1) : 0.f;
+    const uint32_t q = e2m1_round_f16x2(y0, y1);
+    const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&q), __floats2half2_rn(s0, s1));
+    h[p] = *reinterpret_cast<const uint32_t*>(&r);
   }
 }
 
-// NVFP4 round trip of v across the 16-lane block it belongs to (global scale
-// 1): s_b = E4M3(amax / 6), q = E2M1(v / value(s_b)), returns q * value(s_b).
-__device__ __forceinline__ float nvfp4_roundtrip16(float v) {
-  float amax = fabsf(v);
+// The same round trip, in place, as fp32 values.
+__device__ __forceinline__ void nvfp4_roundtrip16x8(float (&v)[8]) {
+  uint32_t h[4];
+  nvfp4_roundtrip16x8_h(v, h);
 #pragma unroll
-  for (int off = 1; off < 16; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
-  if (!(scale > 0.f)) return 0.f;
-  return __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v, scale))), scale);
+  for (int p = 0; p < 4; ++p) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[p]));
+    v[2 * p] = f.x;
+    v[2 * p + 1] = f.y;
+  }
 }
+
 
 
 }  // namespace lmoe

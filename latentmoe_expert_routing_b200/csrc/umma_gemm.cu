@@ -10,10 +10,11 @@
 // expert's weights exactly once.  Both operands are K-major, staged by TMA with
 // the 128-byte swizzle, 64 K-elements per pipeline stage.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring;
-// warp 1 allocates TMEM and one lane issues tcgen05.mma into one of two TMEM
-// accumulators; warps 2-5 drain the other accumulator (tcgen05.ld), apply the
-// epilogue and store.  Every wait is bounded: on timeout the kernel records
+// Warp roles: warp 0 issues TMA loads into a STAGES-deep ring; warp 1
+// allocates TMEM and one lane issues tcgen05.mma into one of two TMEM
+// accumulators; the epilogue warps (one group of four, two for 256-token tiles,
+// whose short-K GEMMs would otherwise wait on the drain) read the other
+// accumulator (tcgen05.ld), apply the epilogue and store.  Every wait is bounded: on timeout the kernel records
 // DEV_ERR_TIMEOUT, unwinds, waits for its own copies / MMAs and frees TMEM.
 #include <cuda.h>
 
@@ -21,8 +22,14 @@
 
 namespace lmoe {
 
+// epilogue groups (four warps each, one per TMEM lane quarter) and block size
+template <int NT> struct UmmaWarps {
+  static constexpr int kEpiGroups = NT >= 256 ? 2 : 1;
+  static constexpr int kThreads = 64 + 128 * kEpiGroups;
+};
+
 template <int NT, int STAGES, typename TO, bool RELU2, bool QA>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(UmmaWarps<NT>::kThreads, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
                  const __grid_constant__ CUtensorMap amap0,
                  const __grid_constant__ CUtensorMap wmap1,
@@ -49,7 +56,10 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128 * UmmaWarps<NT>::kEpiGroups);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -105,7 +115,6 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     // One thread; the loop is kept short (incremental slot and parity,
     // descriptors advanced by constants) because its length sets the step rate.
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, NT);
       const uint64_t desc0 = sw128_desc(smem_u32(smem));
       uint32_t st = 0, pf = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
@@ -115,6 +124,9 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(3); break; }
         tc_fence_after();
         const uint32_t d = tmem + buf * NT;
+        // a ragged tile multiplies only its valid token rows, rounded up to the
+        // MMA's N granularity (16): its cost follows the rows it has
+        const uint32_t idesc = idesc_bf16_f32(kBM, min(NT, (ti.valid + 15) & ~15));
         bool ok = true;
         for (int kt = ti.kb; kt < ti.ke; ++kt) {
           if (!mbar_wait(&full[st], pf)) { fail(4); ok = false; break; }
@@ -136,8 +148,10 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       if (!mbar_wait(mma_done, 0)) fail(5);
     }
   } else {
-    // ---------------- epilogue: warps 2..5 ----------------
+    // ---------------- epilogue: warps 2.. ----------------
+    constexpr int G = UmmaWarps<NT>::kEpiGroups;
     const int q = warp & 3;                  // TMEM lane quarter this warp may read
+    const int grp = (warp - 2) >> 2;         // takes chunks grp, grp + G, ...
     TO* out = reinterpret_cast<TO*>(a.out);
     uint32_t lt = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
@@ -149,12 +163,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       const int n = ti.n0 + 32 * q + lane;   // output column of this thread
       const bool col_ok = n < a.n_out;
       const float gs = a.gscale ? a.gscale[ti.grp] : 1.f;
-#pragma unroll
-      for (int c = 0; c < NT / 8; ++c) {
-        uint32_t r[8];
-        tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, r);
-        tmem_ld_wait();
-        if (c * 8 >= ti.valid) continue;     // uniform across the warp
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * NT;
+      auto emit = [&](const uint32_t (&r)[8], int c) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -170,6 +180,18 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
           if (row < ti.valid && col_ok)
             store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
         }
+      };
+      // two chunks in flight per wait; chunks past the valid rows are skipped
+      // (all conditions are uniform across the warp)
+      for (int c = grp; c < NT / 8 && c * 8 < ti.valid; c += 2 * G) {
+        const int c2 = c + G;
+        const bool two = c2 < NT / 8 && c2 * 8 < ti.valid;
+        uint32_t r0[8], r1[8];
+        tmem_ld8(tbase + c * 8, r0);
+        if (two) tmem_ld8(tbase + c2 * 8, r1);
+        tmem_ld_wait();
+        emit(r0, c);
+        if (two) emit(r1, c2);
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
@@ -245,7 +267,7 @@ static cudaError_t umma_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   }
   int grid = L.max_tiles < sms ? L.max_tiles : sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, 192, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
+  kern<<<grid, UmmaWarps<NT>::kThreads, S::kBytes, st>>>(L.wmap0, L.amap0, L.wmap1, L.amap1, L.args);
   return cudaGetLastError();
 }
 
@@ -299,10 +321,11 @@ __global__ void split_reduce_kernel(const float* __restrict__ ws, int S, int M, 
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const float scale = e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f)));
+    const float scale = amax > 0.f ? e4m3_value(e4m3_encode_pos(__fdiv_rn(amax, 6.0f))) : 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      v[i] = scale > 0.f ? __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v[i], scale))), scale) : 0.f;
+    for (int i = 0; i < 16; ++i)            // (zeros skip the division's slow path)
+      v[i] = (scale > 0.f && v[i] != 0.f)
+                 ? __fmul_rn(e2m1_value(e2m1_encode(__fdiv_rn(v[i], scale))), scale) : 0.f;
   }
   TO* o = out + (size_t)r * N + c0;
 #pragma unroll

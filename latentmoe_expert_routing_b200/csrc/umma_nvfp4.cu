@@ -23,6 +23,13 @@
 //   16-19  epilogue group 1 (odd chunks)
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
+//
+// W4A4 runs the same pipeline on fp16 operands (F16): the activations are
+// NVFP4 round-trip values and the dequantised weights are q * s_b, all exact
+// fp16 numbers, so the hardware E2M1 -> f16x2 conversion expands the weights
+// (about one instruction per element instead of seven) and the MMA computes
+// the same exact products as in bf16.
+#include <cuda_fp16.h>
 #include <stdlib.h>
 
 #include "umma_common.cuh"
@@ -54,7 +61,40 @@ __device__ __forceinline__ int dq_group(int warp) {
   return (warp >= 8 && warp < 16) ? (warp - 8) >> 2 : -1;
 }
 
-template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA>
+// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both
+// K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                      // D format: f32 (A, B format 0: f16)
+       | ((uint32_t)(N >> 3) << 17)     // N / 8
+       | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// NVFP4 record row r in the natural nibble order (both halves, k = 0..63) ->
+// 32 f16x2 words in k order, each exactly q * s_b.
+__device__ __forceinline__ void dequant_row_f16(const uint8_t* rec, int r, uint32_t (&o)[32]) {
+  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
+  const uint32_t s01 = e4m3x2_to_f16x2(sc), s23 = e4m3x2_to_f16x2(sc >> 16);
+  const uint32_t sb[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                          __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {           // k = 32*half + 8i .. +7, block 2*half + i/2
+      uint32_t q[4];
+      e2m1x8_to_f16x2(words[i], q);
+      const __half2 s2 = *reinterpret_cast<const __half2*>(&sb[2 * half + (i >> 1)]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&q[j]), s2);
+        o[16 * half + 4 * i + j] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+    }
+  }
+}
+
+template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA, bool F16>
 __global__ void __launch_bounds__(kWqThreads, 1)
 umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wqmap,
                const UmmaArgs a) {
@@ -163,7 +203,6 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   } else if (warp == 1) {
     // ---------------- MMA issuer (A from TMEM, B from shared memory) ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, NT);
       const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
       uint32_t sa = 0, pa = 0, sw = 0, pw = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
@@ -173,6 +212,9 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(15); break; }
         tc_fence_after();
         const uint32_t d = tmem + buf * NT;
+        // ragged tiles multiply only their valid rows, rounded up to N granularity 16
+        const int n_eff = min(NT, (ti.valid + 15) & ~15);
+        const uint32_t idesc = F16 ? idesc_f16_f32(kBM, n_eff) : idesc_bf16_f32(kBM, n_eff);
         bool ok = true;
         for (int st = 0; st < nsteps; ++st) {
           if (!mbar_wait(&a_full[sa], pa) || !mbar_wait(&w_ready[sw], pw)) { fail(16); ok = false; break; }
@@ -216,7 +258,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const uint8_t* rec = smem + S::kRawOffset + rr * S::kRawSlotBytes;
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t o[32];
-          dequant_row_regs(rec + ks * kWqRecordBytes, r, o);
+          if (F16) dequant_row_f16(rec + ks * kWqRecordBytes, r, o);
+          else dequant_row_regs(rec + ks * kWqRecordBytes, r, o);
           tmem_st32(lane_base + sw * 32 * KS + ks * 32, o);
         }
         tmem_st_wait();
@@ -240,7 +283,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
-      const float gs = a.gscale ? a.gscale[ti.grp] : 1.f;
+      // gscale holds s_g * 2^26 (the bf16 expansion carries 2^-26); exact rescale for fp16
+      const float gs = a.gscale ? (F16 ? a.gscale[ti.grp] * 0x1p-26f : a.gscale[ti.grp]) : 1.f;
       for (int c = grp; c < NT / 8; c += 2) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
         uint32_t rg[8];
@@ -253,11 +297,23 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
         }
-        if (QA) nvfp4_roundtrip16x8(v);
+        if constexpr (QA && F16) {
+          uint32_t hq[4];
+          nvfp4_roundtrip16x8_h(v, hq);
+          unsigned short* o16 = reinterpret_cast<unsigned short*>(a.out);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = c * 8 + j;
-          if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
+          for (int j = 0; j < 8; ++j) {
+            const int row = c * 8 + j;
+            if (row < ti.valid && col_ok)
+              o16[(size_t)(ti.a_row0 + row) * a.ldo + n] = (unsigned short)(hq[j >> 1] >> (16 * (j & 1)));
+          }
+        } else {
+          if (QA) nvfp4_roundtrip16x8(v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int row = c * 8 + j;
+            if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
+          }
         }
       }
       tc_fence_before();
@@ -273,7 +329,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   }
 }
 
-template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA>
+template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA, bool F16>
 static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   using S = WqSmem<NT, SA, RAW>;
   static_assert(S::kBytes <= 232448, "shared memory budget");
@@ -284,7 +340,7 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   static_assert((512 - S::kWCol0) / 32 >= kDqGroups && RAW >= kDqGroups && SA >= 2,
                 "ring too shallow for the dequant groups");
   static_assert(2 * SA + 2 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
-  auto kern = umma_wq_kernel<NT, SA, RAW, TO, RELU2, QA>;
+  auto kern = umma_wq_kernel<NT, SA, RAW, TO, RELU2, QA, F16>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -302,14 +358,19 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
 
 template <int NT, int SA, int RAW>
 static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
-  switch (L.epi) {
-    case UMMA_EPI_BF16: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, false>(L, st);
-    case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false>(L, st);
-    case UMMA_EPI_BF16_Q: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, true>(L, st);
-    case UMMA_EPI_BF16_RELU2_Q: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, true>(L, st);
+  if (L.a_f16) {                         // W4A4: fp16 operands, natural record order
+    switch (L.epi) {
+      case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, SA, RAW, __half, true, true, true>(L, st);
+      case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false, true>(L, st);
+      default: return cudaErrorInvalidValue;
+    }
   }
-  return cudaErrorInvalidValue;
+  switch (L.epi) {
+    case UMMA_EPI_BF16: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, false, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, false, false>(L, st);
+    case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false, false>(L, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st) {

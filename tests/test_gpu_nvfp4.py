@@ -38,6 +38,16 @@ def _gpu_quantize(w):
     return codes.cpu().numpy(), scales.cpu().numpy(), gs.cpu().numpy()
 
 
+def test_hardware_conversions_match_format(L):
+    """The W4A4 path rounds activations with the hardware E2M1 conversion and
+    expands codes and scales with the hardware fp16 conversions; over every
+    finite fp32 input, all 256 E2M1 bytes and all E4M3 scale pairs they must
+    agree with the encoders written from the format definition (which the
+    quantiser test pins to the oracle bit for bit)."""
+    from latentmoe_expert_routing_b200 import binding as B
+    assert B.moe_selftest_nvfp4_convert(torch.cuda.current_stream().cuda_stream) == 0
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_quantizer_bit_exact(L, dtype):
     g = torch.Generator().manual_seed(3)
