@@ -73,7 +73,10 @@ const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K part
 // Dense tensor-core GEMM with split-K when its output tiles cannot fill the
 // SMs (decode-sized T): slices write fp32 partials, a fixed-order reduce applies
 // the epilogue.  g.args.{K0,K1,n_out,ldo,M,out}, g.nt, g.epi and the maps are set.
-moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s) {
+// half0 / half1: the token maps with 128-row boxes (NULL: no pair launch).
+moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
+                             const CUtensorMap* half0 = nullptr,
+                             const CUtensorMap* half1 = nullptr) {
   const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
   const int steps = (g.args.K0 + g.args.K1) / 64;
   // Pick the K split with the least modelled time: waves of the persistent grid
@@ -90,6 +93,14 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s) {
   g.args.ksplit = S;
   g.args.dense_tiles = tiles * S;
   g.max_tiles = tiles * S;
+  if (S == 1 && half0 && umma_pair_eligible(g)) {
+    // 256 x 256 tiles on SM pairs, each CTA loading half of the token rows
+    g.amap0 = *half0;
+    if (half1) g.amap1 = *half1;
+    g.args.dense_tiles = (g.args.n_out / 256) * ceil_div(g.args.M, 256);
+    g.max_tiles = g.args.dense_tiles;
+    return launch_umma_pair(g, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   if (S == 1) return launch_umma(g, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   const UmmaEpi epi = g.epi;
   void* out = g.args.out;
@@ -109,6 +120,13 @@ int nt_index(long rows_per_group) { return rows_per_group <= 16 ? 0 : rows_per_g
 int grouped_nt_index(const moe_config& c, long P) {
   const int i = nt_index(P / c.n_experts);
   return (c.expert_fmt != MOE_EXPERT_DENSE && i == 2) ? 3 : i;
+}
+
+// Grouped bf16 GEMMs with 256-token tiles run on SM pairs (256-row weight
+// blocks); the route kernel builds the tile tables to match.
+bool grouped_pair(const moe_config& c, long P) {
+  return c.dtype == MOE_BF16 && c.expert_fmt == MOE_EXPERT_DENSE &&
+         kNT[grouped_nt_index(c, P)] == 256 && c.d_ff % 256 == 0 && c.d_latent % 256 == 0;
 }
 
 size_t dt_size(moe_dtype d) { return d == MOE_BF16 ? 2 : 4; }
@@ -198,7 +216,8 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
 // up / down, combine, G5 (fc2 + shared down) -- all tcgen05 GEMMs but the gather
 // and the combine.
 template <typename Mark>
-moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out,
+moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMap* xhalf, int T,
+                        void* out,
                         const float* wts, Mark& mark, cudaStream_t s) {
   const moe_config& c = h->cfg;
   const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
@@ -223,12 +242,12 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
   g.args.out = h->z; g.epi = w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
   g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
+  if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   g.wmap0 = h->wm_su;
   g.args.n_out = Fs; g.args.ldo = Fs;
   g.args.dense_tiles = ceil_div(Fs, 128) * ceil_div(T, ntd);
   g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
+  if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   mark(MOE_STAGE_EXPERT_UP);
 
   // step 6: routed experts on permuted latent rows (grouped by expert)
@@ -252,18 +271,20 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
     u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up;
     u.wqmap = h->rm_up[batch_idx(L / 64)];
   }
-  u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
-  if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  const bool pg = grouped_pair(c, P);     // SM pairs: 256-row weight blocks, half-token boxes
+  if (pg) u.amap0 = h->am_zp[3];
+  u.max_tiles = pg ? (int)((P / 256 + E) * (F / 256)) : (int)((P / ntg + E) * ceil_div(F, 128));
+  if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_EXPERT_DOWN);
-  u.wmap0 = h->wm_dn; u.amap0 = h->am_H[gi];
+  u.wmap0 = h->wm_dn; u.amap0 = h->am_H[pg ? 3 : gi];
   u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
   u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
   if (wq) {
     u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn;
     u.wqmap = h->rm_dn[batch_idx(F / 64)];
   }
-  u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
-  if ((e = launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
+  if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_COMBINE);
   launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
   mark(MOE_STAGE_DENSE_OUT);
@@ -275,7 +296,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, int T, void* out
   g.args.dense_tiles = ceil_div(D, 128) * ceil_div(T, ntd);
   g.args.out = out; g.epi = c.out_dtype == MOE_BF16 ? UMMA_EPI_BF16 : UMMA_EPI_F32;
   g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s)) != MOE_OK) return st;
+  if ((st = launch_dense_umma(h, g, s, &h->am_zc[3], &h->am_hsh[3])) != MOE_OK) return st;
   return MOE_OK;
 }
 
@@ -424,17 +445,19 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   mark(MOE_STAGE_ROUTER_LOGITS);
 
   // steps 1-4: logits, sigmoid, biased selection, weights; step 6 bookkeeping
-  CUtensorMap xmap;
+  CUtensorMap xmap, xhalf;
+  const bool wide = nt_index(T) == 2;    // 256-token tiles: SM-pair GEMMs load half boxes
   if (dt == MOE_BF16) {
     // tensor-core logits; the certified selection below makes them exact
     if (!make_tmap_bf16(&xmap, hidden, T, D, kNT[nt_index(T)])) return MOE_ERR_CUDA;
+    if (wide && !make_tmap_bf16(&xhalf, hidden, T, D, 128)) return MOE_ERR_CUDA;
     UmmaLaunch g{};
     g.wmap0 = h->wm_gate; g.amap0 = xmap; g.nt = kNT[nt_index(T)];
     g.args.err = h->err; g.args.E = 1; g.args.M = T;
     g.args.K0 = D; g.args.n_out = E; g.args.ldo = E;
     g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt);
     g.args.out = h->logits; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
-    moe_status ls = launch_dense_umma(h, g, s);
+    moe_status ls = launch_dense_umma(h, g, s, wide ? &xhalf : nullptr);
     if (ls != MOE_OK) return ls;
   } else {
     launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
@@ -445,10 +468,11 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.rsf = c.routed_scaling_factor; ra.topk_idx = idx; ra.topk_w = wts; ra.rank = h->rank;
   ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
   ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
-  if (dt == MOE_BF16) {           // tensor-core tiles: 128 weight rows x NT pairs
+  if (dt == MOE_BF16) {           // tensor-core tiles: 128 (SM pairs: 256) weight rows x NT pairs
     const int nt = kNT[grouped_nt_index(c, (long)T * k)];
-    ra.mt_up = nt; ra.nc_up = ceil_div(F, 128);
-    ra.mt_dn = nt; ra.nc_dn = ceil_div(L, 128);
+    const int bm = grouped_pair(c, (long)T * k) ? 256 : 128;
+    ra.mt_up = nt; ra.nc_up = ceil_div(F, bm);
+    ra.mt_dn = nt; ra.nc_dn = ceil_div(L, bm);
   } else {
     ra.mt_up = kMT; ra.nc_up = ceil_div(F, kChunk);
     ra.mt_dn = kMT; ra.nc_dn = ceil_div(L, kChunk);
@@ -466,7 +490,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   mark(MOE_STAGE_DENSE_IN);
 
   if (dt == MOE_BF16) {
-    moe_status us = forward_umma(h, xmap, T, out, wts, mark, s);
+    moe_status us = forward_umma(h, xmap, wide ? &xhalf : nullptr, T, out, wts, mark, s);
     if (us != MOE_OK) return us;
   } else {
     // step 5 and the shared expert's up projection: both read x

@@ -137,6 +137,10 @@ cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_split_reduce(const float* ws, int S, int M, int N, void* out, UmmaEpi epi,
                                 cudaStream_t st);
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
+// two-SM variant for 256-token tiles (umma_gemm2.cu); the token maps (amap0,
+// amap1) must have 128-row boxes and grouped tile tables 256-row weight blocks
+bool umma_pair_eligible(const UmmaLaunch& L);
+cudaError_t launch_umma_pair(const UmmaLaunch& L, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
                                   uint8_t* codes, uint8_t* scales, float* gscale,
                                   unsigned* amax_tmp, cudaStream_t st);

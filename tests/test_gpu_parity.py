@@ -137,3 +137,16 @@ def test_bf16_wide_tiles_and_many_experts(L):
     lay, g, r = _run_full(L, cfg)
     _assert_routing_exact(g, r)
     _assert_out(g[0], r["out"])
+
+
+@pytest.mark.parametrize("bias_kind", ["normal", "zipf"])
+def test_bf16_sm_pair_tiles(L, bias_kind):
+    """256-token tiles whose weight matrices have rows in multiples of 256 run
+    on SM pairs (two-CTA MMA): grouped up/down and the dense fc1, shared-up and
+    fc2 GEMMs here.  Zipf bias gives experts with many full tiles and experts
+    with a handful of tokens (ragged tiles down to one 16-row MMA step)."""
+    cfg = TINY.replace(dtype="bf16", E=16, k=4, D=512, L=256, F=512, Fs=512, T=1200,
+                       bias_kind=bias_kind)
+    lay, g, r = _run_full(L, cfg)
+    _assert_routing_exact(g, r)
+    _assert_out(g[0], r["out"])
