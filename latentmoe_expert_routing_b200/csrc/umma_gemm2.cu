@@ -108,6 +108,21 @@ __device__ __forceinline__ void commit_pair_local(uint64_t* bar) {
                ::"r"(smem_u32(bar)) : "memory");
 }
 
+// 32 lanes x 32 bits, 32 consecutive columns: thread i receives columns
+// col .. col+31 of TMEM lane (warp's lane base + i)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
 }  // namespace pair2
 
 constexpr int kPairNT = 256;                  // tokens per pair tile (MMA N at most)
@@ -305,7 +320,7 @@ umma_pair_kernel(const __grid_constant__ CUtensorMap wmap0,
       const bool col_ok = n < a.n_out;
       const float gs = a.gscale ? a.gscale[ti.grp] : 1.f;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kPairNT;
-      auto emit = [&](const uint32_t (&r)[8], int c) {
+      auto emit = [&](const uint32_t* r, int c) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -321,15 +336,16 @@ umma_pair_kernel(const __grid_constant__ CUtensorMap wmap0,
           if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
         }
       };
-      for (int c = grp; c < kPairNT / 8 && c * 8 < ti.valid; c += 2 * G) {
-        const int c2 = c + G;
-        const bool two = c2 < kPairNT / 8 && c2 * 8 < ti.valid;
-        uint32_t r0[8], r1[8];
-        tmem_ld8(tbase + c * 8, r0);
-        if (two) tmem_ld8(tbase + c2 * 8, r1);
+      // blocks of 32 columns (one TMEM load and one wait each), alternating
+      // between the groups; chunks past the valid rows are skipped (all
+      // conditions are uniform across the warp)
+      for (int b = grp; b < kPairNT / 32 && b * 32 < ti.valid; b += G) {
+        uint32_t r[32];
+        pair2::tmem_ld32(tbase + b * 32, r);
         tmem_ld_wait();
-        emit(r0, c);
-        if (two) emit(r1, c2);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if ((4 * b + u) * 8 < ti.valid) emit(r + 8 * u, 4 * b + u);
       }
       tc_fence_before();
       __syncwarp();
