@@ -244,4 +244,37 @@ __device__ __forceinline__ void nvfp4_roundtrip16x8(float (&v)[8]) {
 
 
 
+// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both
+// K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                      // D format: f32 (A, B format 0: f16)
+       | ((uint32_t)(N >> 3) << 17)     // N / 8
+       | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// NVFP4 record row r in the natural nibble order (both halves, k = 0..63) ->
+// 32 f16x2 words in k order, each exactly q * s_b.
+__device__ __forceinline__ void dequant_row_f16(const uint8_t* rec, int r, uint32_t (&o)[32]) {
+  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
+  const uint32_t s01 = e4m3x2_to_f16x2(sc), s23 = e4m3x2_to_f16x2(sc >> 16);
+  const uint32_t sb[4] = {__byte_perm(s01, 0, 0x1010), __byte_perm(s01, 0, 0x3232),
+                          __byte_perm(s23, 0, 0x1010), __byte_perm(s23, 0, 0x3232)};
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {           // k = 32*half + 8i .. +7, block 2*half + i/2
+      uint32_t q[4];
+      e2m1x8_to_f16x2(words[i], q);
+      const __half2 s2 = *reinterpret_cast<const __half2*>(&sb[2 * half + (i >> 1)]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&q[j]), s2);
+        o[16 * half + 4 * i + j] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+    }
+  }
+}
+
 }  // namespace lmoe

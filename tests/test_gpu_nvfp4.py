@@ -82,6 +82,22 @@ def test_tiny_nvfp4_layer(L, fmt, T):
         assert rel <= 1e-2, rel
 
 
+@pytest.mark.parametrize("fmt", ["w4a16", "w4a4"])
+@pytest.mark.parametrize("T", [3, 64, 200, 1200])
+def test_nvfp4_mid_layer(L, fmt, T):
+    """Mid-size NVFP4 layer (several 128-row weight blocks per expert, K of
+    256 and 512 = whole 4-slice pipeline steps): T spans the 16-, 64- and
+    128-token tiles and ragged tails, and every output row is checked."""
+    cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt=fmt, E=16, k=4, D=512,
+                                         L=256, F=512, Fs=512)
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    rel, nmax, raw = out_metrics(g[0], r["out"])
+    assert rel <= REL_L2_NVFP4, (rel, nmax)
+    if fmt == "w4a16":
+        assert rel <= 1e-2, rel
+
+
 @pytest.fixture(scope="module")
 def ultra_bf16_weights(L):
     W = L.weights_for(I.CONFIGS["ultra_decode_bf16"])
