@@ -124,14 +124,14 @@ def _oracle_sample(cfg, W, x, n_tok):
     xs, g, b = f(rows), f(W["w_gate"]), f(W["gate_bias"])
     dense = [f(W[n]) for n in ("w_fc1", "w_fc2", "w_shared_up", "w_shared_down")]
     l = O.router_logits(xs, g)
-    _, _, idx, _ = O.route(l, b, cfg.k, cfg.rsf)
+    _, _, idx, _ = O.route(l, b, cfg.k, cfg.rsf, cfg.n_group, cfg.topk_group)
     need = sorted(set(idx.reshape(-1).tolist()))
     up = {e: f(W["w_up"][e]) for e in need}       # fp32 copies; fp64 inside the call
     dn = {e: f(W["w_down"][e]) for e in need}
     t0 = time.perf_counter()
     O.forward(xs, g, b, *dense, lambda e: up[e].astype(np.float64),
               lambda e: dn[e].astype(np.float64), k=cfg.k, rsf=cfg.rsf,
-              expert_fmt=cfg.expert_fmt)
+              expert_fmt=cfg.expert_fmt, n_group=cfg.n_group, topk_group=cfg.topk_group)
     dt = time.perf_counter() - t0
     return n_tok / dt, dt
 

@@ -6,7 +6,12 @@
  *   logits = x . W_gate^T                 (router on the full d_model input)
  *   s      = sigmoid(logits)              (section 5.3)
  *   choice = s + e_score_correction_bias  (section 5.4; selection only)
- *   idx    = top-k(choice)                (section 5.5 with n_group = 1)
+ *   idx    = top-k(choice)                (section 5.5; with n_group > 1 only
+ *                                           experts of the topk_group best
+ *                                           groups compete, a group scored by
+ *                                           the fp32 sum of its two largest
+ *                                           choice scores, ties to the lower
+ *                                           group index)
  *   w      = s[idx] / (sum s[idx] + 1e-20) * routed_scaling_factor
  *   z      = x . W_fc1^T                  (fc1_latent_proj, d_model -> d_latent)
  *   zc[t]  = sum_j w[t,j] * down_e(relu(up_e(z[t]))^2),  e = idx[t,j]
@@ -46,7 +51,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. n_group > 1)     */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. n_group > 64)    */
   MOE_ERR_OOM = 3,           /* device allocation failed in moe_init       */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
   MOE_ERR_TIMEOUT = 5,       /* a bounded device wait gave up              */
@@ -71,8 +76,9 @@ typedef struct {
   int top_k;          /* k: num_experts_per_tok, 22                          */
   int d_ff;           /* F: moe_intermediate_size, 5120                      */
   int d_ff_shared;    /* Fs: moe_shared_expert_intermediate_size, 10240      */
-  int n_group;        /* must be 1 (all experts compete)                     */
-  int topk_group;     /* must be 1                                           */
+  int n_group;        /* 1: all experts compete; else E/n_group consecutive  */
+                      /* experts per group (>= 2), at most 64 groups          */
+  int topk_group;     /* groups kept, 1..n_group; top_k <= topk_group*E/n_group */
   int max_tokens;     /* workspace is sized for up to this many tokens       */
   float routed_scaling_factor;   /* 5.0                                      */
   moe_dtype dtype;               /* activations and dense weights            */

@@ -155,7 +155,14 @@ moe_status validate(const moe_config* c) {
     return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c->out_dtype != MOE_FP32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  if (c->n_group != 1 || c->topk_group != 1) return MOE_ERR_UNSUPPORTED;
+  // group routing: n_group equal groups of >= 2 experts, topk_group of them kept,
+  // enough experts in the kept groups for the top-k
+  if (c->n_group < 1 || c->topk_group < 1 || c->topk_group > c->n_group) return MOE_ERR_INVALID_ARG;
+  if (c->n_group > 1) {
+    if (c->n_experts % c->n_group || c->n_experts / c->n_group < 2) return MOE_ERR_INVALID_ARG;
+    if (c->top_k > c->topk_group * (c->n_experts / c->n_group)) return MOE_ERR_INVALID_ARG;
+    if (c->n_group > 64) return MOE_ERR_UNSUPPORTED;
+  }
   if (c->n_experts > 1024 || c->top_k > 64) return MOE_ERR_UNSUPPORTED;
   if (c->expert_fmt != MOE_EXPERT_DENSE && c->expert_fmt != MOE_EXPERT_NVFP4_W4A16 &&
       c->expert_fmt != MOE_EXPERT_NVFP4_W4A4)
@@ -480,6 +487,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.tiles_up = h->tiles_up; ra.tiles_dn = h->tiles_dn;
   ra.err = h->err;
   ra.cmask = dt == MOE_BF16 ? h->cmask : nullptr;
+  ra.n_group = c.n_group; ra.topk_group = c.topk_group;
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
                 h->stats, h->wstat};

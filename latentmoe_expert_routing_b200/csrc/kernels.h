@@ -30,6 +30,7 @@ struct RouteArgs {
   int32_t* tiles_dn;    // [E + 1]
   int* err;
   uint32_t* cmask;           // [T, ceil(E/32)] candidate bits (certified router) or NULL
+  int n_group, topk_group;   // group routing (section 5.5); n_group <= 1: all experts compete
 };
 
 void launch_router_logits(const void* x, const void* wg, float* logits, int T,

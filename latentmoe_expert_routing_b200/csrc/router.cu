@@ -99,6 +99,55 @@ __device__ __forceinline__ bool ranks_above(float c, int e, float c2, int e2) {
 // block's count of e is the popcount of the mask.
 // ---------------------------------------------------------------------------
 constexpr int kMaxTopK = 64;
+constexpr int kMaxGroups = 64;
+
+// Merge of two (largest, second largest) pairs.
+__device__ __forceinline__ void top2_merge(float& a0, float& a1, float b0, float b1) {
+  const float hi = fmaxf(a0, b0), lo = fminf(a0, b0);
+  a1 = fmaxf(lo, fmaxf(a1, b1));
+  a0 = hi;
+}
+
+// Group routing (section 5.5) for one token held by a warp (lane holds the
+// choice scores of experts lane + 32 i): groups of G = E / n_group consecutive
+// experts, a group's score is the fp32 sum of its two largest choice scores,
+// the topk_group best groups (ties to the lower group index) stay eligible and
+// the others' scores become -inf.  gs: this warp's n_group floats of scratch.
+template <int EPL>
+__device__ void mask_groups_warp(float (&c)[EPL], int E, int n_group, int topk_group, int lane,
+                                 float* gs) {
+  const int G = E / n_group;
+  for (int g = 0; g < n_group; ++g) {
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && e / G == g) top2_merge(m0, m1, c[i], -INFINITY);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+      top2_merge(m0, m1, __shfl_xor_sync(0xffffffffu, m0, off), __shfl_xor_sync(0xffffffffu, m1, off));
+    if (lane == 0) gs[g] = __fadd_rn(m0, m1);
+  }
+  __syncwarp();
+  uint64_t keep = 0;
+  for (int g0 = 0; g0 < n_group; g0 += 32) {
+    const int g = g0 + lane;
+    bool kg = false;
+    if (g < n_group) {
+      int r = 0;
+      for (int o = 0; o < n_group; ++o) r += (gs[o] > gs[g] || (gs[o] == gs[g] && o < g)) ? 1 : 0;
+      kg = r < topk_group;
+    }
+    keep |= (uint64_t)__ballot_sync(0xffffffffu, kg) << g0;
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && !((keep >> (e / G)) & 1ull)) c[i] = -INFINITY;
+  }
+  __syncwarp();
+}
 
 template <int EPL>
 __global__ void __launch_bounds__(1024)
@@ -106,9 +155,11 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              int n_tok, int E, int k, float rsf,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
              int32_t* __restrict__ rank, int32_t* __restrict__ blkcnt, int nblk,
-             int* __restrict__ err, const uint32_t* __restrict__ cmask) {
+             int* __restrict__ err, const uint32_t* __restrict__ cmask, int n_group,
+             int topk_group) {
   extern __shared__ uint32_t mask[];                 // [E]
   __shared__ float rsel[32][kMaxTopK];
+  __shared__ float gsc[32][kMaxGroups];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 32 + warp;
   for (int e = threadIdx.x; e < E; e += blockDim.x) mask[e] = 0u;
@@ -129,6 +180,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
         c[i] = -INFINITY;
       }
     }
+    if (n_group > 1) mask_groups_warp<EPL>(c, E, n_group, topk_group, lane, gsc[warp]);
     uint32_t taken = 0u;                             // bit i: expert lane+32i chosen
     for (int j = 0; j < k; ++j) {
       float bc = -INFINITY;
@@ -292,7 +344,7 @@ template <int EPL>
 static void route_launch_epl(const RouteArgs& a, cudaStream_t st) {
   route_kernel<EPL><<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(
       a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w, a.rank,
-      a.blkcnt, a.nblk, a.err, a.cmask);
+      a.blkcnt, a.nblk, a.err, a.cmask, a.n_group, a.topk_group);
 }
 
 void launch_route_select(const RouteArgs& a, cudaStream_t st) {
@@ -520,7 +572,6 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
   }
   if (lane == 0) { s_red[warp] = ss; s_mx[warp] = mx; s_mn[warp] = mn; }
-  if (e == 0) s_nc = 0;
   __syncthreads();
   float tot = 0.f, xmax = 0.f, xmin = INFINITY;
   for (int w = 0; w < nw; ++w) {
@@ -538,36 +589,98 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
     cu = c + d;
     lo = c - d;
   }
-  // 2. tau: the largest key K with #{lower-bound keys >= K} >= k
-  const uint32_t key = e < E ? f32_order_key(__double2float_rd(lo)) : 0u;
+  // exact logits (one warp per expert) of the experts listed in s_cand[0..n)
+  // whose values are not known yet; s_s / s_c receive sigmoid and choice
+  __shared__ unsigned char s_ex[1024];       // exact value known
+  __shared__ int s_nexact;
+  if (e < 1024) s_ex[e] = 0;
+  if (e == 0) s_nexact = 0;
+  auto compact = [&](bool flag) -> int {     // all threads; returns the list length
+    __syncthreads();
+    if (e == 0) s_nc = 0;
+    __syncthreads();
+    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&s_nc, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (flag) s_cand[base + __popc(bal & ((1u << lane) - 1u))] = e;
+    __syncthreads();
+    return s_nc;
+  };
+  auto exact_list = [&](int n) {             // all threads
+    for (int i = warp; i < n; i += nw) {
+      const int ce = s_cand[i];
+      if (s_ex[ce]) continue;                // uniform across the warp
+      const bool fast = ca.wstat &&
+          products_exact_f32(xmax, xmin, ca.wstat[2 * ce], ca.wstat[2 * ce + 1]);
+      const float l = fast ? exact_logit_warp_f32prod(xr, ca.wg + (size_t)ce * D, D, lane)
+                           : exact_logit_warp(xr, ca.wg + (size_t)ce * D, D, lane);
+      if (lane == 0) {
+        const float sv = sigmoid_fixed(l);
+        s_s[ce] = sv;
+        s_c[ce] = __fadd_rn(sv, a.bias[ce]);
+        s_ex[ce] = 1;
+        atomicAdd(&s_nexact, 1);
+      }
+    }
+    __syncthreads();
+  };
+
+  // 2. group routing (section 5.5): a group's score is the fp32 sum of its two
+  //    largest choice scores.  Every expert that could be one of its group's
+  //    two largest (upper bound >= the group's second largest lower bound) is
+  //    evaluated exactly, which makes every group score exact; the topk_group
+  //    best groups (ties to the lower index) stay eligible.
+  bool elig = e < E;
+  if (a.n_group > 1) {
+    __shared__ float s_lo[1024];
+    __shared__ float s_gv[kMaxGroups];
+    const int ng = a.n_group, G = E / ng;
+    if (e < E) s_lo[e] = __double2float_rd(lo);
+    __syncthreads();
+    for (int g = warp; g < ng; g += nw) {
+      float m0 = -INFINITY, m1 = -INFINITY;
+      for (int j = lane; j < G; j += 32) top2_merge(m0, m1, s_lo[g * G + j], -INFINITY);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+        top2_merge(m0, m1, __shfl_xor_sync(0xffffffffu, m0, off),
+                   __shfl_xor_sync(0xffffffffu, m1, off));
+      if (lane == 0) s_gv[g] = m1;
+    }
+    __syncthreads();
+    const bool gc = e < E && cu >= (double)s_gv[e / G];
+    exact_list(compact(gc));
+    for (int g = warp; g < ng; g += nw) {
+      float m0 = -INFINITY, m1 = -INFINITY;
+      for (int j = lane; j < G; j += 32)
+        if (s_ex[g * G + j]) top2_merge(m0, m1, s_c[g * G + j], -INFINITY);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+        top2_merge(m0, m1, __shfl_xor_sync(0xffffffffu, m0, off),
+                   __shfl_xor_sync(0xffffffffu, m1, off));
+      if (lane == 0) s_gv[g] = __fadd_rn(m0, m1);
+    }
+    __syncthreads();
+    if (e < E) {
+      const int g = e / G;
+      int r = 0;
+      for (int o = 0; o < ng; ++o) r += (s_gv[o] > s_gv[g] || (s_gv[o] == s_gv[g] && o < g)) ? 1 : 0;
+      elig = r < a.topk_group;
+      if (s_ex[e]) lo = cu = (double)s_c[e];   // the interval collapses to the exact value
+    }
+  }
+  // 3. tau: the largest key K with #{eligible lower-bound keys >= K} >= k;
+  //    candidates (eligible, upper bound >= tau), compacted, exact logits
+  const uint32_t key = elig ? f32_order_key(__double2float_rd(lo)) : 0u;
   uint32_t K = 0;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t trial = K | (1u << bit);
     if (__syncthreads_count(key >= trial) >= k) K = trial;
   }
   const double tau = (double)f32_from_key(K);
-  // 3. candidates, compacted, then exact logits (one warp per candidate)
-  const bool cand = e < E && cu >= tau;
-  const uint32_t bal = __ballot_sync(0xffffffffu, cand);
-  int base = 0;
-  if (lane == 0 && bal) base = atomicAdd(&s_nc, __popc(bal));
-  base = __shfl_sync(0xffffffffu, base, 0);
-  if (cand) s_cand[base + __popc(bal & ((1u << lane) - 1u))] = e;
-  __syncthreads();
-  const int nc = s_nc;
-  for (int i = warp; i < nc; i += nw) {
-    const int ce = s_cand[i];
-    const bool fast = ca.wstat &&
-        products_exact_f32(xmax, xmin, ca.wstat[2 * ce], ca.wstat[2 * ce + 1]);
-    const float l = fast ? exact_logit_warp_f32prod(xr, ca.wg + (size_t)ce * D, D, lane)
-                         : exact_logit_warp(xr, ca.wg + (size_t)ce * D, D, lane);
-    if (lane == 0) {
-      const float sv = sigmoid_fixed(l);
-      s_s[ce] = sv;
-      s_c[ce] = __fadd_rn(sv, a.bias[ce]);
-    }
-  }
-  __syncthreads();
+  const bool cand = elig && cu >= tau;
+  const int nc = compact(cand);
+  exact_list(nc);
   // 4. exact ranks among the candidates
   if (cand) {
     const float c = s_c[e];
@@ -587,7 +700,7 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
     float S = 0.f;
     for (int j = 0; j < k; ++j) S = __fadd_rn(S, s_rsel[j]);
     s_red[0] = __fadd_rn(S, 1e-20f);
-    if (ca.stats) atomicAdd(ca.stats, (unsigned long long)nc);
+    if (ca.stats) atomicAdd(ca.stats, (unsigned long long)s_nexact);
   }
   __syncthreads();
   if (e < k) a.topk_w[(size_t)t * k + e] = __fmul_rn(__fdiv_rn(s_rsel[e], s_red[0]), a.rsf);

@@ -119,4 +119,5 @@ def weights_for(cfg, device="cuda"):
 def layer_for(cfg, weights, max_tokens=None, out_dtype=None):
     return LatentMoE(cfg.D, cfg.L, cfg.E, cfg.k, cfg.F, cfg.Fs, weights,
                      max_tokens=max_tokens or cfg.T, rsf=cfg.rsf, dtype=cfg.dtype,
-                     expert_fmt=cfg.expert_fmt, out_dtype=out_dtype)
+                     expert_fmt=cfg.expert_fmt, out_dtype=out_dtype,
+                     n_group=cfg.n_group, topk_group=cfg.topk_group)

@@ -31,7 +31,8 @@ def oracle_rows(cfg, W, x_rows, rows=None):
     return O.forward(np32(x), np32(W["w_gate"]), np32(W["gate_bias"]), np32(W["w_fc1"]),
                      np32(W["w_fc2"]), np32(W["w_shared_up"]), np32(W["w_shared_down"]),
                      lambda e: get(up, e), lambda e: get(down, e), k=cfg.k, rsf=cfg.rsf,
-                     expert_fmt=cfg.expert_fmt)
+                     expert_fmt=cfg.expert_fmt, n_group=cfg.n_group,
+                     topk_group=cfg.topk_group)
 
 
 def out_metrics(gpu_out, ref):

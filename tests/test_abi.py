@@ -58,7 +58,9 @@ def _w(B, ptr=4096):
 @pytest.mark.parametrize("kw,status", [
     (dict(top_k=17), 1), (dict(d_model=0), 1), (dict(d_latent=60), 1),
     (dict(max_tokens=0), 1), (dict(dtype=7), 1),
-    (dict(n_group=2), 2), (dict(topk_group=2), 2), (dict(n_experts=2048), 2),
+    (dict(n_group=3), 1), (dict(topk_group=2), 1), (dict(n_group=16), 1),
+    (dict(n_group=0), 1), (dict(n_group=4, top_k=5), 1),
+    (dict(n_group=128, topk_group=8, n_experts=256), 2), (dict(n_experts=2048), 2),
     (dict(top_k=80, n_experts=100), 2),
 ])
 def test_init_rejects_bad_config_before_any_launch(B, kw, status):

@@ -150,3 +150,23 @@ def test_bf16_sm_pair_tiles(L, bias_kind):
     lay, g, r = _run_full(L, cfg)
     _assert_routing_exact(g, r)
     _assert_out(g[0], r["out"])
+
+
+@pytest.mark.parametrize("dtype,E,k,n_group,topk_group,T", [
+    ("fp32", 16, 4, 4, 2, 64),       # exact-logit router
+    ("bf16", 16, 4, 4, 2, 129),      # certified router, tensor-core GEMMs
+    ("bf16", 64, 8, 8, 3, 300),
+    ("bf16", 64, 6, 32, 4, 65),      # groups of two experts
+    ("bf16", 32, 4, 4, 4, 33),       # every group kept
+])
+def test_group_routing(L, dtype, E, k, n_group, topk_group, T):
+    """Group routing (section 5.5): only experts of the topk_group groups with
+    the largest top-2 sums compete; indices, weights and grouping must equal
+    the oracle's bit for bit, the output within tolerance."""
+    cfg = TINY.replace(dtype=dtype, E=E, k=k, n_group=n_group, topk_group=topk_group, T=T)
+    lay, g, r = _run_full(L, cfg)
+    _assert_routing_exact(g, r)
+    _assert_out(g[0], r["out"])
+    G = E // n_group
+    groups = np.unique(g[1].cpu().numpy() // G, axis=None)
+    assert all(len(set((row // G).tolist())) <= topk_group for row in g[1].cpu().numpy())

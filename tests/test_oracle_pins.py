@@ -334,3 +334,52 @@ def test_e4m3_vector_encoder_matches_scalar_definition():
     mids = [(O.e4m3_value(c) + O.e4m3_value(c + 1)) / 2 for c in range(0, 0x7E)]
     y = np.concatenate([y, mids, [0.0, 448.0, 500.0]])
     assert [O.e4m3_encode(v) for v in y] == O.e4m3_encode_vec(y).tolist()
+
+
+def _brute_group_mask(c, n_group, topk_group):
+    """Group selection written independently: a group's score is the largest
+    fp32 sum over pairs of its experts (= the sum of its two largest), and the
+    kept set is the one subset of topk_group groups whose every member ranks
+    above every non-member ((score, -index) order), found by enumeration."""
+    import itertools
+    T, E = c.shape
+    G = E // n_group
+    out = np.zeros((T, E), dtype=bool)
+    for t in range(T):
+        sc = []
+        for g in range(n_group):
+            vals = c[t, g * G:(g + 1) * G]
+            sc.append(max(np.float32(vals[i]) + np.float32(vals[j])
+                          for i in range(G) for j in range(i + 1, G)))
+        above = lambda a, b: sc[a] > sc[b] or (sc[a] == sc[b] and a < b)
+        kept = [S for S in itertools.combinations(range(n_group), topk_group)
+                if all(above(a, b) for a in S for b in range(n_group) if b not in S)]
+        assert len(kept) == 1
+        for g in kept[0]:
+            out[t, g * G:(g + 1) * G] = True
+    return out
+
+
+@pytest.mark.parametrize("E,n_group,topk_group", [(12, 4, 2), (16, 8, 3), (12, 6, 1), (8, 2, 2)])
+def test_group_mask_against_enumeration(E, n_group, topk_group):
+    rng = np.random.RandomState(E * 100 + n_group)
+    c = rng.standard_normal((40, E)).astype(np.float32)
+    c[:5] = np.round(c[:5])                    # exact ties between group scores
+    assert np.array_equal(O.group_mask(c, n_group, topk_group),
+                          _brute_group_mask(c, n_group, topk_group))
+
+
+def test_group_routing_selects_inside_kept_groups_and_reduces_to_plain_topk():
+    rng = np.random.RandomState(21)
+    l = rng.standard_normal((50, 32)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(32)).astype(np.float32)
+    _, choice, idx, w = O.route(l, b, 6, 5.0, n_group=8, topk_group=3)
+    m = O.group_mask(choice, 8, 3)
+    assert all(m[t, idx[t]].all() for t in range(50))
+    # within the kept groups the choice is the plain top-k
+    ref = O.select_topk(np.where(m, choice, -np.inf).astype(np.float32), 6)
+    assert np.array_equal(idx, ref)
+    # keeping every group is plain routing
+    assert np.array_equal(O.route(l, b, 6, 5.0, n_group=8, topk_group=8)[2],
+                          O.route(l, b, 6, 5.0)[2])
+    assert np.allclose(w.sum(axis=1), 5.0, rtol=1e-6)
