@@ -123,7 +123,11 @@ moe_status moe_forward(moe_handle* handle, const void* hidden, int T, void* out,
 
 /* Same as moe_forward with HOST buffers: copies hidden to the device, runs the
  * layer, copies out (and topk_idx / topk_w when non-NULL) back, and
- * synchronises `stream` before returning.  Pinned host memory is fastest. */
+ * synchronises `stream` before returning.  Pinned host memory is fastest.
+ * The second call with the same T captures the layer's launches into a CUDA
+ * graph (on a stream private to the handle) that later calls with that T
+ * replay on `stream`; results are identical to moe_forward's.  Profiling
+ * (moe_profile_enable) keeps every call eager. */
 moe_status moe_forward_host(moe_handle* handle, const void* hidden_host, int T,
                             void* out_host, int32_t* topk_idx_host,
                             float* topk_w_host, void* stream);

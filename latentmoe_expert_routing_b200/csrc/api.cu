@@ -31,6 +31,12 @@ struct moe_handle {
   int* err = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;   // moe_forward_host buffers
   int last_T = 0;
+  // moe_forward_host: the forward on the staging buffers as a CUDA graph,
+  // captured on the second call with the same T (the first configures every
+  // kernel eagerly) on a private stream and replayed on the caller's stream
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t host_graph = nullptr;
+  int host_graph_T = 0, host_eager_T = 0, host_graph_off = 0;
   // tensor-core path (bf16): permuted latent rows and cached TMA maps
   void* z_perm = nullptr;
   float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
@@ -331,6 +337,8 @@ void moe_destroy(moe_handle* h) {
   int cur = 0;
   cudaGetDevice(&cur);
   cudaSetDevice(h->device);
+  if (h->host_graph) cudaGraphExecDestroy(h->host_graph);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (void* p : h->owned) cudaFree(p);
   for (cudaEvent_t e : h->ev)
     if (e) cudaEventDestroy(e);
@@ -557,7 +565,35 @@ moe_status moe_forward_host(moe_handle* h, const void* hidden_host, int T, void*
   }
   cudaError_t e = cudaMemcpyAsync(h->x_stage, hidden_host, in_bytes, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  moe_status st = moe_forward(h, h->x_stage, T, h->out_stage, nullptr, nullptr, s);
+  moe_status st = MOE_OK;
+  if (!h->prof && !h->host_graph_off && h->host_graph && h->host_graph_T == T) {
+    if (cudaGraphLaunch(h->host_graph, s) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (!h->prof && !h->host_graph_off && h->host_eager_T == T) {
+    // same T again: capture the forward once, then replay it
+    if (h->host_graph) { cudaGraphExecDestroy(h->host_graph); h->host_graph = nullptr; }
+    if (!h->cap_stream && cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    cudaGraph_t g = nullptr;
+    bool ok = cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    if (ok) {
+      st = moe_forward(h, h->x_stage, T, h->out_stage, nullptr, nullptr, h->cap_stream);
+      ok = cudaStreamEndCapture(h->cap_stream, &g) == cudaSuccess && st == MOE_OK;
+    }
+    if (ok) ok = cudaGraphInstantiate(&h->host_graph, g, 0) == cudaSuccess;
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    if (ok) {
+      h->host_graph_T = T;
+      if (cudaGraphLaunch(h->host_graph, s) != cudaSuccess) return MOE_ERR_CUDA;
+    } else {                             // capture unavailable: stay eager
+      h->host_graph = nullptr;
+      h->host_graph_off = 1;
+      st = moe_forward(h, h->x_stage, T, h->out_stage, nullptr, nullptr, s);
+    }
+  } else {
+    st = moe_forward(h, h->x_stage, T, h->out_stage, nullptr, nullptr, s);
+    h->host_eager_T = T;
+  }
   if (st != MOE_OK) return st;
   const size_t P = (size_t)T * c.top_k;
   e = cudaMemcpyAsync(out_host, h->out_stage, out_bytes, cudaMemcpyDeviceToHost, s);

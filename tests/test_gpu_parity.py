@@ -122,6 +122,25 @@ def test_host_entry_point_matches_device_entry_point(L):
     assert torch.equal(oh, out.cpu()) and torch.equal(ih, idx.cpu())
 
 
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_host_entry_point_repeated_calls(L, dtype):
+    """Repeated host calls with one T replay a captured graph of the forward;
+    every call, with new inputs and a change of T in between, must equal the
+    device entry point on the same inputs."""
+    cfg = TINY.replace(dtype=dtype, T=129)
+    W = L.weights_for(cfg)
+    lay = L.layer_for(cfg, W, out_dtype="fp32")
+    for i, T in enumerate([129, 129, 129, 64, 64, 129, 129]):
+        x = I.hidden(cfg.replace(seed=i), "cuda", T=T)
+        out, idx, w = lay(x)
+        torch.cuda.synchronize()
+        xh = x.cpu().pin_memory()
+        oh = torch.empty(T, cfg.D, dtype=torch.float32).pin_memory()
+        ih = torch.empty(T, cfg.k, dtype=torch.int32).pin_memory()
+        lay.forward_host(xh, oh, ih)
+        assert torch.equal(oh, out.cpu()) and torch.equal(ih, idx.cpu()), (i, T)
+
+
 @pytest.mark.parametrize("T", [1, 3, 64, 129, 300])
 def test_tiny_bf16_tensor_core_path(L, T):
     """bf16 layers run on the tcgen05 GEMMs; T spans 16-, 64- and 256-row
