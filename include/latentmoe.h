@@ -225,7 +225,10 @@ moe_status moe_selftest_wait_timeout(moe_handle* handle, int microseconds, void*
  * library's encoder written from the format definition, as values (-0 == +0);
  * (2) the hardware E2M1 -> fp16 expansion of all 256 code pairs and (3) the
  * hardware E4M3 -> fp16 expansion of all 65536 scale pairs with the format's
- * values.  Writes the number of disagreements (0 expected) to
+ * values; (4) for every E4M3 scale s and every v within 64 ulps of an E2M1
+ * decision point times s, the code of the quotient taken from RN(1/s) with one
+ * FMA-refined correction (the block-scaled GEMM's activation rounding) against
+ * the code of the IEEE quotient v / s.  Writes the number of disagreements (0 expected) to
  * *mismatches_host and synchronises `stream`.  MOE_ERR_INVALID_ARG for a NULL
  * pointer; MOE_ERR_OOM when the device counter cannot be allocated;
  * MOE_ERR_CUDA on a launch or copy failure. */

@@ -50,6 +50,14 @@ struct moe_handle {
   CUtensorMap rm_up[3], rm_dn[3];                // record maps, batches of 1, 2, 4
   float *gs_up = nullptr, *gs_dn = nullptr;
   unsigned long long* stats = nullptr;           // exactly recomputed logits
+  // W4A4 on the block-scaled FP4 tensor cores (128-token tiles): weights as
+  // plain codes / scales, activations as codes / scales, and their maps
+  uint8_t *wc_up = nullptr, *ws_up = nullptr, *wc_dn = nullptr, *ws_dn = nullptr;
+  float* z32 = nullptr;                          // fc1 output before rounding
+  uint8_t *zq = nullptr, *zs = nullptr, *zq_perm = nullptr, *zs_perm = nullptr;
+  uint8_t *hq = nullptr, *hs = nullptr;
+  float* one = nullptr;                          // activations' global scale (1.0)
+  Mxf4Maps mx_up{}, mx_dn{};
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
   CUtensorMap am_zp[4], am_H[4], am_zc[4], am_hsh[4];   // token boxes of 16, 64, 256, 128 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
@@ -197,24 +205,41 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
   uint8_t *codes = nullptr, *scales = nullptr;
   unsigned* amax = nullptr;
   const size_t n = E * F * L;
-  if (cudaMalloc(&codes, n / 2) != cudaSuccess || cudaMalloc(&scales, n / 16) != cudaSuccess ||
-      cudaMalloc(&amax, E * 4) != cudaSuccess) {
+  const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
+  if (w4a4) {                // kept: the block-scaled FP4 GEMMs read the plain layout
+    if (!dev_alloc(h, &h->wc_up, n / 2) || !dev_alloc(h, &h->ws_up, n / 16) ||
+        !dev_alloc(h, &h->wc_dn, n / 2) || !dev_alloc(h, &h->ws_dn, n / 16))
+      return MOE_ERR_OOM;
+  } else if (cudaMalloc(&codes, n / 2) != cudaSuccess || cudaMalloc(&scales, n / 16) != cudaSuccess) {
     cudaGetLastError();
-    cudaFree(codes); cudaFree(scales); cudaFree(amax);
+    cudaFree(codes); cudaFree(scales);
     return MOE_ERR_OOM;
   }
+  if (cudaMalloc(&amax, E * 4) != cudaSuccess) {
+    cudaGetLastError();
+    if (!w4a4) { cudaFree(codes); cudaFree(scales); }
+    return MOE_ERR_OOM;
+  }
+  uint8_t *cu = w4a4 ? h->wc_up : codes, *su = w4a4 ? h->ws_up : scales;
+  uint8_t *cd = w4a4 ? h->wc_dn : codes, *sd = w4a4 ? h->ws_dn : scales;
   // W4A4 streams fp16 operands: its records keep the plain nibble order
   const int natural = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
-  cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, codes, scales,
+  cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, cu, su,
                                         h->gs_up, amax, s);
   if (e == cudaSuccess)
-    e = launch_repack_gemm(codes, scales, (int)E, (int)F, (int)L, h->rec_up, natural, s);
+    e = launch_repack_gemm(cu, su, (int)E, (int)F, (int)L, h->rec_up, natural, s);
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_up, h->gs_up, (int)E, s);
   if (e == cudaSuccess)
-    e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, codes, scales, h->gs_dn,
+    e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, cd, sd, h->gs_dn,
                               amax, s);
   if (e == cudaSuccess)
-    e = launch_repack_gemm(codes, scales, (int)E, (int)L, (int)F, h->rec_dn, natural, s);
+    e = launch_repack_gemm(cd, sd, (int)E, (int)L, (int)F, h->rec_dn, natural, s);
+  if (e == cudaSuccess && w4a4 && L % 256 == 0 && F % 256 == 0 &&
+      !(make_tmap_u8(&h->mx_up.wcode, h->wc_up, (long)(E * F), (int)(L / 2), 128, 128, true) &&
+        make_tmap_u8(&h->mx_up.wscale, h->ws_up, (long)(E * F), (int)(L / 16), 16, 128, false) &&
+        make_tmap_u8(&h->mx_dn.wcode, h->wc_dn, (long)(E * L), (int)(F / 2), 128, 128, true) &&
+        make_tmap_u8(&h->mx_dn.wscale, h->ws_dn, (long)(E * L), (int)(F / 16), 16, 128, false)))
+    e = cudaErrorInvalidValue;
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
   for (int i = 0; i < 3 && e == cudaSuccess; ++i)
     if (!make_tmap_records(&h->rm_up[i], h->rec_up, (long)recs_up, 1 << i) ||
@@ -223,6 +248,13 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   cudaFree(codes); cudaFree(scales); cudaFree(amax);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// W4A4 expert GEMMs run on the block-scaled FP4 tensor cores when the tiles are
+// 128 tokens wide and both K (L for up, F for down) are multiples of 256.
+bool use_mxf4(const moe_config& c, long P) {
+  return c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 && c.dtype == MOE_BF16 &&
+         kNT[grouped_nt_index(c, P)] == 128 && c.d_latent % 256 == 0 && c.d_ff % 256 == 0;
 }
 
 // Tensor-core path for bf16 layers: G1 (fc1, shared up), row gather, grouped
@@ -253,7 +285,9 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
   const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
   const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
-  g.args.out = h->z; g.epi = w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
+  const bool mx = use_mxf4(c, P) && h->z32;   // W4A4 on the block-scaled FP4 tensor cores
+  g.args.out = mx ? (void*)h->z32 : h->z;
+  g.epi = mx ? UMMA_EPI_F32 : w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
   g.max_tiles = g.args.dense_tiles;
   if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   g.wmap0 = h->wm_su;
@@ -264,6 +298,31 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   mark(MOE_STAGE_EXPERT_UP);
 
   // step 6: routed experts on permuted latent rows (grouped by expert)
+  if (mx) {
+    // z rounded to NVFP4 (global scale 1) as codes / scales, gathered per pair;
+    // up: ReLU^2 rounded to NVFP4 as codes / scales; down: fp32
+    if ((e = launch_quantize_rows_nvfp4(h->z32, T, L, h->one, h->zq, h->zs, s)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launch_gather_bytes(h->zq, h->perm, h->zq_perm, P, k, L / 2, s);
+    launch_gather_bytes(h->zs, h->perm, h->zs_perm, P, k, L / 16, s);
+    UmmaLaunch u{};
+    u.args.err = h->err;
+    u.args.E = E; u.args.offsets = h->offsets; u.nt = ntg;
+    u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
+    u.args.tiles = h->tiles_up; u.args.out = h->hq; u.args.gscale = h->gs_up;
+    u.epi = UMMA_EPI_F16_RELU2_Q;
+    u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
+    if ((e = launch_umma_mxf4(u, h->mx_up, h->hs, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    mark(MOE_STAGE_EXPERT_DOWN);
+    u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
+    u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.args.gscale = h->gs_dn;
+    u.epi = UMMA_EPI_F32;
+    u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
+    if ((e = launch_umma_mxf4(u, h->mx_dn, nullptr, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    mark(MOE_STAGE_COMBINE);
+    launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
+    mark(MOE_STAGE_DENSE_OUT);
+  } else {
   // (W4A4: z holds NVFP4 round-trip values, exact in fp16, the experts' operand type)
   if (w4a4) launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, s);
   else launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
@@ -301,6 +360,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   mark(MOE_STAGE_COMBINE);
   launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
   mark(MOE_STAGE_DENSE_OUT);
+  }
 
   // step 7: out = zc W_fc2^T + h_sh W_sd^T, one accumulator over K = L + Fs
   g.wmap0 = h->wm_fc2; g.amap0 = h->am_zc[di];
@@ -430,6 +490,26 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
     if (c.expert_fmt != MOE_EXPERT_DENSE) {
       moe_status q = quantize_experts(h, s);
       if (q != MOE_OK) { moe_destroy(h); return q; }
+    }
+    if (c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 && L % 256 == 0 && F % 256 == 0) {
+      // activations as NVFP4 codes / scales for the block-scaled FP4 GEMMs
+      const float one = 1.0f;
+      if (!dev_alloc(h, &h->z32, T * L * 4) || !dev_alloc(h, &h->zq, T * L / 2) ||
+          !dev_alloc(h, &h->zs, T * L / 16) || !dev_alloc(h, &h->zq_perm, P * L / 2) ||
+          !dev_alloc(h, &h->zs_perm, P * L / 16) || !dev_alloc(h, &h->hq, P * F / 2) ||
+          !dev_alloc(h, &h->hs, P * F / 16) || !dev_alloc(h, &h->one, 4)) {
+        moe_destroy(h);
+        return MOE_ERR_OOM;
+      }
+      if (cudaMemcpyAsync(h->one, &one, 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+          cudaStreamSynchronize(s) != cudaSuccess ||
+          !make_tmap_u8(&h->mx_up.acode, h->zq_perm, (long)P, (int)(L / 2), 128, 128, true) ||
+          !make_tmap_u8(&h->mx_up.ascale, h->zs_perm, (long)P, (int)(L / 16), 16, 128, false) ||
+          !make_tmap_u8(&h->mx_dn.acode, h->hq, (long)P, (int)(F / 2), 128, 128, true) ||
+          !make_tmap_u8(&h->mx_dn.ascale, h->hs, (long)P, (int)(F / 16), 16, 128, false)) {
+        moe_destroy(h);
+        return MOE_ERR_CUDA;
+      }
     }
   }
   if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||

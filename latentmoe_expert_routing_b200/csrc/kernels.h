@@ -142,6 +142,25 @@ cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
 // amap1) must have 128-row boxes and grouped tile tables 256-row weight blocks
 bool umma_pair_eligible(const UmmaLaunch& L);
 cudaError_t launch_umma_pair(const UmmaLaunch& L, cudaStream_t st);
+// bytes [rows, row_bytes] (uint8 tensor map); swizzle128: 128-byte swizzle
+bool make_tmap_u8(CUtensorMap* map, const void* base, long rows, int row_bytes, int box_bytes,
+                  int box_rows, bool swizzle128);
+// Block-scaled NVFP4 x NVFP4 grouped GEMM (umma_mxf4.cu): weights and tokens as
+// E2M1 codes (2 per byte, K-major) + E4M3 scales per 16 (K/16 bytes per row).
+// Maps: codes with 128-byte x 128-row boxes (128-byte swizzle), scales with
+// 16-byte x 128-row boxes.  epi UMMA_EPI_F16_RELU2_Q writes ReLU^2 rounded to
+// NVFP4 as codes to args.out [rows][n_out/2] and scales to out_scales
+// [rows][n_out/16]; UMMA_EPI_F32 writes fp32.  nt must be 128, K0 a multiple of 256.
+struct Mxf4Maps { CUtensorMap wcode, wscale, acode, ascale; };
+cudaError_t launch_umma_mxf4(const UmmaLaunch& L, const Mxf4Maps& m, uint8_t* out_scales,
+                             cudaStream_t st);
+// NVFP4 codes / scales of fp32 rows [rows, K] with global scale *gscale (1 for
+// activations): the quantiser's encoding, plain layout
+cudaError_t launch_quantize_rows_nvfp4(const float* x, int rows, int K, const float* gscale,
+                                       uint8_t* codes, uint8_t* scales, cudaStream_t st);
+// dst[p] = src[perm[p] / k], rows of row_bytes bytes (multiple of 16)
+void launch_gather_bytes(const void* src, const int32_t* perm, void* dst, long P, int k,
+                         int row_bytes, cudaStream_t st);
 cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int rows, int K,
                                   uint8_t* codes, uint8_t* scales, float* gscale,
                                   unsigned* amax_tmp, cudaStream_t st);

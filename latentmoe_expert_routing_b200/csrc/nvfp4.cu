@@ -179,12 +179,53 @@ __global__ void nvfp4_convert_check_kernel(unsigned long long* bad) {
     if ((c0 & 0x7Fu) != 0x7Fu && __low2float(p) != e4m3_value(c0)) ++n;
     if ((c1 & 0x7Fu) != 0x7Fu && __high2float(p) != e4m3_value(c1)) ++n;
   }
+  // E2M1 decision of v / s taken from r = RN(1 / s) with one FMA-refined
+  // correction (the block-scaled GEMM's activation rounding) against the IEEE
+  // division, for every E4M3 scale code
+  // and every v within 64 ulps of a decision point (or saturation) times s:
+  // elsewhere the two, within about one ulp of each other, cannot differ.
+  const float pts[8] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f, 6.0f};
+  for (uint64_t i = tid; i < 126ull * 8 * 129; i += nth) {
+    const uint32_t code = 1u + (uint32_t)(i / (8 * 129));
+    const int t = (int)((i / 129) % 8), d = (int)(i % 129) - 64;
+    const float sv = e4m3_value(code), rc = __fdiv_rn(1.0f, sv);
+    const float v = __uint_as_float(__float_as_uint(__fmul_rn(pts[t], sv)) + d);
+    const float exact = e2m1_value(e2m1_encode(__fdiv_rn(v, sv)));
+    const uint32_t h = e2m1_round_f16x2(nvfp4_div(v, sv, rc), 0.f);
+    if (__low2float(*reinterpret_cast<const __half2*>(&h)) != exact) ++n;
+  }
   if (n) atomicAdd(bad, n);
 }
 
 cudaError_t launch_nvfp4_convert_check(unsigned long long* bad, cudaStream_t st) {
   nvfp4_convert_check_kernel<<<4 * 148, 256, 0, st>>>(bad);
   return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows_nvfp4(const float* x, int rows, int K, const float* gscale,
+                                       uint8_t* codes, uint8_t* scales, cudaStream_t st) {
+  if (K % 16) return cudaErrorInvalidValue;
+  const long nb = (long)rows * (K / 16);
+  if (nb == 0) return cudaSuccess;
+  quantize_blocks_kernel<<<ceil_div(nb, 256), 256, 0, st>>>(x, 1, rows, K, gscale, codes, scales);
+  return cudaGetLastError();
+}
+
+__global__ void gather_bytes_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ perm,
+                                    uint4* __restrict__ dst, long P, int k, int row_vecs) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= P * row_vecs) return;
+  const long p = i / row_vecs;
+  const int c = (int)(i - p * row_vecs);
+  dst[i] = src[(long)(perm[p] / k) * row_vecs + c];
+}
+
+void launch_gather_bytes(const void* src, const int32_t* perm, void* dst, long P, int k,
+                         int row_bytes, cudaStream_t st) {
+  const int rv = row_bytes / 16;
+  const long n = P * rv;
+  if (n == 0) return;
+  gather_bytes_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)src, perm, (uint4*)dst, P, k, rv);
 }
 
 // one thread per 8 elements of a permuted row

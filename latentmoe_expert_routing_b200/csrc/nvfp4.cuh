@@ -78,6 +78,13 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   return d;
 }
 
+// v / s for the E2M1 decision from r = RN(1 / s): one multiply and one
+// FMA-refined correction (the residual v - y0 s is exact); 0 when r = 0.
+__device__ __forceinline__ float nvfp4_div(float v, float s, float r) {
+  const float y0 = __fmul_rn(v, r);
+  return __fmaf_rn(__fmaf_rn(-y0, s, v), r, y0);
+}
+
 // E2M1 round trip of two fp32 values (round to nearest, ties to the even
 // code, saturating at 6: the same decisions as e2m1_encode) -> f16x2 of the
 // rounded values, y0 in the low half.

@@ -240,6 +240,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
          CUDA_SUCCESS;
 }
 
+bool make_tmap_u8(CUtensorMap* map, const void* base, long rows, int row_bytes, int box_bytes,
+                  int box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base || rows <= 0 || row_bytes <= 0 || (row_bytes % 16) || (box_bytes % 16)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_tmap_records(CUtensorMap* map, const void* base, long n_records, int batch) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || !base || n_records <= 0 || batch < 1 || batch > 4) return false;
