@@ -309,16 +309,30 @@ def run_ours(a):
     b_dn = _expert_bytes(cfg, n_touched) + P * cfg.F * es + P * cfg.L * 4
     t_launch = (stage_ms["expert_up"] + stage_ms["expert_down"]) / 2
     achieved = (b_up + b_dn) / 2 / (t_launch * 1e-3) / 1e9
-    kname = ("umma_gemm_kernel (grouped expert up, expert down)" if cfg.dtype == "bf16"
-             else "grouped_rows_kernel (expert up, expert down)")
+    prefill = P / cfg.E > 64                 # 128- / 256-token tiles
+    fp4_mma = prefill and cfg.expert_fmt == "w4a4" and cfg.L % 256 == 0 and cfg.F % 256 == 0
+    if cfg.dtype != "bf16":
+        kname = "grouped_rows_kernel (expert up, expert down)"
+    elif fp4_mma:
+        kname = "umma_mxf4_kernel (block-scaled FP4, grouped expert up, expert down)"
+    elif cfg.expert_fmt != "dense":
+        kname = "umma_wq_kernel (NVFP4 records, grouped expert up, expert down)"
+    elif prefill and cfg.L % 256 == 0 and cfg.F % 256 == 0:
+        kname = "umma_pair_kernel (two-SM, grouped expert up, expert down)"
+    else:
+        kname = "umma_gemm_kernel (grouped expert up, expert down)"
     if P / cfg.E >= 64:
-        # prefill-sized: tensor-core bound; flops per launch = 2 * P * L * F
+        # prefill-sized: tensor-core bound; flops per launch = 2 * P * L * F.
+        # The block-scaled FP4 MMA's peak: measured sustained bf16 x 4 (the
+        # nominal dense FP4 / bf16 ratio, 9 / 2.25 PFLOP/s).
         fl = 2.0 * P * cfg.L * cfg.F
-        peak = tf_sus or tf
+        peak = (tf_sus or tf) * (4.0 if fp4_mma else 1.0)
         roof = {"kernel": kname, "bound": "tensor", "achieved": fl / (t_launch * 1e-3) / 1e12,
                 "peak": peak, "unit": "TFLOP/s",
                 "frac": fl / (t_launch * 1e-3) / 1e12 / peak, "traffic": None,
-                "peak_source": f"{src} (sustained bf16)", "flops_per_launch": fl}
+                "peak_source": (f"{src} sustained bf16 x 4 (nominal fp4/bf16)" if fp4_mma
+                                else f"{src} (sustained bf16)"),
+                "flops_per_launch": fl}
     else:
         roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": hbm,
                 "unit": "GB/s", "frac": achieved / hbm,
@@ -330,7 +344,9 @@ def run_ours(a):
             "metric": METRIC, "value": D.job_throughput(T, world, ms_max * 1e-3), "unit": UNIT,
             "n_gpus": world, "steps": a.steps, "warmup": max(a.warmup, 3),
             "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "vs_baseline": None,
+            "dtype": cfg.dtype if cfg.expert_fmt == "dense" else f"{cfg.dtype}+nvfp4-{cfg.expert_fmt}",
+            "data": "synthetic",
             "config": {"workload": cfg.name, "T": T, "d_model": cfg.D, "d_latent": cfg.L,
                        "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
                        "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
