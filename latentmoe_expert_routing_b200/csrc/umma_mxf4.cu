@@ -327,17 +327,26 @@ umma_mxf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
           uint32_t codes, sc[2];
           nvfp4_codes16x8(v, rcp, codes, sc);
           const uint32_t other = __shfl_xor_sync(0xffffffffu, codes, 1);
-          uint8_t* hq = reinterpret_cast<uint8_t*>(a.out);
+          // b[j] = this column's code of token j (low nibble) and the next
+          // column's (high nibble); even lanes store one byte per token row
+          uint32_t b[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int row = c * 8 + j;
-            if (row >= ti.valid || !col_ok) continue;
-            const size_t r = (size_t)(ti.a_row0 + row);
-            if ((lane & 1) == 0)
-              hq[r * (a.ldo / 2) + n / 2] =
-                  (uint8_t)(((codes >> (4 * j)) & 0xFu) | (((other >> (4 * j)) & 0xFu) << 4));
-            if ((lane & 15) == 0)
-              out_scales[r * (a.ldo / 16) + n / 16] = (uint8_t)(sc[j >> 2] >> (8 * (j & 3)));
+          for (int j = 0; j < 8; ++j)
+            b[j] = ((codes >> (4 * j)) & 0xFu) | (((other >> (4 * j)) & 0xFu) << 4);
+          const int nrow = min(8, ti.valid - c * 8);
+          const size_t r0 = (size_t)(ti.a_row0 + c * 8);
+          uint8_t* hq = reinterpret_cast<uint8_t*>(a.out) + r0 * (a.ldo / 2) + n / 2;
+          uint8_t* hs = out_scales + r0 * (a.ldo / 16) + n / 16;
+          const size_t sq = a.ldo / 2, ss = a.ldo / 16;
+          if (col_ok && (lane & 1) == 0) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (j < nrow) hq[j * sq] = (uint8_t)b[j];
+          }
+          if (col_ok && (lane & 15) == 0) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (j < nrow) hs[j * ss] = (uint8_t)(sc[j >> 2] >> (8 * (j & 3)));
           }
         } else {
           float* out = reinterpret_cast<float*>(a.out);
