@@ -141,6 +141,38 @@ __device__ __forceinline__ void nvfp4_codes16x8(const float (&v)[8], const float
   }
 }
 
+// Transpose within groups of 8 lanes: on entry x[i] of lane l is element
+// (row l, column i) of the group's 8 x 8 block; on exit x[i] of lane l is
+// element (row i, column l).  Three butterfly stages (xor 4, 2, 1).
+__device__ __forceinline__ void transpose8(float (&x)[8], int lane) {
+#pragma unroll
+  for (int s = 4; s >= 1; s >>= 1) {
+    const bool hi = lane & s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & s) continue;
+      const float send = hi ? x[i] : x[i + s];
+      const float got = __shfl_xor_sync(0xffffffffu, send, s);
+      if (hi) x[i] = got; else x[i + s] = got;
+    }
+  }
+}
+
+// Codes of 8 values (consecutive columns of one token), two per byte, the
+// even column in the low nibble: 4 bytes.
+__device__ __forceinline__ uint32_t e2m1_codes8(const float (&y)[8]) {
+  uint32_t d;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(d)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return d;
+}
+
 }  // namespace mxf4
 
 template <bool UP>
@@ -323,30 +355,26 @@ umma_mxf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
           if (!col_ok) v[j] = 0.f;
         }
         if constexpr (UP) {
-          // H as NVFP4 codes [rows][n_out / 2] and scales [rows][n_out / 16]
-          uint32_t codes, sc[2];
-          nvfp4_codes16x8(v, rcp, codes, sc);
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, codes, 1);
-          // b[j] = this column's code of token j (low nibble) and the next
-          // column's (high nibble); even lanes store one byte per token row
-          uint32_t b[8];
+          // H as NVFP4 codes [rows][n_out / 2] and scales [rows][n_out / 16].
+          // After the transpose lane l holds token c*8 + (l & 7), columns
+          // n0 + 32q + 8*(l >> 3) + i; its 16-column block is shared with lane l ^ 8.
+          transpose8(v, lane);
+          float am = 0.f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            b[j] = ((codes >> (4 * j)) & 0xFu) | (((other >> (4 * j)) & 0xFu) << 4);
-          const int nrow = min(8, ti.valid - c * 8);
-          const size_t r0 = (size_t)(ti.a_row0 + c * 8);
-          uint8_t* hq = reinterpret_cast<uint8_t*>(a.out) + r0 * (a.ldo / 2) + n / 2;
-          uint8_t* hs = out_scales + r0 * (a.ldo / 16) + n / 16;
-          const size_t sq = a.ldo / 2, ss = a.ldo / 16;
-          if (col_ok && (lane & 1) == 0) {
+          for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
+          const uint32_t sc = am > 0.f ? e4m3_encode_pos(__fdiv_rn(am, 6.0f)) : 0u;
+          const float sv = e4m3_value(sc), r = rcp[sc];
+          float y[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (j < nrow) hq[j * sq] = (uint8_t)b[j];
-          }
-          if (col_ok && (lane & 15) == 0) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              if (j < nrow) hs[j * ss] = (uint8_t)(sc[j >> 2] >> (8 * (j & 3)));
+          for (int i = 0; i < 8; ++i) y[i] = nvfp4_div(v[i], sv, r);
+          const uint32_t word = e2m1_codes8(y);
+          const int row = c * 8 + (lane & 7);
+          if (row < ti.valid) {
+            const size_t rr = (size_t)(ti.a_row0 + row);
+            const int col = ti.n0 + 32 * q + 8 * (lane >> 3);
+            *reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.out) + rr * (a.ldo / 2) + col / 2) = word;
+            if (((lane >> 3) & 1) == 0) out_scales[rr * (a.ldo / 16) + col / 16] = (uint8_t)sc;
           }
         } else {
           float* out = reinterpret_cast<float*>(a.out);
