@@ -58,6 +58,10 @@ struct moe_handle {
   uint8_t *hq = nullptr, *hs = nullptr;
   float* one = nullptr;                          // activations' global scale (1.0)
   Mxf4Maps mx_up{}, mx_dn{};
+  // SM-pair block-scaled GEMMs: scales as atoms (weights [row block][K/64],
+  // tokens [token tile][2][K/64]); codes shared with the maps above
+  uint8_t *wa_up = nullptr, *wa_dn = nullptr, *zs_t = nullptr, *hs_t = nullptr;
+  Mxf4Maps mxp_up{}, mxp_dn{};
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
   CUtensorMap am_zp[4], am_H[4], am_zc[4], am_hsh[4];   // token boxes of 16, 64, 256, 128 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
@@ -240,6 +244,22 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
         make_tmap_u8(&h->mx_dn.wcode, h->wc_dn, (long)(E * L), (int)(F / 2), 128, 128, true) &&
         make_tmap_u8(&h->mx_dn.wscale, h->ws_dn, (long)(E * L), (int)(F / 16), 16, 128, false)))
     e = cudaErrorInvalidValue;
+  if (e == cudaSuccess && w4a4 && L % 256 == 0 && F % 256 == 0) {
+    // the weights' scales again as atoms for the SM-pair GEMMs (256-byte rows,
+    // one 8-row box = one 256-K stage of a 128-row block)
+    if (!dev_alloc(h, &h->wa_up, n / 16) || !dev_alloc(h, &h->wa_dn, n / 16)) {
+      cudaFree(amax);
+      return MOE_ERR_OOM;
+    }
+    e = launch_sf_atoms(h->ws_up, (long)(E * F), (int)L, h->wa_up, s);
+    if (e == cudaSuccess) e = launch_sf_atoms(h->ws_dn, (long)(E * L), (int)F, h->wa_dn, s);
+    h->mxp_up.wcode = h->mx_up.wcode;
+    h->mxp_dn.wcode = h->mx_dn.wcode;
+    if (e == cudaSuccess &&
+        !(make_tmap_u8(&h->mxp_up.wscale, h->wa_up, (long)(n / 16 / 256), 256, 256, 8, false) &&
+          make_tmap_u8(&h->mxp_dn.wscale, h->wa_dn, (long)(n / 16 / 256), 256, 256, 8, false)))
+      e = cudaErrorInvalidValue;
+  }
   if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
   for (int i = 0; i < 3 && e == cudaSuccess; ++i)
     if (!make_tmap_records(&h->rm_up[i], h->rec_up, (long)recs_up, 1 << i) ||
@@ -255,6 +275,12 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
 bool use_mxf4(const moe_config& c, long P) {
   return c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 && c.dtype == MOE_BF16 &&
          kNT[grouped_nt_index(c, P)] == 128 && c.d_latent % 256 == 0 && c.d_ff % 256 == 0;
+}
+
+// ... and on SM pairs (256-token x 256-output tiles, tokens as the MMA's A
+// operand) once the experts average a full pair tile of pairs.
+bool use_mxf4_pair(const moe_config& c, long P) {
+  return use_mxf4(c, P) && P >= 256L * c.n_experts;
 }
 
 // Tensor-core path for bf16 layers: G1 (fc1, shared up), row gather, grouped
@@ -303,22 +329,31 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     // up: ReLU^2 rounded to NVFP4 as codes / scales; down: fp32
     if ((e = launch_quantize_rows_nvfp4(h->z32, T, L, h->one, h->zq, h->zs, s)) != cudaSuccess)
       return MOE_ERR_CUDA;
+    const bool mp = use_mxf4_pair(c, P);    // SM pairs: 256-token tiles, 256-row weight blocks
     launch_gather_bytes(h->zq, h->perm, h->zq_perm, P, k, L / 2, s);
-    launch_gather_bytes(h->zs, h->perm, h->zs_perm, P, k, L / 16, s);
+    if (mp) {
+      if ((e = launch_gather_sf_tiles(h->zs, h->perm, h->offsets, h->tiles_up, E, F / 256, P, k, L,
+                                      h->zs_t, s)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    } else {
+      launch_gather_bytes(h->zs, h->perm, h->zs_perm, P, k, L / 16, s);
+    }
     UmmaLaunch u{};
     u.args.err = h->err;
     u.args.E = E; u.args.offsets = h->offsets; u.nt = ntg;
     u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
     u.args.tiles = h->tiles_up; u.args.out = h->hq; u.args.gscale = h->gs_up;
     u.epi = UMMA_EPI_F16_RELU2_Q;
-    u.max_tiles = (int)((P / ntg + E) * ceil_div(F, 128));
-    if ((e = launch_umma_mxf4(u, h->mx_up, h->hs, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    u.max_tiles = mp ? (int)((P / 256 + E) * (F / 256)) : (int)((P / ntg + E) * ceil_div(F, 128));
+    e = mp ? launch_umma_mxf4_pair(u, h->mxp_up, h->hs_t, s) : launch_umma_mxf4(u, h->mx_up, h->hs, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     mark(MOE_STAGE_EXPERT_DOWN);
     u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
     u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.args.gscale = h->gs_dn;
     u.epi = UMMA_EPI_F32;
-    u.max_tiles = (int)((P / ntg + E) * ceil_div(L, 128));
-    if ((e = launch_umma_mxf4(u, h->mx_dn, nullptr, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    u.max_tiles = mp ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
+    e = mp ? launch_umma_mxf4_pair(u, h->mxp_dn, nullptr, s) : launch_umma_mxf4(u, h->mx_dn, nullptr, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
     mark(MOE_STAGE_COMBINE);
     launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
     mark(MOE_STAGE_DENSE_OUT);
@@ -510,6 +545,19 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
         moe_destroy(h);
         return MOE_ERR_CUDA;
       }
+      // token-tile scale atoms of the SM-pair GEMMs: at most P / 256 + E tiles
+      const size_t ntt = P / 256 + E;
+      if (!dev_alloc(h, &h->zs_t, ntt * L * 16) || !dev_alloc(h, &h->hs_t, ntt * F * 16)) {
+        moe_destroy(h);
+        return MOE_ERR_OOM;
+      }
+      h->mxp_up.acode = h->mx_up.acode;
+      h->mxp_dn.acode = h->mx_dn.acode;
+      if (!make_tmap_u8(&h->mxp_up.ascale, h->zs_t, (long)(ntt * L / 16), 256, 256, 8, false) ||
+          !make_tmap_u8(&h->mxp_dn.ascale, h->hs_t, (long)(ntt * F / 16), 256, 256, 8, false)) {
+        moe_destroy(h);
+        return MOE_ERR_CUDA;
+      }
     }
   }
   if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||
@@ -564,8 +612,9 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
   ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
   if (dt == MOE_BF16) {           // tensor-core tiles: 128 (SM pairs: 256) weight rows x NT pairs
-    const int nt = kNT[grouped_nt_index(c, (long)T * k)];
-    const int bm = grouped_pair(c, (long)T * k) ? 256 : 128;
+    const bool mp = use_mxf4_pair(c, (long)T * k) && h->z32;   // as forward_umma decides
+    const int nt = mp ? 256 : kNT[grouped_nt_index(c, (long)T * k)];
+    const int bm = (mp || grouped_pair(c, (long)T * k)) ? 256 : 128;
     ra.mt_up = nt; ra.nc_up = ceil_div(F, bm);
     ra.mt_dn = nt; ra.nc_dn = ceil_div(L, bm);
   } else {

@@ -154,6 +154,24 @@ bool make_tmap_u8(CUtensorMap* map, const void* base, long rows, int row_bytes, 
 struct Mxf4Maps { CUtensorMap wcode, wscale, acode, ascale; };
 cudaError_t launch_umma_mxf4(const UmmaLaunch& L, const Mxf4Maps& m, uint8_t* out_scales,
                              cudaStream_t st);
+// The same products on SM pairs (umma_mxf4_pair.cu): 256-token x 256-output
+// tiles, tokens as the MMA's A operand; the tile tables must use 256-token
+// tiles and 256-row weight blocks; n_out and w_group_rows multiples of 256.
+//   The pair kernel reads scales as atoms (512 B: 128 rows x one 64-K step, row
+//   32c + i at byte 16 i + 4 c, see launch_sf_atoms): Mxf4Maps::wscale over the
+//   weights' atoms [rows / 128][K / 64] and ascale over the tokens' atoms
+//   [token tile][2][K / 64], both viewed as rows of 256 B with 8-row boxes (one
+//   256-K stage of one 128-row block); the up epilogue writes H's scales as
+//   token-tile atoms to out_scales.
+cudaError_t launch_umma_mxf4_pair(const UmmaLaunch& L, const Mxf4Maps& m, uint8_t* out_scales,
+                                  cudaStream_t st);
+// plain scales [rows][K/16] -> atoms [rows / 128][K / 64] (rows % 128 == 0, K % 64 == 0)
+cudaError_t launch_sf_atoms(const uint8_t* plain, long rows, int K, uint8_t* atoms, cudaStream_t st);
+// per-token plain scales [T][K/16] -> the permuted pairs' token-tile atoms
+// [tile][2][K / 64] (tiles: the GEMM's tile table of 256-token tiles, nc blocks)
+cudaError_t launch_gather_sf_tiles(const uint8_t* plain, const int32_t* perm,
+                                   const int32_t* offsets, const int32_t* tiles, int E, int nc,
+                                   long P, int k, int K, uint8_t* atoms, cudaStream_t st);
 // NVFP4 codes / scales of fp32 rows [rows, K] with global scale *gscale (1 for
 // activations): the quantiser's encoding, plain layout
 cudaError_t launch_quantize_rows_nvfp4(const float* x, int rows, int K, const float* gscale,

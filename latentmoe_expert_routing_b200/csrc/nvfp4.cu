@@ -228,6 +228,73 @@ void launch_gather_bytes(const void* src, const int32_t* perm, void* dst, long P
   gather_bytes_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)src, perm, (uint4*)dst, P, k, rv);
 }
 
+// ---- scale-factor atoms of the SM-pair block-scaled FP4 GEMM ---------------
+// An atom holds the E4M3 scales of 128 rows for one 64-K step (512 B): row
+// 32c + i of the block at byte 16 i + 4 c, its four scales (16-element blocks
+// 4s .. 4s+3 of step s) in order -- the tensor-memory scale-factor layout of
+// tcgen05.mma kind::mxf4nvf4 row for row, which tcgen05.cp copies unchanged.
+// The kernels move 4-byte words: word (row, step) of the plain layout
+// [rows][K/16] goes to word 128 atom + 4 i + c.
+
+// weights: atoms [rows / 128][K / 64], rows a multiple of 128
+__global__ void sf_atoms_kernel(const uint32_t* __restrict__ plain, long rows, int ksteps,
+                                uint32_t* __restrict__ atoms) {
+  const long w = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (w >= rows * ksteps) return;
+  const long r = w / ksteps;
+  const int s = (int)(w - r * ksteps);
+  atoms[((r >> 7) * ksteps + s) * 128 + (r & 31) * 4 + ((r >> 5) & 3)] = plain[w];
+}
+
+cudaError_t launch_sf_atoms(const uint8_t* plain, long rows, int K, uint8_t* atoms, cudaStream_t st) {
+  if (rows % 128 || K % 64) return cudaErrorInvalidValue;
+  const int ks = K / 64;
+  const long n = rows * ks;
+  if (n == 0) return cudaSuccess;
+  sf_atoms_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint32_t*)plain, rows, ks,
+                                                     (uint32_t*)atoms);
+  return cudaGetLastError();
+}
+
+// permuted pairs: pair p of expert e, local row l = p - offsets[e], belongs to
+// token tile t = tiles[e] / nc + l / 256 (tiles: the GEMM's tile table built
+// with 256-token tiles and nc column blocks), block b = (l / 128) % 2, atom
+// row l % 128; its scales are those of token perm[p] / k.  Output atoms
+// [tile][2][K / 64]; rows of a tile past the expert's pairs stay unwritten.
+__global__ void gather_sf_tiles_kernel(const uint32_t* __restrict__ plain,
+                                       const int32_t* __restrict__ perm,
+                                       const int32_t* __restrict__ offsets,
+                                       const int32_t* __restrict__ tiles, int E, int nc, long P,
+                                       int k, int ksteps, uint32_t* __restrict__ atoms) {
+  const long w = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (w >= P * ksteps) return;
+  const long p = w / ksteps;
+  const int s = (int)(w - p * ksteps);
+  int lo = 0, hi = E;                        // the expert e with offsets[e] <= p < offsets[e + 1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offsets[mid] <= p) lo = mid; else hi = mid;
+  }
+  const long l = p - offsets[lo];
+  const long t = tiles[lo] / nc + (l >> 8);
+  const int b = (int)(l >> 7) & 1, r = (int)(l & 127);
+  atoms[((t * 2 + b) * ksteps + s) * 128 + (r & 31) * 4 + (r >> 5)] =
+      plain[(long)(perm[p] / k) * ksteps + s];
+}
+
+cudaError_t launch_gather_sf_tiles(const uint8_t* plain, const int32_t* perm,
+                                   const int32_t* offsets, const int32_t* tiles, int E, int nc,
+                                   long P, int k, int K, uint8_t* atoms, cudaStream_t st) {
+  if (K % 64 || nc < 1) return cudaErrorInvalidValue;
+  const int ks = K / 64;
+  const long n = P * ks;
+  if (n == 0) return cudaSuccess;
+  gather_sf_tiles_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint32_t*)plain, perm, offsets,
+                                                            tiles, E, nc, P, k, ks,
+                                                            (uint32_t*)atoms);
+  return cudaGetLastError();
+}
+
 // one thread per 8 elements of a permuted row
 __global__ void gather_rows_f16_kernel(const uint4* __restrict__ z, const int32_t* __restrict__ perm,
                                        uint4* __restrict__ zp, long P, int k, int row_vecs) {

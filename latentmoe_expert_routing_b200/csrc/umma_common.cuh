@@ -100,6 +100,46 @@ __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, const int32_t* s_
   return true;
 }
 
+// ---- SM-pair (cta_group::2) tiles: 256 weight rows x 256 tokens ----------
+constexpr int kPairNT = 256;                  // tokens per pair tile (MMA N at most)
+constexpr int kPairBM = 256;                  // weight rows per pair tile (MMA M)
+
+// Pair tile -> (group, 256-row weight block, token rows).  Grouped mode uses
+// the device tile table built with 256-token tiles and 256-row blocks.
+__device__ __forceinline__ bool decode_pair_tile(const UmmaArgs& a, const int32_t* s_tiles,
+                                                 const int32_t* s_off, int tile, TileInfo& ti) {
+  const int nmb = a.n_out / kPairBM;
+  int e = 0, base = 0, cnt = a.M, local = tile;
+  if (a.offsets) {
+    int lo = 0, hi = a.E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tiles[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+    base = s_off[e];
+    cnt = s_off[e + 1] - base;
+    local = tile - s_tiles[e];
+  }
+  const int nnb = (cnt + kPairNT - 1) / kPairNT;
+  if (nnb == 0) return false;
+  const int mblk = local / nnb, nb = local - mblk * nnb;
+  if (mblk >= nmb) return false;
+  ti.grp = e;
+  ti.mblk = mblk;
+  ti.n0 = mblk * kPairBM;
+  ti.w_row0 = e * a.w_group_rows + ti.n0;
+  ti.a_row0 = base + nb * kPairNT;
+  ti.valid = min(kPairNT, cnt - nb * kPairNT);
+  ti.kb = 0;
+  ti.ke = (a.K0 + a.K1) / kBK;
+  ti.slice = 0;
+  return true;
+}
+
+// MMA N of a pair tile: its valid tokens rounded up to 16 (each CTA holds N/2)
+__device__ __forceinline__ int pair_n(int valid) { return min(kPairNT, (valid + 15) & ~15); }
+
 __device__ __forceinline__ int total_tiles(const UmmaArgs& a, const int32_t* s_tiles) {
   return a.offsets ? s_tiles[a.E] : a.dense_tiles;
 }

@@ -30,6 +30,7 @@
 // fp32 rows.
 #include <cuda_fp16.h>
 
+#include "mxf4_sm100.cuh"
 #include "umma_common.cuh"
 
 namespace lmoe {
@@ -56,91 +57,6 @@ constexpr int kTmemCols = 512;
 static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
 static_assert(kBytes <= 232448, "shared memory budget");
 
-// Instruction descriptor, kind::mxf4nvf4: E2M1 A and B (format 1), UE4M3
-// scales (format 0), both K-major, K = 64, M x N; scale-factor byte ids 0.
-__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N) {
-  return (1u << 7)                       // A format: E2M1
-       | (1u << 10)                      // B format: E2M1
-       | ((uint32_t)(N >> 3) << 17)      // N / 8
-       | ((uint32_t)(M >> 4) << 24);     // M / 16 (bit 23 = 0: UE4M3 scales)
-}
-
-__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
-        "r"(sfb_tmem));
-}
-
-// 32 lanes x 32 bits, 16 consecutive columns
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};"
-      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-        "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
-        "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-
-// E2M1 codes of two fp32 values (round to nearest, ties to the even code,
-// saturating): y0's code in bits 0-3, y1's in bits 4-7.
-__device__ __forceinline__ uint32_t e2m1_codes2(float y0, float y1) {
-  uint32_t d;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(d) : "f"(y0), "f"(y1));
-  return d & 0xFFu;
-}
-
-// NVFP4 round (global scale 1) of this lane's 8 token values v >= 0 within the
-// 16-lane block of output columns it belongs to, as codes: nibble j of codes =
-// E2M1 code of token j, byte j of scodes (two words) = the E4M3 block-scale
-// code of token j.  The decisions are those of the quantiser, s_b =
-// E4M3(amax / 6) and q = E2M1(v / value(s_b)); the quotient is y0 = v * r with
-// r = RN(1 / s) refined once, y = y0 + (v - y0 s) r (two FMAs; the residual
-// is exact), which lies within an ulp of v / s and equals it at the decision
-// points themselves, so a decision can only differ for v within a few ulps of
-// (point x s); moe_selftest_nvfp4_convert checks every such v for every scale
-// code against the IEEE division.
-__device__ __forceinline__ void nvfp4_codes16x8(const float (&v)[8], const float* rcp,
-                                                uint32_t& codes, uint32_t (&scodes)[2]) {
-  const int lane = threadIdx.x & 31;
-  const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-  float m4[4], m2[2];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float lo = fabsf(v[i]), hi = fabsf(v[i + 4]);
-    m4[i] = fmaxf(b3 ? hi : lo, __shfl_xor_sync(0xffffffffu, b3 ? lo : hi, 8));
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-    m2[i] = fmaxf(b2 ? m4[i + 2] : m4[i], __shfl_xor_sync(0xffffffffu, b2 ? m4[i] : m4[i + 2], 4));
-  float m1 = fmaxf(b1 ? m2[1] : m2[0], __shfl_xor_sync(0xffffffffu, b1 ? m2[0] : m2[1], 2));
-  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));   // token 4*b3 + 2*b2 + b1
-  const uint32_t sc = m1 > 0.f ? e4m3_encode_pos(__fdiv_rn(m1, 6.0f)) : 0u;
-  const float r = rcp[sc], sv = e4m3_value(sc);           // r = 0 for the zero scale
-  const int base = lane & 16;
-  codes = 0u;
-  scodes[0] = scodes[1] = 0u;
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const uint32_t c0 = __shfl_sync(0xffffffffu, sc, base | (4 * p));
-    const uint32_t c1 = __shfl_sync(0xffffffffu, sc, base | (4 * p + 2));
-    const float r0 = __shfl_sync(0xffffffffu, r, base | (4 * p));
-    const float r1 = __shfl_sync(0xffffffffu, r, base | (4 * p + 2));
-    const float s0 = __shfl_sync(0xffffffffu, sv, base | (4 * p));
-    const float s1 = __shfl_sync(0xffffffffu, sv, base | (4 * p + 2));
-    codes |= e2m1_codes2(nvfp4_div(v[2 * p], s0, r0), nvfp4_div(v[2 * p + 1], s1, r1)) << (8 * p);
-    scodes[p >> 1] |= (c0 | (c1 << 8)) << (16 * (p & 1));
-  }
-}
-
 // Transpose within groups of 8 lanes: on entry x[i] of lane l is element
 // (row l, column i) of the group's 8 x 8 block; on exit x[i] of lane l is
 // element (row i, column l).  Three butterfly stages (xor 4, 2, 1).
@@ -156,21 +72,6 @@ __device__ __forceinline__ void transpose8(float (&x)[8], int lane) {
       if (hi) x[i] = got; else x[i + s] = got;
     }
   }
-}
-
-// Codes of 8 values (consecutive columns of one token), two per byte, the
-// even column in the low nibble: 4 bytes.
-__device__ __forceinline__ uint32_t e2m1_codes8(const float (&y)[8]) {
-  uint32_t d;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(d)
-      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
-  return d;
 }
 
 }  // namespace mxf4

@@ -83,11 +83,14 @@ def test_tiny_nvfp4_layer(L, fmt, T):
 
 
 @pytest.mark.parametrize("fmt", ["w4a16", "w4a4"])
-@pytest.mark.parametrize("T", [3, 64, 200, 1200])
+@pytest.mark.parametrize("T", [3, 64, 200, 600, 1200])
 def test_nvfp4_mid_layer(L, fmt, T):
     """Mid-size NVFP4 layer (several 128-row weight blocks per expert, K of
     256 and 512 = whole 4-slice pipeline steps): T spans the 16-, 64- and
-    128-token tiles and ragged tails, and every output row is checked."""
+    128-token tiles and ragged tails, and every output row is checked.  For
+    W4A4, T = 600 (~150 pairs per expert) runs the one-SM block-scaled FP4
+    GEMMs and T = 1200 (~300) the SM-pair ones, whose last token tile of an
+    expert leaves the second CTA without valid rows."""
     cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt=fmt, E=16, k=4, D=512,
                                          L=256, F=512, Fs=512)
     lay, g, r = _run_full(L, cfg, T)
