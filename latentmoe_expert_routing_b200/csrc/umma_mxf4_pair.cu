@@ -54,7 +54,7 @@ namespace mxf4p {
 constexpr int kStages = 5;
 constexpr int kStageK = 256;                      // K elements per stage (4 MMAs of 64)
 constexpr int kEpiGroups = 4;                     // four warps each, 64 columns per group
-constexpr int kThreads = 96 + 128 * kEpiGroups;   // producer, MMA, scale copies, epilogue
+constexpr int kThreads = 128 + 128 * kEpiGroups;  // producer, MMA, 2 scale copiers, epilogue
 constexpr int kCodeBytes = 128 * 128;             // 128 rows x 128 B of codes
 constexpr int kAtomBytes = 512;                   // scales of 128 rows x one 64-K step
 constexpr int kASfBytes = 4 * kAtomBytes;         // A: the CTA's 128 rows, 4 steps
@@ -97,7 +97,8 @@ umma_mxf4_pair_kernel(const __grid_constant__ CUtensorMap wcode_map,
   uint64_t* acc_full = empty + kStages;                              // both CTAs
   uint64_t* acc_empty = acc_full + 1;                                // leader's
   uint64_t* sf_done = acc_empty + 1;                                 // [kStages], leader's
-  uint64_t* mma_done = sf_done + kStages;
+  uint64_t* cp_drain = sf_done + kStages;                            // [2], leader's
+  uint64_t* mma_done = cp_drain + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_tiles = reinterpret_cast<int32_t*>(smem + kTableOffset);
@@ -119,6 +120,8 @@ umma_mxf4_pair_kernel(const __grid_constant__ CUtensorMap wcode_map,
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * 4 * kEpiGroups);  // every epilogue warp of the pair
     for (int s = 0; s < kStages; ++s) mbar_init(&sf_done[s], 1);
+    mbar_init(&cp_drain[0], 1);
+    mbar_init(&cp_drain[1], 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -236,19 +239,24 @@ umma_mxf4_pair_kernel(const __grid_constant__ CUtensorMap wcode_map,
       pair2::commit_pair_local(mma_done);
       if (!mbar_wait(mma_done, 0)) fail(65);
     }
-  } else if (warp == 2) {
-    // ------- scale copies (leader CTA, one lane): stage atoms -> TMEM -------
+  } else if (warp < 4) {
+    // ------- scale copies (leader CTA, one lane each of warps 2 and 3, even
+    // and odd stages): stage atoms -> TMEM -------
     // Per 64-K step A's atom -> 4 columns and B's two atoms -> 8 columns of the
     // stage's TMEM slot, in both CTAs; a commit tells the MMA thread.  A stage
     // landing means the MMAs that last read its slot completed (the producer
-    // refilled it only after their commit).
+    // refilled it only after their commit).  Each tcgen05 instruction holds
+    // its issuing thread for tens of cycles, so the copies are spread over two
+    // threads and kept off the MMA thread.
     if (leader && lane == 0) {
+      const uint32_t mine = (uint32_t)(warp - 2);
       uint32_t it = 0;
       for (int tile = pid; tile < ntiles && !*abort_flag; tile += npairs) {
         TileInfo ti;
         if (!decode_pair_tile(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
         for (int kt = 0; kt < nsteps; ++kt, ++it) {
+          if ((it & 1u) != mine) continue;
           const uint32_t st = it % kStages;
           if (!mbar_wait(&full[st], (it / kStages) & 1)) { fail(68); ok = false; break; }
           tc_fence_after();
@@ -266,17 +274,15 @@ umma_mxf4_pair_kernel(const __grid_constant__ CUtensorMap wcode_map,
         }
         if (!ok) break;
       }
-      // the copies are complete before the pair may exit (bounded)
-      const uint32_t n = it < (uint32_t)kStages ? it : (uint32_t)kStages;
-      for (uint32_t j = 0; j < n; ++j) {
-        const uint32_t i = it - 1 - j;
-        if (!mbar_wait(&sf_done[i % kStages], (i / kStages) & 1)) { fail(69); break; }
-      }
+      // this thread's copies are complete before the pair may exit (a
+      // private barrier: the stage barriers are shared with the other copier)
+      pair2::commit_pair_local(&cp_drain[mine]);
+      if (!mbar_wait(&cp_drain[mine], 0)) fail(69);
     }
   } else {
-    // ---------------- epilogue: warps 3-18 of both CTAs ----------------
+    // ---------------- epilogue: warps 4-19 of both CTAs ----------------
     const int q = warp & 3;                  // TMEM lane quarter: D rows 32q .. 32q+31
-    const int grp = (warp - 3) >> 2;         // D columns 64 grp .. 64 grp + 63
+    const int grp = (warp - 4) >> 2;         // D columns 64 grp .. 64 grp + 63
     const uint32_t empty_leader = pair2::map_to_rank(acc_empty, 0);
     uint32_t lt = 0;
     for (int tile = pid; tile < ntiles && !*abort_flag; tile += npairs) {
