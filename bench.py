@@ -313,6 +313,9 @@ def run_ours(a):
     fp4_mma = prefill and cfg.expert_fmt == "w4a4" and cfg.L % 256 == 0 and cfg.F % 256 == 0
     if cfg.dtype != "bf16":
         kname = "grouped_rows_kernel (expert up, expert down)"
+    elif fp4_mma and P >= 256 * cfg.E:
+        kname = ("umma_mxf4_pair_kernel (SM-pair block-scaled FP4, grouped expert up, "
+                 "expert down)")
     elif fp4_mma:
         kname = "umma_mxf4_kernel (block-scaled FP4, grouped expert up, expert down)"
     elif cfg.expert_fmt != "dense":
