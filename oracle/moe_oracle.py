@@ -415,6 +415,54 @@ def forward(x, w_gate, bias, w_fc1, w_fc2, w_su, w_sd, get_up, get_down, *,
 
 
 # ---------------------------------------------------------------------------
+# Block wrapper (report "Nemotron-3-Ultra architecture", the layer stack of
+# NemotronHModel.forward: every NemotronHBlock applies a pre-norm RMSNorm,
+# runs its mixer -- here the LatentMoE layer -- and adds the result to the
+# residual stream).  The pages give neither the RMSNorm formula's rounding
+# nor its epsilon: the norm is the textbook y = g * x / sqrt(mean(x^2) + eps)
+# with eps a parameter, evaluated in fp64 in a defined order, and the mixer
+# reads y rounded once to the layer's dtype.
+# ---------------------------------------------------------------------------
+
+
+def rmsnorm_spec(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """y[t] = (x[t] * r_t) * g, r_t = 1 / sqrt(dot_spec(x[t], x[t]) / D + eps),
+    one IEEE fp64 rounding per operation (squares are exact); eps is taken as
+    its fp32 value."""
+    x64 = np.asarray(x, dtype=np.float64)
+    g64 = np.asarray(g, dtype=np.float64)
+    ss = dot_spec(x64, x64)
+    r = 1.0 / np.sqrt(ss / np.float64(x64.shape[-1]) + np.float64(np.float32(eps)))
+    return (x64 * r[..., None]) * g64
+
+
+def round_fp64_to_bf16(y: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 (8 significant bits), ties to the
+    even significand, returned as float32 (exact).  With y = m * 2**e, m in
+    [0.5, 1), the result is rint(m * 256) / 256 * 2**e: rint rounds half to
+    even and every step is exact.  Values must be 0 or normal in bf16
+    (|y| >= 2**-126), which holds for normalised activations."""
+    y = np.asarray(y, dtype=np.float64)
+    m, e = np.frexp(y)
+    nz = y != 0
+    assert np.all(np.abs(y[nz]) >= 2.0 ** -126), "bf16 subnormal range"
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e).astype(np.float32)
+
+
+def block_forward(x, norm_weight, eps, *layer_args, dtype="bf16", **layer_kw):
+    """out = x + layer(RMSNorm(x)): the layer (`forward`) reads the normalised
+    rows rounded to `dtype` ("bf16" or "fp32"); returns forward's dict with
+    out replaced by the block output and y_in = the rows the layer read."""
+    y = rmsnorm_spec(x, norm_weight, eps)
+    y_in = round_fp64_to_bf16(y) if dtype == "bf16" else y.astype(np.float32)
+    r = forward(y_in, *layer_args, **layer_kw)
+    r["layer_out"] = r["out"]
+    r["out"] = np.asarray(x, dtype=np.float64) + r["out"]
+    r["y_in"] = y_in
+    return r
+
+
+# ---------------------------------------------------------------------------
 # Shapes and work (section 2.3.4 parameter list; section 3.1.3 MoE FLOPs)
 # ---------------------------------------------------------------------------
 

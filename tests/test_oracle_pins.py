@@ -383,3 +383,77 @@ def test_group_routing_selects_inside_kept_groups_and_reduces_to_plain_topk():
     assert np.array_equal(O.route(l, b, 6, 5.0, n_group=8, topk_group=8)[2],
                           O.route(l, b, 6, 5.0)[2])
     assert np.allclose(w.sum(axis=1), 5.0, rtol=1e-6)
+
+
+# ---- block wrapper: RMSNorm and the residual add ---------------------------
+
+
+def test_rmsnorm_closed_forms_and_invariants():
+    """Pins of rmsnorm_spec that do not restate its formula:
+    * eps = 0, x = c * ones with c a power of two: every step is exact, so
+      y = sign(c) * g exactly;
+    * eps = 0: scaling x by a power of two changes nothing, bit for bit;
+    * eps = 0, g = 1: the normalised rows have mean square 1 (to rounding);
+    * x = 0 gives y = 0 (eps keeps the root positive);
+    * eps shrinks the result: |y(eps)| < |y(0)| for eps > 0."""
+    D = 512
+    rng = np.random.RandomState(5)
+    g = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    for c in (1.0, -0.25, 8.0):
+        x = np.full((1, D), c)
+        assert np.array_equal(O.rmsnorm_spec(x, g, 0.0), (np.sign(c) * g.astype(np.float64))[None])
+    x = rng.standard_normal((6, D)).astype(np.float32)
+    assert np.array_equal(O.rmsnorm_spec(4.0 * x, g, 0.0), O.rmsnorm_spec(x, g, 0.0))
+    y = O.rmsnorm_spec(x, np.ones(D, np.float32), 0.0)
+    assert np.allclose((y ** 2).mean(axis=1), 1.0, rtol=1e-12)
+    assert np.array_equal(O.rmsnorm_spec(np.zeros((2, D)), g, 1e-5), np.zeros((2, D)))
+    assert np.all(np.abs(O.rmsnorm_spec(x, g, 1e-2)) < np.abs(O.rmsnorm_spec(x, g, 0.0)))
+
+
+def test_bf16_rounding_from_fp64_against_brute_force():
+    """round_fp64_to_bf16 equals the nearest point of an enumerated bf16 grid
+    (ties to the even significand), including exact midpoints."""
+    grid = np.array(sorted({float(np.float32(np.uint32(b << 16).view(np.float32)))
+                            for b in range(0x3E00, 0x4100)}))       # 2^-3 .. 8
+    rng = np.random.RandomState(9)
+    mids = (grid[:-1] + grid[1:]) / 2
+    ys = np.concatenate([grid, mids, mids + 2.0 ** -40, mids - 2.0 ** -40,
+                         rng.uniform(0.2, 7.0, 2000)])
+    ys = np.concatenate([ys, -ys])
+    got = O.round_fp64_to_bf16(ys).astype(np.float64)
+    for y, r in zip(ys, got):
+        a = np.abs(y)
+        i = np.searchsorted(grid, a)
+        lo, hi = grid[max(i - 1, 0)], grid[min(i, len(grid) - 1)]
+        if a - lo < hi - a:
+            want = lo
+        elif hi - a < a - lo:
+            want = hi
+        else:                                   # tie: the even significand
+            even = lambda v: (np.float32(v).view(np.uint32) >> 16) % 2 == 0
+            want = lo if even(lo) else hi
+        assert r == np.copysign(want, y), (y, r, want)
+
+
+def test_block_forward_residual_pins():
+    """With zero experts, zero shared expert and zero fc2 the layer adds
+    nothing and the block returns its input; with g = 0 the layer reads zero
+    rows, whose output is zero whatever the routing."""
+    rng = np.random.RandomState(3)
+    T, D, L, E, k, F, Fs = 5, 64, 16, 8, 2, 32, 32
+    x = rng.standard_normal((T, D)).astype(np.float32)
+    wg = rng.standard_normal((E, D)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(E)).astype(np.float32)
+    zero = lambda *s: np.zeros(s, np.float32)
+    r = O.block_forward(x, np.ones(D, np.float32), 1e-5, wg, b, rng.standard_normal((L, D)),
+                        zero(D, L), rng.standard_normal((Fs, D)), zero(D, Fs),
+                        lambda e: zero(F, L), lambda e: zero(L, F), k=k, rsf=5.0, dtype="fp32")
+    assert np.array_equal(r["out"], x.astype(np.float64))
+    up = rng.standard_normal((E, F, L)).astype(np.float32)
+    dn = rng.standard_normal((E, L, F)).astype(np.float32)
+    r = O.block_forward(x, np.zeros(D, np.float32), 1e-5, wg, b, rng.standard_normal((L, D)),
+                        rng.standard_normal((D, L)), rng.standard_normal((Fs, D)),
+                        rng.standard_normal((D, Fs)), lambda e: up[e], lambda e: dn[e],
+                        k=k, rsf=5.0, dtype="fp32")
+    assert np.array_equal(r["y_in"], np.zeros((T, D), np.float32))
+    assert np.array_equal(r["out"], x.astype(np.float64))
