@@ -121,6 +121,31 @@ moe_status moe_init(moe_handle** handle, const moe_config* cfg,
 moe_status moe_forward(moe_handle* handle, const void* hidden, int T, void* out,
                        int32_t* topk_idx, float* topk_w, void* stream);
 
+/* The block around the layer (report "Nemotron-3-Ultra architecture", layer
+ * stack: NemotronHBlock = pre-norm RMSNorm, mixer, residual add):
+ *   y   = RMSNorm(hidden) = (hidden * r) * norm_weight,
+ *         r = 1 / sqrt(sum_k hidden_k^2 / D + eps), per row
+ *   out = hidden + layer(y)           (layer = moe_forward on y)
+ *   norm_weight [D] dtype, device; eps > 0 and finite (the pages give no value;
+ *   1e-5 is usual) -- its fp32 value is used.
+ * The norm is evaluated in fp64 in a defined order (sum of squares in the
+ * order of the exact router logits, one IEEE rounding per operation) and y is
+ * rounded once to dtype (bf16: 8 significant bits, half to even), so the
+ * layer reads the same rows as the CPU reference; topk_idx / topk_w describe
+ * the routing of y.  The residual add is done in fp32 on the layer's output
+ * (out_dtype) and hidden.  Buffers, errors and asynchrony as moe_forward;
+ * the normalised rows live in a library-owned buffer sized for max_tokens. */
+moe_status moe_block_forward(moe_handle* handle, const void* hidden, int T,
+                             const void* norm_weight, float eps, void* out,
+                             int32_t* topk_idx, float* topk_w, void* stream);
+
+/* The block's RMSNorm on its own (the same kernel moe_block_forward runs):
+ * y[T, D] = RMSNorm(x[T, D]) with norm_weight [D], all device buffers in
+ * `dtype`, asynchronous on `stream`; MOE_ERR_INVALID_ARG for NULL buffers,
+ * T < 0, D <= 0 or eps not positive and finite. */
+moe_status moe_rmsnorm(const void* x, const void* norm_weight, int T, int D, float eps,
+                       moe_dtype dtype, void* y, void* stream);
+
 /* Same as moe_forward with HOST buffers: copies hidden to the device, runs the
  * layer, copies out (and topk_idx / topk_w when non-NULL) back, and
  * synchronises `stream` before returning.  Pinned host memory is fastest.

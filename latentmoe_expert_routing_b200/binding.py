@@ -53,6 +53,8 @@ SIGNATURES = [
     ("moe_init", _i, [_p(_vp), _p(moe_config), _p(moe_weights), _vp]),
     ("moe_forward", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     ("moe_forward_host", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
+    ("moe_block_forward", _i, [_vp, _vp, _i, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]),
+    ("moe_rmsnorm", _i, [_vp, _vp, _i, _i, ctypes.c_float, _i, _vp, _vp]),
     ("moe_get_routing", _i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     ("moe_profile_enable", _i, [_vp, _i]),
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
@@ -104,6 +106,17 @@ def moe_init(cfg: moe_config, w: moe_weights, stream: int):
 def moe_forward(h, hidden_ptr, T, out_ptr, topk_idx_ptr, topk_w_ptr, stream):
     _check(_lib.moe_forward(h, hidden_ptr, T, out_ptr, topk_idx_ptr, topk_w_ptr,
                             stream), "moe_forward")
+
+
+def moe_block_forward(h, hidden_ptr, T, norm_weight_ptr, eps, out_ptr, topk_idx_ptr, topk_w_ptr,
+                      stream):
+    _check(_lib.moe_block_forward(h, hidden_ptr, T, norm_weight_ptr, eps, out_ptr, topk_idx_ptr,
+                                  topk_w_ptr, stream), "moe_block_forward")
+
+
+def moe_rmsnorm(x_ptr, norm_weight_ptr, T, D, eps, dtype, y_ptr, stream):
+    _check(_lib.moe_rmsnorm(x_ptr, norm_weight_ptr, T, D, eps, dtype, y_ptr, stream),
+           "moe_rmsnorm")
 
 
 def moe_forward_host(h, hidden_ptr, T, out_ptr, topk_idx_ptr, topk_w_ptr, stream):

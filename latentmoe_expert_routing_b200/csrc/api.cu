@@ -27,6 +27,7 @@ struct moe_handle {
   int32_t *counts = nullptr, *offsets = nullptr, *perm = nullptr, *pos = nullptr;
   int32_t *tiles_up = nullptr, *tiles_dn = nullptr;
   void *z = nullptr, *h_sh = nullptr, *H = nullptr, *zc = nullptr;
+  void* xn = nullptr;                            // block wrapper: normalised rows [T, D]
   float* Y = nullptr;
   int* err = nullptr;
   void *x_stage = nullptr, *out_stage = nullptr;   // moe_forward_host buffers
@@ -490,7 +491,8 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
        dev_alloc(h, &h->tiles_up, (E + 1) * 4) && dev_alloc(h, &h->tiles_dn, (E + 1) * 4) &&
        dev_alloc(h, &h->z, T * L * ds) && dev_alloc(h, &h->h_sh, T * Fs * ds) &&
        dev_alloc(h, &h->H, P * F * ds) && dev_alloc(h, &h->Y, P * L * 4) &&
-       dev_alloc(h, &h->zc, T * L * ds) && dev_alloc(h, &h->err, 16);
+       dev_alloc(h, &h->zc, T * L * ds) && dev_alloc(h, &h->xn, T * c.d_model * ds) &&
+       dev_alloc(h, &h->err, 16);
   if (!ok) { moe_destroy(h); return MOE_ERR_OOM; }
   if (c.dtype == MOE_BF16) {
     if (c.d_model % 64 || c.d_latent % 64 || c.d_ff % 64 || c.d_ff_shared % 64) {
@@ -678,6 +680,25 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   return cuda_status(cudaGetLastError());
 }
 
+moe_status moe_block_forward(moe_handle* h, const void* hidden, int T, const void* norm_weight,
+                             float eps, void* out, int32_t* topk_idx, float* topk_w,
+                             void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (T == 0) { h->last_T = 0; return MOE_OK; }
+  if (!hidden || !out || !norm_weight || !aligned16(hidden) || !aligned16(out) ||
+      !(eps > 0.f) || !(eps < INFINITY))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_rmsnorm(hidden, norm_weight, T, c.d_model, eps, c.dtype, h->xn, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const moe_status st = moe_forward(h, h->xn, T, out, topk_idx, topk_w, stream);
+  if (st != MOE_OK) return st;
+  return launch_residual_add(out, c.out_dtype, hidden, c.dtype, (long)T * c.d_model, s) == cudaSuccess
+             ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_forward_host(moe_handle* h, const void* hidden_host, int T, void* out_host,
                             int32_t* topk_idx_host, float* topk_w_host, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
@@ -783,6 +804,15 @@ moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int row
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   cudaFree(amax);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_rmsnorm(const void* x, const void* norm_weight, int T, int D, float eps,
+                       moe_dtype dtype, void* y, void* stream) {
+  if (!x || !norm_weight || !y || T < 0 || D <= 0 || !(eps > 0.f) || !(eps < INFINITY))
+    return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_BF16 && dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
+  return launch_rmsnorm(x, norm_weight, T, D, eps, dtype, y, (cudaStream_t)stream) == cudaSuccess
+             ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_get_router_stats(moe_handle* h, unsigned long long* exact_logits, void* stream) {

@@ -86,6 +86,13 @@ void launch_grouped(const GroupedArgs& a, int max_tiles, cudaStream_t st);
 void launch_combine(const float* Y, const float* topk_w, const int32_t* pos,
                     void* zc, int T, int k, int L, moe_dtype out_dt, cudaStream_t st);
 
+// Block wrapper (block.cu): y = RMSNorm(x) with weight g [D] in the defined
+// fp64 order, rounded to dt; out += x (residual add, fp32 math)
+cudaError_t launch_rmsnorm(const void* x, const void* g, int T, int D, float eps, moe_dtype dt,
+                           void* y, cudaStream_t st);
+cudaError_t launch_residual_add(void* out, moe_dtype out_dt, const void* x, moe_dtype x_dt, long n,
+                                cudaStream_t st);
+
 }  // namespace lmoe
 
 namespace lmoe {

@@ -62,6 +62,27 @@ class LatentMoE:
                       topk_idx.data_ptr(), topk_w.data_ptr(), self.stream)
         return out, topk_idx, topk_w
 
+    def block(self, x, norm_weight, eps=1e-5, out=None, topk_idx=None, topk_w=None):
+        """The block around the layer: out = x + layer(RMSNorm(x)); norm_weight [D]
+        in the layer dtype (moe_block_forward)."""
+        T = x.shape[0]
+        D, k = self.dims["D"], self.dims["k"]
+        if x.dtype != _TORCH_DT[self.dtype] or not x.is_cuda or x.shape[1] != D:
+            raise ValueError("x must be a cuda [T, d_model] tensor in the layer dtype")
+        if norm_weight.dtype != x.dtype or not norm_weight.is_cuda or norm_weight.numel() != D:
+            raise ValueError("norm_weight must be a cuda [d_model] tensor in the layer dtype")
+        x = x.contiguous()
+        g = norm_weight.contiguous()
+        if out is None:
+            out = torch.empty(T, D, dtype=_TORCH_DT[self.out_dtype], device=x.device)
+        if topk_idx is None:
+            topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+        B.moe_block_forward(self.handle, x.data_ptr(), T, g.data_ptr(), float(eps),
+                            out.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), self.stream)
+        return out, topk_idx, topk_w
+
     def forward_host(self, x_host, out_host, topk_idx_host=None, topk_w_host=None):
         """Host buffers in and out (pinned is fastest); synchronises."""
         B.moe_forward_host(self.handle, x_host.data_ptr(), x_host.shape[0],
