@@ -37,6 +37,8 @@ def _args():
     ap.add_argument("--config", default="ultra_decode_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the block around the layer: out = x + layer(RMSNorm(x))")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step eagerly instead of replaying a CUDA graph")
     return ap.parse_args()
@@ -115,7 +117,7 @@ def _expert_bytes(cfg, n_touched):
     return n_touched * cfg.F * cfg.L * es
 
 
-def _oracle_sample(cfg, W, x, n_tok, min_s=0.0):
+def _oracle_sample(cfg, W, x, n_tok, min_s=0.0, norm=None):
     """Time the oracle, as it stands, on the first n_tok token rows: one forward,
     or repeated forwards until min_s seconds (at most 12)."""
     import numpy as np
@@ -124,17 +126,27 @@ def _oracle_sample(cfg, W, x, n_tok, min_s=0.0):
     f = lambda t: t.detach().float().cpu().numpy()
     xs, g, b = f(rows), f(W["w_gate"]), f(W["gate_bias"])
     dense = [f(W[n]) for n in ("w_fc1", "w_fc2", "w_shared_up", "w_shared_down")]
-    l = O.router_logits(xs, g)
+    rows = xs
+    if norm is not None:                        # the block routes its normalised rows
+        y = O.rmsnorm_spec(xs, f(norm[0]), norm[1])
+        rows = O.round_fp64_to_bf16(y) if cfg.dtype == "bf16" else y.astype(np.float32)
+    l = O.router_logits(rows, g)
     _, _, idx, _ = O.route(l, b, cfg.k, cfg.rsf, cfg.n_group, cfg.topk_group)
     need = sorted(set(idx.reshape(-1).tolist()))
     up = {e: f(W["w_up"][e]) for e in need}       # fp32 copies; fp64 inside the call
     dn = {e: f(W["w_down"][e]) for e in need}
     reps, dt = 0, 0.0
+    kw = dict(k=cfg.k, rsf=cfg.rsf, expert_fmt=cfg.expert_fmt, n_group=cfg.n_group,
+              topk_group=cfg.topk_group)
     while reps < 12 and (reps == 0 or dt < min_s):
         t0 = time.perf_counter()
-        O.forward(xs, g, b, *dense, lambda e: up[e].astype(np.float64),
-                  lambda e: dn[e].astype(np.float64), k=cfg.k, rsf=cfg.rsf,
-                  expert_fmt=cfg.expert_fmt, n_group=cfg.n_group, topk_group=cfg.topk_group)
+        if norm is None:
+            O.forward(xs, g, b, *dense, lambda e: up[e].astype(np.float64),
+                      lambda e: dn[e].astype(np.float64), **kw)
+        else:                                   # the block: (norm weight, eps)
+            O.block_forward(xs, f(norm[0]), norm[1], g, b, *dense,
+                            lambda e: up[e].astype(np.float64),
+                            lambda e: dn[e].astype(np.float64), dtype=cfg.dtype, **kw)
         dt += time.perf_counter() - t0
         reps += 1
     return reps * n_tok / dt, dt, reps
@@ -155,6 +167,28 @@ def _measured_traffic(cfg, n_touched):
     if h.hexdigest() != d["source_sha256"]:
         return None
     return d["dram_bytes_per_touched_expert"] * n_touched
+
+
+def _graph_kernel_nodes(graph):
+    """Kernel nodes of a captured CUDA graph (its cudaGraph_t kept): the
+    library's launches per step.  None when the runtime cannot be queried."""
+    import ctypes
+    try:
+        rt = ctypes.CDLL("libcudart.so.12")
+    except OSError:
+        return None
+    g = ctypes.c_void_p(graph.raw_cuda_graph())
+    n = ctypes.c_size_t(0)
+    if rt.cudaGraphGetNodes(g, None, ctypes.byref(n)) != 0:
+        return None
+    nodes = (ctypes.c_void_p * n.value)()
+    if rt.cudaGraphGetNodes(g, nodes, ctypes.byref(n)) != 0:
+        return None
+    kinds = [ctypes.c_int(-1) for _ in range(n.value)]
+    for i in range(n.value):
+        if rt.cudaGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(kinds[i])) != 0:
+            return None
+    return sum(1 for k in kinds if k.value == 0)        # cudaGraphNodeTypeKernel
 
 
 def _cores():
@@ -233,8 +267,14 @@ def run_ours(a):
     wts = torch.empty(T, cfg.k, dtype=torch.float32, device="cuda")
     st = torch.cuda.current_stream()
 
+    g = I.norm_weight(cfg, "cuda")
+    eps = 1e-5
+
     def step():
-        lay(x, out, idx, wts)
+        if a.block:
+            lay.block(x, g, eps, out, idx, wts)
+        else:
+            lay(x, out, idx, wts)
 
     barrier = D.barrier
 
@@ -246,12 +286,14 @@ def run_ours(a):
     graph = None
     if not a.no_graph:
         # the whole forward (every library launch) captured once, replayed per step
-        graph = torch.cuda.CUDAGraph()
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(graph):
             step()
+        graph.instantiate()
         graph.replay()
         torch.cuda.synchronize()
         step = graph.replay
+    launches = _graph_kernel_nodes(graph) if graph is not None else None
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -282,15 +324,26 @@ def run_ours(a):
     exact_per_token = lay.router_stats() / T
 
     # end to end through the host entry point: pinned H2D of x, D2H of out
+    # (the block has no host entry: its device call between explicit copies)
     xh = x.cpu().pin_memory()
     oh = torch.empty(T, cfg.D, dtype=tdt).pin_memory()
+
+    def host_step():
+        if a.block:
+            x.copy_(xh, non_blocking=True)
+            lay.block(x, g, eps, out, idx, wts)
+            oh.copy_(out, non_blocking=True)
+            st.synchronize()
+        else:
+            lay.forward_host(xh, oh)
+
     for _ in range(2):
-        lay.forward_host(xh, oh)
+        host_step()
     barrier()
     h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0.record(st)
     for _ in range(a.steps):
-        lay.forward_host(xh, oh)
+        host_step()
     h1.record(st)
     torch.cuda.synchronize()
     e2e_ms = D.max_over_ranks(h0.elapsed_time(h1) / a.steps, "cuda")
@@ -298,7 +351,8 @@ def run_ours(a):
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         n_tok = min(T, 2 if cfg.D >= 4096 else T)
-        v, dt, reps = _oracle_sample(cfg, W, x, n_tok, min_s=10.0)   # ~10 s of CPU work
+        v, dt, reps = _oracle_sample(cfg, W, x, n_tok, min_s=10.0,   # ~10 s of CPU work
+                                     norm=(g, eps) if a.block else None)
         cpu = {"value": v, "unit": UNIT, "cores": _cores(), "kind": "oracle",
                "sample": f"first {n_tok} of {T} tokens, {reps} fp64 numpy oracle forwards "
                          f"({dt:.1f} s)"}
@@ -359,6 +413,7 @@ def run_ours(a):
                        "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
                        "parallelism": f"replicas{world}",
                        "cuda_graph": graph is not None,
+                       "block": bool(a.block),
                        "l2": "no flush: each step streams the touched experts' weights "
                              f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
             "roofline": roof,
@@ -369,7 +424,9 @@ def run_ours(a):
                                  ((stage_ms["expert_up"] + stage_ms["expert_down"]) * 1e-3) / 1e9,
             "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,
             "clocks": clk_s,
-            "gpu_launches": 10 * a.steps,
+            # library kernels in the timed region: the captured step's kernel
+            # nodes (every one a launch of this library) times the steps
+            "gpu_launches": None if launches is None else launches * a.steps,
             "e2e": {"value": D.job_throughput(T, world, e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": T * cfg.D * es,
                     "d2h_bytes_per_step": T * cfg.D * es},

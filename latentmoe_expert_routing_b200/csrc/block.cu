@@ -10,9 +10,11 @@
 // (i, r), then a tree over lane offsets 16, 8, 4, 2, 1), each square exact and
 // each addition, the division by D, the addition of eps (its fp32 value), the
 // square root and the reciprocal one IEEE rounding; then two fp64 products.
-// Rounding to bf16 keeps 8 significant bits, half to even, computed exactly
-// as rint(m * 256) / 256 * 2^e for y = m * 2^e, m in [0.5, 1) (normal bf16
-// range; normalised activations are far from it).
+// Rounding to bf16 keeps 8 significant bits, half to even: on the fp64 bit
+// pattern, add 2^44 - 1 plus the last kept bit at bit 45 and clear the 45 low
+// bits (a carry moves into the exponent), which is rint(m * 256) / 256 * 2^e
+// for y = m * 2^e, m in [0.5, 1), in the normal bf16 range (normalised
+// activations are far from its ends).
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -25,46 +27,51 @@ __device__ __forceinline__ double load_f64(const __nv_bfloat16* p) { return (dou
 __device__ __forceinline__ double load_f64(const float* p) { return (double)*p; }
 
 __device__ __forceinline__ void store_norm(__nv_bfloat16* p, double y) {
-  int e;
-  const double m = frexp(y, &e);                       // y = m * 2^e, |m| in [0.5, 1)
-  const double v = ldexp(rint(m * 256.0) / 256.0, e);  // 8 significant bits, exact
-  *p = __float2bfloat16_rn((float)v);                  // representable: no rounding
+  const unsigned long long b = (unsigned long long)__double_as_longlong(y);
+  const unsigned long long r = (b + 0xFFFFFFFFFFFull + ((b >> 45) & 1ull)) & ~0x1FFFFFFFFFFFull;
+  *p = __float2bfloat16_rn((float)__longlong_as_double((long long)r));   // representable: exact
 }
 __device__ __forceinline__ void store_norm(float* p, double y) { *p = __double2float_rn(y); }
 
-// one warp per row
+// one CTA per row: warp 0 sums the squares in the defined order (lane p
+// takes elements 256 i + 8 p + r, increasing (i, r)), then every thread
+// scales its share of the row
 template <typename TI>
 __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const TI* __restrict__ x, const TI* __restrict__ g, int T, int D, float eps,
                TI* __restrict__ y) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  if (row >= T) return;
+  __shared__ double s_r;
+  const int row = blockIdx.x;
   const TI* xr = x + (size_t)row * D;
-  double acc = 0.0;
-  for (int i = 0; 256 * i < D; ++i)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    double acc = 0.0;
+    for (int i = 0; 256 * i < D; ++i)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int k = 256 * i + 8 * lane + r;
-      if (k < D) {
-        const double v = load_f64(xr + k);
-        acc = fma(v, v, acc);                          // the square is exact: one rounding
+      for (int r = 0; r < 8; ++r) {
+        const int k = 256 * i + 8 * lane + r;
+        if (k < D) {
+          const double v = load_f64(xr + k);
+          acc = fma(v, v, acc);                        // the square is exact: one rounding
+        }
       }
-    }
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
-  double rs = 0.0;
-  if (lane == 0)
-    rs = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(acc, (double)D), (double)eps)));
-  rs = __shfl_sync(0xffffffffu, rs, 0);
+    for (int off = 16; off >= 1; off >>= 1)
+      acc = __dadd_rn(acc, __shfl_down_sync(0xffffffffu, acc, off));
+    if (lane == 0)
+      s_r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(acc, (double)D), (double)eps)));
+  }
+  __syncthreads();
+  const double rs = s_r;
   TI* yr = y + (size_t)row * D;
-  for (int k = lane; k < D; k += 32)
+  for (int k = threadIdx.x; k < D; k += blockDim.x)
     store_norm(yr + k, __dmul_rn(__dmul_rn(load_f64(xr + k), rs), load_f64(g + k)));
 }
 
 cudaError_t launch_rmsnorm(const void* x, const void* g, int T, int D, float eps, moe_dtype dt,
                            void* y, cudaStream_t st) {
   if (T <= 0) return cudaSuccess;
-  const int blocks = (T + 7) / 8;
+  const int blocks = T;
   if (dt == MOE_BF16)
     rmsnorm_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)g, T, D,
                                            eps, (__nv_bfloat16*)y);
