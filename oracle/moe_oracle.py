@@ -13,7 +13,7 @@ may import this module.  It shares no code with the CUDA library and never
 imports it; its inputs come from latentmoe_expert_routing_b200.inputs (a seeded
 generator with none of the layer's arithmetic).
 
-Readings where the pages leave a step open (each one is listed in the design doc):
+Readings where the pages leave a step open:
   * router logits: the reference computes x.W^T in fp32 with an unspecified
     summation order.  Here the logit is DEFINED as the fp64 sum of the exact
     products in the fixed order of `dot_spec`, rounded once to fp32.
