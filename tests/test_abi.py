@@ -84,3 +84,18 @@ def test_calls_on_null_handle(B):
     assert B.lib.moe_get_routing(None, None, None, None, None, None) == 1
     assert B.lib.moe_sync(None, None) == 1
     B.lib.moe_destroy(None)
+
+
+def test_block_entry_points_validate_before_any_launch(B):
+    """moe_block_forward and moe_rmsnorm reject bad arguments with
+    MOE_ERR_INVALID_ARG before touching the device."""
+    assert B.lib.moe_block_forward(None, None, 1, None, 1e-5, None, None, None, None) == 1
+    p = ctypes.c_void_p(256)                   # never dereferenced: validation fails first
+    for eps in (0.0, -1.0, float("inf"), float("nan")):
+        assert B.lib.moe_rmsnorm(p, p, 4, 64, eps, B.MOE_BF16, p, None) == 1
+    assert B.lib.moe_rmsnorm(None, p, 4, 64, 1e-5, B.MOE_BF16, p, None) == 1
+    assert B.lib.moe_rmsnorm(p, None, 4, 64, 1e-5, B.MOE_BF16, p, None) == 1
+    assert B.lib.moe_rmsnorm(p, p, 4, 64, 1e-5, B.MOE_BF16, None, None) == 1
+    assert B.lib.moe_rmsnorm(p, p, -1, 64, 1e-5, B.MOE_BF16, p, None) == 1
+    assert B.lib.moe_rmsnorm(p, p, 4, 0, 1e-5, B.MOE_BF16, p, None) == 1
+    assert B.lib.moe_rmsnorm(p, p, 4, 64, 1e-5, 7, p, None) == 1
