@@ -16,7 +16,8 @@
 //   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
 //   2      activation producer (TMA tiles into the A ring)
-//   3      idle
+//   3      16-token tiles: second MMA issuer (16-K steps 2-3 of every slice into
+//          a second accumulator); otherwise idle
 //   4-7    epilogue group 0 (even 8-column chunks of the accumulator)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
 //          alternate steps; each thread expands its weight row's slices
@@ -47,7 +48,9 @@ struct WqSmem {
   static constexpr int kBarOffset = kRawOffset + RAW * kRawSlotBytes;
   static constexpr int kTableOffset = kBarOffset + 1024;               // 128 barrier slots
   static constexpr int kBytes = kTableOffset + kTableBytes + 1024;     // + alignment
-  static constexpr int kWCol0 = 2 * NT;                                // W slots after the accumulators
+  // 16-token tiles keep two accumulator pairs (two MMA threads, section below)
+  static constexpr int kAccCols = (NT == 16 ? 4 : 2) * NT;
+  static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
   static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
 };
 
@@ -84,6 +87,12 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // 16-token tiles: two threads issue the MMAs (16-K steps 0-1 and 2-3 of every
+  // slice) into two accumulators that the epilogue adds; each tcgen05
+  // instruction holds its issuing thread for tens of cycles, and a 128 x 16 x 16
+  // MMA is far shorter than that
+  constexpr bool SPLIT = NT == 16;
+  constexpr uint32_t NM = SPLIT ? 2 : 1;    // MMA threads
   const int kt_all = a.K0 / kBK;
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
   // tile has a multiple of KS slices
@@ -92,11 +101,11 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   const int SW = (512 - S::kWCol0) / (32 * KS);                        // W slots of 32*KS columns
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], 1); }
-    for (int s = 0; s < SW; ++s) { mbar_init(&w_ready[s], kDqGroupThreads); mbar_init(&w_empty[s], 1); }
+    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], NM); }
+    for (int s = 0; s < SW; ++s) { mbar_init(&w_ready[s], kDqGroupThreads); mbar_init(&w_empty[s], NM); }
     for (int r = 0; r < RAW; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], kDqGroupThreads); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 256); }
-    mbar_init(mma_done, 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], NM); mbar_init(&acc_empty[b], 256); }
+    mbar_init(mma_done, NM);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&amap);
@@ -167,8 +176,9 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         if (!mbar_wait(&a_full[i % SA], (i / SA) & 1)) { fail(14); break; }
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (A from TMEM, B from shared memory) ----------------
+  } else if (warp == 1 || (SPLIT && warp == 3)) {
+    // ---------------- MMA issuer(s) (A from TMEM, B from shared memory) ----------------
+    const int half = warp == 3;               // SPLIT: 16-K steps 2 half .. 2 half + 1
     if (lane == 0) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
       uint32_t sa = 0, pa = 0, sw = 0, pw = 0, lt = 0;
@@ -178,7 +188,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const uint32_t buf = lt & 1, use = lt >> 1;
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(15); break; }
         tc_fence_after();
-        const uint32_t d = tmem + buf * NT;
+        const uint32_t d = tmem + (2 * half + buf) * NT;
         // ragged tiles multiply only their valid rows, rounded up to N granularity 16
         const int n_eff = min(NT, (ti.valid + 15) & ~15);
         const uint32_t idesc = F16 ? idesc_f16_f32(kBM, n_eff) : idesc_bf16_f32(kBM, n_eff);
@@ -189,10 +199,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
           uint32_t wt = tmem + S::kWCol0 + sw * 32 * KS;
           uint64_t bd = bdesc0 + (uint64_t)(sa * (S::kASlotBytes >> 4));
           for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
-            mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
-            mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
-            mma_bf16_ts(d, wt + 16, bd + 4, idesc, 1u);
-            mma_bf16_ts(d, wt + 24, bd + 6, idesc, 1u);
+            if (SPLIT) {
+              const int j = 2 * half;
+              mma_bf16_ts(d, wt + 8 * j, bd + 2 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(d, wt + 8 * j + 8, bd + 2 * j + 2, idesc, 1u);
+            } else {
+              mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
+              mma_bf16_ts(d, wt + 16, bd + 4, idesc, 1u);
+              mma_bf16_ts(d, wt + 24, bd + 6, idesc, 1u);
+            }
           }
           mma_commit(&a_empty[sa]);          // both slots free once these MMAs finish
           mma_commit(&w_empty[sw]);
@@ -254,13 +270,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       const float gs = a.gscale ? (F16 ? a.gscale[ti.grp] * 0x1p-26f : a.gscale[ti.grp]) : 1.f;
       for (int c = grp; c < NT / 8; c += 2) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
-        uint32_t rg[8];
+        uint32_t rg[8], rh[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, rg);
+        if (SPLIT) tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (2 + buf) * NT + c * 8, rh);
         tmem_ld_wait();
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          v[j] = __fmul_rn(__uint_as_float(rg[j]), gs);
+          const float acc = SPLIT ? __fadd_rn(__uint_as_float(rg[j]), __uint_as_float(rh[j]))
+                                  : __uint_as_float(rg[j]);
+          v[j] = __fmul_rn(acc, gs);
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
         }
