@@ -62,7 +62,12 @@ typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
 
 /* Routed-expert weight format (report section 8.1; NVFP4 = E2M1 elements in
  * 16-element blocks along K, one E4M3 scale per block, one FP32 global scale
- * per expert matrix). */
+ * per expert matrix).  W4A4 also rounds the experts' inputs to NVFP4: the
+ * latent rows z along L and the ReLU^2 activations along F, in 16-element
+ * blocks with global scale 1 (round to nearest even, saturating).  Numerics
+ * within the documented tolerance of the emulated NVFP4 layer; the kernels
+ * chosen depend only on the batch shape (block-scaled FP4 tensor cores from
+ * 64 token-expert pairs per expert when L and F are multiples of 256). */
 typedef enum {
   MOE_EXPERT_DENSE = 0,        /* experts in `dtype`                          */
   MOE_EXPERT_NVFP4_W4A16 = 1,  /* NVFP4 weights, bf16 activations             */
