@@ -1,16 +1,47 @@
-"""The seeded generator: deterministic, chunk-independent, right moments."""
+"""The seeded generator: deterministic, chunk-independent, N(0, 1)."""
 import math
 
+import numpy as np
+import pytest
 import torch
+from scipy import stats
 
 from latentmoe_expert_routing_b200 import inputs as I
 
 
-def test_unit_normal_moments_and_range():
-    v = I.unit_normal(0, 1, 0, 1 << 20)
-    assert abs(v.mean().item()) < 5e-3
-    assert abs(v.var().item() - 1.0) < 5e-3
-    assert v.abs().max().item() <= 2 * math.sqrt(3.0)
+def test_log_unit_against_libm():
+    rng = np.random.RandomState(0)
+    u = np.concatenate([rng.uniform(0, 1, 200000), np.arange(1, 4097) * 2.0 ** -32,
+                        1 - np.arange(0, 4096) * 2.0 ** -53, [2.0 ** -32, 0.5, 1.0],
+                        [math.sqrt(0.5), np.nextafter(math.sqrt(0.5), 1)]])
+    got = I.log_unit(torch.from_numpy(u)).numpy()
+    ref = np.log(u)
+    assert got[-3] == 0.0 and got[-4] == -math.log(2.0)
+    ulp = np.abs(got - ref) / np.spacing(np.abs(ref) + (ref == 0))
+    assert ulp.max() <= 4
+
+
+def test_cos_2pi_against_libm_and_quadrants():
+    rng = np.random.RandomState(1)
+    u = np.concatenate([rng.uniform(0, 1, 200000), np.arange(0, 4096) * 2.0 ** -32,
+                        [0.0, 0.125, 0.25, 0.375, 0.5, 0.625, 0.75, 0.875]])
+    got = I.cos_2pi(torch.from_numpy(u)).numpy()
+    assert np.abs(got - np.cos(2 * np.pi * u)).max() <= 2e-15
+    # the quadrant points: exact values where the reduced angle is 0
+    assert got[-8:].tolist()[::2] == [1.0, 0.0, -1.0, 0.0]
+    assert np.abs(got[-7] - math.sqrt(0.5)) <= 2e-16
+
+
+def test_unit_normal_is_standard_normal():
+    v = I.unit_normal(0, 1, 0, 1 << 22).numpy()
+    assert abs(v.mean()) < 2e-3 and abs(v.var() - 1.0) < 3e-3
+    assert stats.kstest(v[:1 << 20], "norm").pvalue > 1e-3
+    n = len(v)
+    for c in (2.0, 3.0, 4.0):                       # two-sided tail masses
+        p = 2 * stats.norm.sf(c)
+        got = np.count_nonzero(np.abs(v) > c)
+        assert abs(got - n * p) < 6 * math.sqrt(n * p), (c, got, n * p)
+    assert np.abs(v).max() <= math.sqrt(-2 * math.log(2.0 ** -32)) + 1e-12
 
 
 def test_chunking_and_offsets_do_not_change_values():
@@ -52,3 +83,19 @@ def test_zipf_bias_profile():
     p = torch.exp(2 * b)
     assert abs(p.sum().item() - 1) < 1e-5
     assert abs(p[0].item() / p[1].item() - 2 ** 1.1) < 1e-4
+
+
+@pytest.mark.gpu
+def test_generator_bit_identical_on_gpu():
+    """The CPU oracle and the GPU path read the same tensors when each
+    generates them on its own device."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    a = I.unit_normal(0, 9, (1 << 33) - 5000, 1 << 20)
+    b = I.unit_normal(0, 9, (1 << 33) - 5000, 1 << 20, device="cuda").cpu()
+    assert torch.equal(a.view(torch.int64), b.view(torch.int64))
+    cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", D=512, L=256, F=512, Fs=512)
+    for f in (I.w_gate, I.w_fc1, I.w_shared_down, I.hidden):
+        assert torch.equal(f(cfg).view(torch.int16), f(cfg, "cuda").cpu().view(torch.int16))
+    assert torch.equal(I.w_up(cfg, [3]).view(torch.int16),
+                       I.w_up(cfg, [3], device="cuda").cpu().view(torch.int16))
