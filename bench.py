@@ -5,7 +5,11 @@
 
 A step is one moe_forward over one batch of T synthetic tokens (router, routing
 bookkeeping, latent projection, routed experts, combine, fc2 and the shared
-expert).  Default workload: the Ultra-shape decode layer, bf16, T=64.  With N>1
+expert).  Default workload: the Ultra-shape decode layer, bf16, T=64 (the line's
+value); on one GPU the other workloads of the metric -- Ultra prefill bf16
+T=8192, Ultra decode W4A16 T=256, skewed prefill W4A4 T=16384 -- follow on the
+same weights and are reported under "workloads", each with its own roofline,
+stage times, clocks and end-to-end figure.  With N>1
 (torchrun) every rank runs its own replica on its own tokens (weak scaling, no
 collective on the data path); value = all ranks' tokens / max-over-ranks time.
 `--impl reference` times the CPU oracle on the host cores instead.
@@ -41,6 +45,10 @@ def _args():
                     help="time the block around the layer: out = x + layer(RMSNorm(x))")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--workloads", default="auto",
+                    help="extra workloads timed after --config and reported under "
+                         "'workloads': all, none, a comma list, or auto (all for the "
+                         "default Ultra decode on one GPU, none otherwise)")
     return ap.parse_args()
 
 
@@ -246,17 +254,38 @@ def _weights(cfg, dev):
                 w_shared_down=I.w_shared_down(cfg, dev), w_up=up, w_down=down)
 
 
-def run_ours(a):
+def _layer_roofline(cfg, T, ms, hbm, tf, tf_sus, src, n_touched):
+    """The whole layer against its own bound: HBM bytes of the touched experts
+    and the dense weights at decode sizes; at prefill sizes the layer's FLOPs
+    against the tensor peak (W4A4: expert FLOPs at the FP4 rate, the rest at
+    bf16, ideal time = their sum)."""
+    fl = {"gate": 2 * cfg.D * cfg.E, "fc1": 2 * cfg.D * cfg.L, "fc2": 2 * cfg.L * cfg.D,
+          "shared": 4 * cfg.D * cfg.Fs}
+    dense_fl = T * sum(fl.values())
+    expert_fl = T * cfg.k * 4 * cfg.L * cfg.F
+    if T * cfg.k / cfg.E < 64:
+        es = 4 if cfg.dtype == "fp32" else 2
+        dense_b = (cfg.E * cfg.D + 2 * cfg.D * cfg.L + 2 * cfg.D * cfg.Fs) * es
+        b = 2 * _expert_bytes(cfg, n_touched) + dense_b
+        return {"bound": "hbm", "bytes": b, "achieved": b / (ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s", "frac": b / (ms * 1e-3) / 1e9 / hbm, "peak_source": src}
+    peak = tf_sus or tf
+    w4a4 = cfg.expert_fmt == "w4a4"
+    ideal = dense_fl / (peak * 1e12) + expert_fl / (peak * (4.0 if w4a4 else 1.0) * 1e12)
+    tot = dense_fl + expert_fl
+    return {"bound": "tensor", "flops": tot, "achieved": tot / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "ideal_ms": ideal * 1e3, "frac": ideal / (ms * 1e-3),
+            "peak_source": (f"{src} sustained bf16" +
+                            (" (experts at x4, the nominal fp4/bf16 ratio)" if w4a4 else ""))}
+
+
+def _measure(a, cfg, W, rank, world, local, cpu_leg):
+    """Time one workload on this rank's replica; returns its line fields."""
     import torch
-    from latentmoe_expert_routing_b200 import dist as D
-    rank, world, local = _dist()
-    torch.cuda.set_device(local)
-    D.init("nccl", 300, torch.device("cuda", local))
     from latentmoe_expert_routing_b200 import binding as B
+    from latentmoe_expert_routing_b200 import dist as D
     from latentmoe_expert_routing_b200 import inputs as I
     from latentmoe_expert_routing_b200 import layer as LY
-    cfg = I.CONFIGS[a.config]
-    W = _weights(cfg, "cuda")
     lay = LY.layer_for(cfg, W, out_dtype=cfg.dtype)
     x = I.hidden(cfg, "cuda", T=cfg.T, start_row=0) if rank == 0 else \
         I.hidden(cfg.replace(seed=rank), "cuda")
@@ -297,12 +326,11 @@ def run_ours(a):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if True:
-        e0.record(st)
-        for _ in range(a.steps):
-            step()
-        e1.record(st)
-        torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(a.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
     clk.__exit__()
     barrier()
     lay.sync()
@@ -319,6 +347,7 @@ def run_ours(a):
     stage_ms = {k: statistics.median(s[k] for s in stages) for k in stages[0]}
     counts, _, _, _ = lay.routing(T)
     n_touched = int((counts > 0).sum().item())
+    max_vio = float(counts.max().item()) / (T * cfg.k / cfg.E)
     lay.router_stats()
     step()
     exact_per_token = lay.router_stats() / T
@@ -349,7 +378,7 @@ def run_ours(a):
     e2e_ms = D.max_over_ranks(h0.elapsed_time(h1) / a.steps, "cuda")
 
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if cpu_leg:
         n_tok = min(T, 2 if cfg.D >= 4096 else T)
         v, dt, reps = _oracle_sample(cfg, W, x, n_tok, min_s=10.0,   # ~10 s of CPU work
                                      norm=(g, eps) if a.block else None)
@@ -399,42 +428,81 @@ def run_ours(a):
                 "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": _measured_traffic(cfg, n_touched),
                 "peak_source": src, "bytes_per_launch": (b_up + b_dn) / 2}
-    if rank == 0:
-        clk_s = clk.summary()
-        line = {
-            "metric": METRIC, "value": D.job_throughput(T, world, ms_max * 1e-3), "unit": UNIT,
-            "n_gpus": world, "steps": a.steps, "warmup": max(a.warmup, 3),
-            "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": cfg.dtype if cfg.expert_fmt == "dense" else f"{cfg.dtype}+nvfp4-{cfg.expert_fmt}",
-            "data": "synthetic",
-            "config": {"workload": cfg.name, "T": T, "d_model": cfg.D, "d_latent": cfg.L,
-                       "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
-                       "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
-                       "parallelism": f"replicas{world}",
-                       "cuda_graph": graph is not None,
-                       "block": bool(a.block),
-                       "l2": "no flush: each step streams the touched experts' weights "
-                             f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
-            "roofline": roof,
-            "stages_ms": stage_ms,
-            "experts_touched": n_touched,
-            "router_exact_logits_per_token": exact_per_token,
-            "expert_weight_gbs": 2 * _expert_bytes(cfg, n_touched) /
-                                 ((stage_ms["expert_up"] + stage_ms["expert_down"]) * 1e-3) / 1e9,
-            "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,
-            "clocks": clk_s,
-            # library kernels in the timed region: the captured step's kernel
-            # nodes (every one a launch of this library) times the steps
-            "gpu_launches": None if launches is None else launches * a.steps,
-            "e2e": {"value": D.job_throughput(T, world, e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": T * cfg.D * es,
-                    "d2h_bytes_per_step": T * cfg.D * es},
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line))
+    res = {
+        "value": D.job_throughput(T, world, ms_max * 1e-3), "ms_per_step": ms_max,
+        "dtype": cfg.dtype if cfg.expert_fmt == "dense" else f"{cfg.dtype}+nvfp4-{cfg.expert_fmt}",
+        "config": {"workload": cfg.name, "T": T, "d_model": cfg.D, "d_latent": cfg.L,
+                   "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
+                   "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
+                   "bias": cfg.bias_kind, "outlier_rows": len(I.outlier_rows(cfg)),
+                   "parallelism": f"replicas{world}",
+                   "cuda_graph": graph is not None,
+                   "block": bool(a.block),
+                   "l2": "no flush: each step streams the touched experts' weights "
+                         f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
+        "roofline": roof,
+        "layer_roofline": _layer_roofline(cfg, T, ms_max, hbm, tf, tf_sus, src, n_touched),
+        "stages_ms": stage_ms,
+        "experts_touched": n_touched,
+        "max_load_over_mean": max_vio,
+        "router_exact_logits_per_token": exact_per_token,
+        "expert_weight_gbs": 2 * _expert_bytes(cfg, n_touched) /
+                             ((stage_ms["expert_up"] + stage_ms["expert_down"]) * 1e-3) / 1e9,
+        "layer_hbm_frac": (2 * _expert_bytes(cfg, n_touched) / (ms_max * 1e-3) / 1e9) / hbm,
+        "clocks": clk.summary(),
+        # library kernels in the timed region: the captured step's kernel
+        # nodes (every one a launch of this library) times the steps
+        "gpu_launches": None if launches is None else launches * a.steps,
+        "e2e": {"value": D.job_throughput(T, world, e2e_ms * 1e-3), "unit": UNIT,
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": T * cfg.D * es,
+                "d2h_bytes_per_step": T * cfg.D * es},
+        "cpu_baseline": cpu,
+    }
     del graph
+    lay.close()
     del lay
+    return res
+
+
+# the other workloads of the headline metric, timed after the headline one on
+# the same weights (Ultra shape, bf16 dense weights; NVFP4 layers quantise them)
+EXTRA_WORKLOADS = ["ultra_prefill_bf16", "ultra_decode_w4a16", "skewed_prefill_w4a4"]
+
+
+def run_ours(a):
+    import torch
+    from latentmoe_expert_routing_b200 import dist as D
+    rank, world, local = _dist()
+    torch.cuda.set_device(local)
+    D.init("nccl", 300, torch.device("cuda", local))
+    from latentmoe_expert_routing_b200 import inputs as I
+    cfg = I.CONFIGS[a.config]
+    W = _weights(cfg, "cuda")
+    head = _measure(a, cfg, W, rank, world, local,
+                    cpu_leg=rank == 0 and world == 1 and not a.no_cpu_baseline)
+    extras = {}
+    names = EXTRA_WORKLOADS if a.workloads == "all" else \
+        [] if a.workloads == "none" else a.workloads.split(",")
+    if a.workloads == "auto":
+        names = EXTRA_WORKLOADS if (world == 1 and cfg.name == "ultra_decode_bf16") else []
+    for name in names:
+        c = I.CONFIGS[name]
+        same = all(getattr(c, f) == getattr(cfg, f) for f in ("D", "L", "E", "F", "Fs", "dtype"))
+        Wc = dict(W) if same else _weights(c, "cuda")
+        if c.bias_kind != cfg.bias_kind:
+            Wc["gate_bias"] = I.gate_bias(c, "cuda")
+        torch.cuda.empty_cache()
+        extras[name] = _measure(a, c, Wc, rank, world, local, cpu_leg=False)
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+                "steps": a.steps, "warmup": max(a.warmup, 3),
+                "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "data": "synthetic"}
+        line.update({k: v for k, v in head.items() if k not in ("value", "ms_per_step")})
+        if extras:
+            line["workloads"] = extras
+        print(json.dumps(line))
     D.finish()
     return 0
 

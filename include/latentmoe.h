@@ -55,7 +55,8 @@ typedef enum {
   MOE_ERR_OOM = 3,           /* device allocation failed in moe_init       */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed                 */
   MOE_ERR_TIMEOUT = 5,       /* a bounded device wait gave up              */
-  MOE_ERR_DEVICE_CHECK = 6   /* a kernel saw an out-of-range index         */
+  MOE_ERR_DEVICE_CHECK = 6   /* a kernel saw an out-of-range index or a    */
+                             /* NaN router logit                           */
 } moe_status;
 
 typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
@@ -91,28 +92,54 @@ typedef struct {
   moe_dtype out_dtype;           /* dtype of `out`                           */
 } moe_config;
 
-/* Weights, all DEVICE pointers, row-major [out, in].  With borrow != 0 the
- * library keeps the pointers and the caller must keep the memory alive and
- * unchanged until moe_destroy(); with borrow == 0 moe_init copies them.
- * Dense experts are read from w_up/w_down; NVFP4 formats quantise w_up/w_down
- * at init into library-owned codes and scales (the caller's dense experts may
- * be freed after moe_init returns). */
+/* Weights, row-major [out, in] (report section 2.3.4).  Pointers are device
+ * pointers when weights_on_device != 0, host pointers otherwise (moe_init then
+ * copies them to library-owned device memory; pinned host memory copies
+ * fastest).  Every pointer must be 16-byte aligned.
+ *
+ * Dense weights.  With borrow != 0 (device pointers only) the library keeps
+ * the pointers and the caller must keep the memory alive and unchanged until
+ * moe_destroy(); with borrow == 0 moe_init copies them.
+ *
+ * Routed experts.  MOE_EXPERT_DENSE reads w_up / w_down.  The NVFP4 formats
+ * (report section 8.1; NVFP4 format details) take EITHER dense w_up / w_down,
+ * which moe_init quantises (moe_quantize_nvfp4's arithmetic) and does not
+ * keep, OR the pre-quantised tensors below with w_up = w_down = NULL, as an
+ * NVFP4 checkpoint ships them:
+ *   codes  [E, rows, K/2]  E2M1, two per byte, the even element in the low nibble
+ *   scales [E, rows, K/16] E4M3 block scales, one per 16 consecutive elements along K
+ *   gscale [E]             fp32 global scale of each expert matrix
+ * with (rows, K) = (F, L) for up and (L, F) for down; a weight is
+ * value(code) * value(scale) * gscale.  moe_init repacks them into its own
+ * layouts; the caller may free them once moe_init returns.  NaN scales (E4M3
+ * code 0x7F / 0xFF) are not accepted by the GEMMs and give undefined output. */
 typedef struct {
   const void* w_gate;          /* [E, D]  dtype                               */
-  const float* gate_bias;      /* [E]     fp32 e_score_correction_bias        */
+  const float* gate_bias;      /* [E]     fp32 e_score_correction_bias, finite */
   const void* w_fc1;           /* [L, D]  dtype                               */
   const void* w_fc2;           /* [D, L]  dtype                               */
   const void* w_shared_up;     /* [Fs, D] dtype                               */
   const void* w_shared_down;   /* [D, Fs] dtype                               */
-  const void* w_up;            /* [E, F, L] dtype                             */
-  const void* w_down;          /* [E, L, F] dtype                             */
+  const void* w_up;            /* [E, F, L] dtype, or NULL (pre-quantised)    */
+  const void* w_down;          /* [E, L, F] dtype, or NULL (pre-quantised)    */
   int borrow;
+  const uint8_t* up_codes;     /* [E, F, L/2]   pre-quantised NVFP4, or NULL  */
+  const uint8_t* up_scales;    /* [E, F, L/16]                                */
+  const float* up_gscale;      /* [E]                                         */
+  const uint8_t* down_codes;   /* [E, L, F/2]                                 */
+  const uint8_t* down_scales;  /* [E, L, F/16]                                */
+  const float* down_gscale;    /* [E]                                         */
+  int weights_on_device;       /* 1: device pointers; 0: host pointers        */
 } moe_weights;
 
 typedef struct moe_handle moe_handle;
 
-/* Validate cfg, allocate the workspace for cfg->max_tokens and take the
- * weights (see moe_weights).  Synchronises `stream` before returning. */
+/* Validate cfg and the weights, allocate the workspace for cfg->max_tokens and
+ * take the weights (see moe_weights).  MOE_ERR_INVALID_ARG for a NULL or
+ * misaligned pointer, a non-finite gate_bias entry, borrow != 0 with host
+ * pointers, or an expert source that is neither complete dense nor complete
+ * pre-quantised (pre-quantised tensors need an NVFP4 format).  Synchronises
+ * `stream` before returning. */
 moe_status moe_init(moe_handle** handle, const moe_config* cfg,
                     const moe_weights* weights, void* stream);
 
@@ -171,6 +198,10 @@ moe_status moe_forward_host(moe_handle* handle, const void* hidden_host, int T,
 moe_status moe_get_routing(moe_handle* handle, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* pos, void* stream);
 
+/* Tokens per expert of the last forward: counts [E] int32, device, async on
+ * `stream` (the same values moe_get_routing writes). */
+moe_status moe_get_expert_counts(moe_handle* handle, int32_t* counts, void* stream);
+
 /* Stage timing.  With `on` != 0 every later moe_forward records a CUDA event
  * on its stream before each stage; moe_profile_read() waits for the last
  * forward's events and writes up to n stage durations in milliseconds, in the
@@ -188,9 +219,11 @@ enum {
 moe_status moe_profile_enable(moe_handle* handle, int on);
 moe_status moe_profile_read(moe_handle* handle, float* stage_ms, int n);
 
-/* Router only -- logits, sigmoid, biased top-k and weights, the same results
- * bit for bit as moe_forward's topk_idx / topk_w -- for callers that cannot
- * allocate device memory.  The report has no counterpart of this entry point.
+/* Router only -- logits, sigmoid, biased top-k over all experts and weights,
+ * the same results bit for bit as moe_forward's topk_idx / topk_w on a layer
+ * with n_group == 1 (this call has no group routing) -- for callers that
+ * cannot allocate device memory.  The report has no counterpart of this entry
+ * point.
  *
  * Some callers may not call cudaMalloc or let a library call it: a serving
  * loop that owns every byte of a fixed HBM budget, a framework whose allocator
@@ -207,8 +240,16 @@ moe_status moe_profile_read(moe_handle* handle, float* stage_ms, int n);
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  All calls on a device share the one array and
  * it keeps the last call's contents, so calls that overlap on the GPU (other
- * streams, other host threads) race: serialise them.  The error word is
- * cleared at the start of each call.
+ * streams, other host threads) race: serialise them.
+ *
+ * Errors.  Arguments are checked on the host before any launch; a CUDA error
+ * already pending on the calling thread returns MOE_ERR_CUDA before the array
+ * is touched (the pending error is left for its owner).  Problems the kernels
+ * detect -- a NaN router logit, or a token slot that cannot be filled because
+ * fewer than top_k experts have a choice score above -inf (such a slot's index
+ * is written as 0x7fffffff) -- set the array's error word, which accumulates
+ * over calls until moe_sync(NULL, stream) drains `stream` and reports and
+ * clears it (MOE_ERR_DEVICE_CHECK).
  *   hidden [T, d_model] dtype, w_gate [n_experts, d_model] dtype, gate_bias
  *   [n_experts] fp32, topk_idx [T, top_k] int32, topk_w [T, top_k] fp32: all
  *   device pointers, hidden and w_gate 16-byte aligned.  Asynchronous. */
@@ -264,7 +305,11 @@ moe_status moe_selftest_wait_timeout(moe_handle* handle, int microseconds, void*
  * MOE_ERR_CUDA on a launch or copy failure. */
 moe_status moe_selftest_nvfp4_convert(unsigned long long* mismatches_host, void* stream);
 
-/* Drain `stream` and report (then clear) the device error word. */
+/* Drain `stream` and report (then clear) the handle's device error word:
+ * MOE_ERR_TIMEOUT when a bounded wait gave up, MOE_ERR_DEVICE_CHECK for the
+ * other device-side checks.  With handle == NULL the word reported is
+ * moe_route_noalloc's, in its fixed array on the current device (MOE_OK when
+ * no such call ran there). */
 moe_status moe_sync(moe_handle* handle, void* stream);
 
 /* Free everything moe_init allocated.  NULL is ignored. */

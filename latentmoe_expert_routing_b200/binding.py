@@ -38,7 +38,11 @@ class moe_weights(ctypes.Structure):
                 ("w_fc1", ctypes.c_void_p), ("w_fc2", ctypes.c_void_p),
                 ("w_shared_up", ctypes.c_void_p), ("w_shared_down", ctypes.c_void_p),
                 ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
-                ("borrow", ctypes.c_int)]
+                ("borrow", ctypes.c_int),
+                ("up_codes", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
+                ("up_gscale", ctypes.c_void_p), ("down_codes", ctypes.c_void_p),
+                ("down_scales", ctypes.c_void_p), ("down_gscale", ctypes.c_void_p),
+                ("weights_on_device", ctypes.c_int)]
 
 
 class MoeError(RuntimeError):
@@ -56,6 +60,7 @@ SIGNATURES = [
     ("moe_block_forward", _i, [_vp, _vp, _i, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]),
     ("moe_rmsnorm", _i, [_vp, _vp, _i, _i, ctypes.c_float, _i, _vp, _vp]),
     ("moe_get_routing", _i, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    ("moe_get_expert_counts", _i, [_vp, _vp, _vp]),
     ("moe_profile_enable", _i, [_vp, _i]),
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
     ("moe_route_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i,
@@ -132,6 +137,10 @@ def moe_get_routing(h, counts, offsets, perm, pos, stream):
 MOE_NUM_STAGES = 7
 STAGES = ["router_logits", "route", "dense_in", "expert_up", "expert_down",
           "combine", "dense_out"]
+
+
+def moe_get_expert_counts(h, counts, stream):
+    _check(_lib.moe_get_expert_counts(h, counts, stream), "moe_get_expert_counts")
 
 
 def moe_profile_enable(h, on):

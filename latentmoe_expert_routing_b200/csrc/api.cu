@@ -45,7 +45,6 @@ struct moe_handle {
   float* splitws = nullptr;                      // split-K partials of the dense GEMMs
   size_t splitws_elems = 0;
   int sms = 148;
-  uint32_t* cmask = nullptr;                     // [T, 32] candidate bits per token
   // NVFP4 experts: GEMM-layout records and per-expert global scales
   uint8_t *rec_up = nullptr, *rec_dn = nullptr;
   CUtensorMap rm_up[3], rm_dn[3];                // record maps, batches of 1, 2, 4
@@ -198,47 +197,82 @@ int max_tiles(const moe_config& c, int T, int N) {
   return t > 0x7fffffff ? 0x7fffffff : (int)t;
 }
 
-// NVFP4 experts: quantise up [E,F,L] and down [E,L,F] (plain layout, in
-// temporary buffers), then repack into the GEMM records the kernel streams.
-moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
+// NVFP4 experts: the plain layout (codes [E,rows,K/2], E4M3 scales [E,rows,K/16],
+// global scales [E]) of up [E,F,L] and down [E,L,F] -- taken from the caller's
+// pre-quantised tensors, or made by quantising the caller's dense experts --
+// repacked into the GEMM records the kernels stream.  W4A4 keeps the plain
+// layout too (the block-scaled FP4 GEMMs read it) plus its scale atoms.
+// Host sources are staged through temporary device buffers.
+struct TempBuf {
+  void* p = nullptr;
+  ~TempBuf() { if (p) cudaFree(p); }
+  bool alloc(size_t bytes) {
+    if (cudaMalloc(&p, bytes ? bytes : 16) == cudaSuccess) return true;
+    cudaGetLastError();
+    p = nullptr;
+    return false;
+  }
+};
+
+moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s) {
   const moe_config& c = h->cfg;
   const size_t E = c.n_experts, F = c.d_ff, L = c.d_latent;
   const size_t recs_up = E * ((F + 127) / 128) * (L / 64), recs_dn = E * ((L + 127) / 128) * (F / 64);
   if (!dev_alloc(h, &h->rec_up, recs_up * 4608) || !dev_alloc(h, &h->rec_dn, recs_dn * 4608) ||
       !dev_alloc(h, &h->gs_up, E * 4) || !dev_alloc(h, &h->gs_dn, E * 4))
     return MOE_ERR_OOM;
-  uint8_t *codes = nullptr, *scales = nullptr;
-  unsigned* amax = nullptr;
   const size_t n = E * F * L;
   const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
+  const bool pre = w->up_codes != nullptr;
+  const bool dev = w->weights_on_device != 0;
+  TempBuf codes, scales, dense, amax;
   if (w4a4) {                // kept: the block-scaled FP4 GEMMs read the plain layout
     if (!dev_alloc(h, &h->wc_up, n / 2) || !dev_alloc(h, &h->ws_up, n / 16) ||
         !dev_alloc(h, &h->wc_dn, n / 2) || !dev_alloc(h, &h->ws_dn, n / 16))
       return MOE_ERR_OOM;
-  } else if (cudaMalloc(&codes, n / 2) != cudaSuccess || cudaMalloc(&scales, n / 16) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(codes); cudaFree(scales);
+  } else if (!(pre && dev) && (!codes.alloc(n / 2) || !scales.alloc(n / 16))) {
     return MOE_ERR_OOM;
   }
-  if (cudaMalloc(&amax, E * 4) != cudaSuccess) {
-    cudaGetLastError();
-    if (!w4a4) { cudaFree(codes); cudaFree(scales); }
-    return MOE_ERR_OOM;
-  }
-  uint8_t *cu = w4a4 ? h->wc_up : codes, *su = w4a4 ? h->ws_up : scales;
-  uint8_t *cd = w4a4 ? h->wc_dn : codes, *sd = w4a4 ? h->ws_dn : scales;
+  if (!pre && (!amax.alloc(E * 4) || (!dev && !dense.alloc(n * 2)))) return MOE_ERR_OOM;
   // W4A4 streams fp16 operands: its records keep the plain nibble order
-  const int natural = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
-  cudaError_t e = launch_quantize_nvfp4(h->w_up, MOE_BF16, (int)E, (int)F, (int)L, cu, su,
-                                        h->gs_up, amax, s);
-  if (e == cudaSuccess)
-    e = launch_repack_gemm(cu, su, (int)E, (int)F, (int)L, h->rec_up, natural, s);
-  if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_up, h->gs_up, (int)E, s);
-  if (e == cudaSuccess)
-    e = launch_quantize_nvfp4(h->w_down, MOE_BF16, (int)E, (int)L, (int)F, cd, sd, h->gs_dn,
-                              amax, s);
-  if (e == cudaSuccess)
-    e = launch_repack_gemm(cd, sd, (int)E, (int)L, (int)F, h->rec_dn, natural, s);
+  const int natural = w4a4;
+  struct Proj {
+    int rows, K;
+    const void* dense;
+    const uint8_t *codes, *scales;
+    const float* gs_src;
+    uint8_t *keep_c, *keep_s, *rec;
+    float* gs;
+  } proj[2] = {
+      {(int)F, (int)L, w->w_up, w->up_codes, w->up_scales, w->up_gscale, h->wc_up, h->ws_up,
+       h->rec_up, h->gs_up},
+      {(int)L, (int)F, w->w_down, w->down_codes, w->down_scales, w->down_gscale, h->wc_dn,
+       h->ws_dn, h->rec_dn, h->gs_dn}};
+  cudaError_t e = cudaSuccess;
+  for (const Proj& q : proj) {
+    uint8_t* cu = w4a4 ? q.keep_c : (pre && dev) ? const_cast<uint8_t*>(q.codes)
+                                                 : static_cast<uint8_t*>(codes.p);
+    uint8_t* su = w4a4 ? q.keep_s : (pre && dev) ? const_cast<uint8_t*>(q.scales)
+                                                 : static_cast<uint8_t*>(scales.p);
+    if (pre) {
+      if (cu != q.codes) e = cudaMemcpyAsync(cu, q.codes, n / 2, cudaMemcpyDefault, s);
+      if (e == cudaSuccess && su != q.scales)
+        e = cudaMemcpyAsync(su, q.scales, n / 16, cudaMemcpyDefault, s);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(q.gs, q.gs_src, E * 4, cudaMemcpyDefault, s);
+    } else {
+      const void* src = q.dense;
+      if (!dev) {
+        e = cudaMemcpyAsync(dense.p, q.dense, n * 2, cudaMemcpyDefault, s);
+        src = dense.p;
+      }
+      if (e == cudaSuccess)
+        e = launch_quantize_nvfp4(src, MOE_BF16, (int)E, q.rows, q.K, cu, su, q.gs,
+                                  static_cast<unsigned*>(amax.p), s);
+    }
+    if (e == cudaSuccess) e = launch_repack_gemm(cu, su, (int)E, q.rows, q.K, q.rec, natural, s);
+    if (e == cudaSuccess) e = launch_gemm_gscale(q.gs, q.gs, (int)E, s);
+    if (e != cudaSuccess) break;
+  }
   if (e == cudaSuccess && w4a4 && L % 256 == 0 && F % 256 == 0 &&
       !(make_tmap_u8(&h->mx_up.wcode, h->wc_up, (long)(E * F), (int)(L / 2), 128, 128, true) &&
         make_tmap_u8(&h->mx_up.wscale, h->ws_up, (long)(E * F), (int)(L / 16), 16, 128, false) &&
@@ -248,10 +282,7 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
   if (e == cudaSuccess && w4a4 && L % 256 == 0 && F % 256 == 0) {
     // the weights' scales again as atoms for the SM-pair GEMMs (256-byte rows,
     // one 8-row box = one 256-K stage of a 128-row block)
-    if (!dev_alloc(h, &h->wa_up, n / 16) || !dev_alloc(h, &h->wa_dn, n / 16)) {
-      cudaFree(amax);
-      return MOE_ERR_OOM;
-    }
+    if (!dev_alloc(h, &h->wa_up, n / 16) || !dev_alloc(h, &h->wa_dn, n / 16)) return MOE_ERR_OOM;
     e = launch_sf_atoms(h->ws_up, (long)(E * F), (int)L, h->wa_up, s);
     if (e == cudaSuccess) e = launch_sf_atoms(h->ws_dn, (long)(E * L), (int)F, h->wa_dn, s);
     h->mxp_up.wcode = h->mx_up.wcode;
@@ -261,13 +292,13 @@ moe_status quantize_experts(moe_handle* h, cudaStream_t s) {
           make_tmap_u8(&h->mxp_dn.wscale, h->wa_dn, (long)(n / 16 / 256), 256, 256, 8, false)))
       e = cudaErrorInvalidValue;
   }
-  if (e == cudaSuccess) e = launch_gemm_gscale(h->gs_dn, h->gs_dn, (int)E, s);
   for (int i = 0; i < 3 && e == cudaSuccess; ++i)
     if (!make_tmap_records(&h->rm_up[i], h->rec_up, (long)recs_up, 1 << i) ||
         !make_tmap_records(&h->rm_dn[i], h->rec_dn, (long)recs_dn, 1 << i))
       e = cudaErrorInvalidValue;
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  cudaFree(codes); cudaFree(scales); cudaFree(amax);
+  // the temporary buffers are freed on return: drain their users first
+  const cudaError_t sync = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = sync;
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -449,9 +480,35 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const void* ptrs[] = {w->w_gate, w->gate_bias, w->w_fc1, w->w_fc2, w->w_shared_up,
-                        w->w_shared_down, w->w_up, w->w_down};
+                        w->w_shared_down};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  // the routed experts: complete dense tensors, or complete pre-quantised NVFP4
+  const void* pq[] = {w->up_codes, w->up_scales, w->up_gscale, w->down_codes, w->down_scales,
+                      w->down_gscale};
+  int n_pre = 0;
+  for (const void* p : pq) n_pre += p != nullptr;
+  if (n_pre == 6) {
+    if (w->w_up || w->w_down || cfg->expert_fmt == MOE_EXPERT_DENSE) return MOE_ERR_INVALID_ARG;
+    for (const void* p : pq)
+      if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  } else if (n_pre != 0 || !w->w_up || !w->w_down || !aligned16(w->w_up) ||
+             !aligned16(w->w_down)) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  const bool on_dev = w->weights_on_device != 0;
+  if (w->borrow && !on_dev) return MOE_ERR_INVALID_ARG;
+  {
+    // e_score_correction_bias must be finite: the selection kernels reserve
+    // -inf for experts that may not be chosen
+    std::vector<float> b(cfg->n_experts);
+    if (cudaMemcpy(b.data(), w->gate_bias, b.size() * 4, cudaMemcpyDefault) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_INVALID_ARG;
+    }
+    for (float v : b)
+      if (!(v - v == 0.f)) return MOE_ERR_INVALID_ARG;
+  }
   moe_handle* h = new (std::nothrow) moe_handle();
   if (!h) return MOE_ERR_OOM;
   h->cfg = *cfg;
@@ -461,23 +518,27 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
   const size_t T = c.max_tokens, k = c.top_k, P = T * k, nblk = (T + 31) / 32;
   const size_t ds = dt_size(c.dtype);
   cudaStream_t s = (cudaStream_t)stream;
+  // NVFP4 layers read their dense experts (if given) only while quantising
+  const bool dense_experts = c.expert_fmt == MOE_EXPERT_DENSE;
   bool ok = true;
   if (w->borrow) {
     h->w_gate = w->w_gate; h->w_fc1 = w->w_fc1; h->w_fc2 = w->w_fc2;
-    h->w_su = w->w_shared_up; h->w_sd = w->w_shared_down;
-    h->w_up = w->w_up; h->w_down = w->w_down; h->bias = w->gate_bias;
+    h->w_su = w->w_shared_up; h->w_sd = w->w_shared_down; h->bias = w->gate_bias;
+    if (dense_experts) { h->w_up = w->w_up; h->w_down = w->w_down; }
   } else {
     struct { const void* src; const void** dst; size_t bytes; } cp[] = {
         {w->w_gate, &h->w_gate, E * D * ds},    {w->w_fc1, &h->w_fc1, L * D * ds},
         {w->w_fc2, &h->w_fc2, D * L * ds},      {w->w_shared_up, &h->w_su, Fs * D * ds},
-        {w->w_shared_down, &h->w_sd, D * Fs * ds}, {w->w_up, &h->w_up, E * F * L * ds},
-        {w->w_down, &h->w_down, E * L * F * ds}, {w->gate_bias, (const void**)&h->bias, E * 4}};
+        {w->w_shared_down, &h->w_sd, D * Fs * ds}, {w->gate_bias, (const void**)&h->bias, E * 4},
+        {w->w_up, &h->w_up, E * F * L * ds},    {w->w_down, &h->w_down, E * L * F * ds}};
     for (auto& q : cp) {
+      if (!dense_experts && (q.dst == &h->w_up || q.dst == &h->w_down)) continue;
       void* d = nullptr;
       ok = ok && dev_alloc(h, &d, q.bytes);
       if (!ok) break;
       *q.dst = d;
-      if (cudaMemcpyAsync(d, q.src, q.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+      // host or device source (unified addressing tells which)
+      if (cudaMemcpyAsync(d, q.src, q.bytes, cudaMemcpyDefault, s) != cudaSuccess) {
         moe_destroy(h);
         return MOE_ERR_CUDA;
       }
@@ -504,7 +565,6 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
     if (!dev_alloc(h, &h->splitws, h->splitws_elems * 4) ||
         !dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
         !dev_alloc(h, &h->wstat, E * 8) ||
-        !dev_alloc(h, &h->cmask, T * 32 * 4) ||
         !dev_alloc(h, &h->stats, 16)) {
       moe_destroy(h);
       return MOE_ERR_OOM;
@@ -514,8 +574,8 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
     bool m = make_tmap_bf16(&h->wm_gate, h->w_gate, E, D, 128) &&
              make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
              make_tmap_bf16(&h->wm_su, h->w_su, Fs, D, 128) &&
-             make_tmap_bf16(&h->wm_up, h->w_up, E * F, L, 128) &&
-             make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128) &&
+             (!dense_experts || (make_tmap_bf16(&h->wm_up, h->w_up, E * F, L, 128) &&
+                                 make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128))) &&
              make_tmap_bf16(&h->wm_fc2, h->w_fc2, D, L, 128) &&
              make_tmap_bf16(&h->wm_sd, h->w_sd, D, Fs, 128);
     for (int i = 0; i < 4 && m; ++i)
@@ -525,7 +585,7 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
           make_tmap_bf16(&h->am_hsh[i], h->h_sh, T, Fs, kNT[i]);
     if (!m) { moe_destroy(h); return MOE_ERR_CUDA; }
     if (c.expert_fmt != MOE_EXPERT_DENSE) {
-      moe_status q = quantize_experts(h, s);
+      moe_status q = quantize_experts(h, w, s);
       if (q != MOE_OK) { moe_destroy(h); return q; }
     }
     if (c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 && L % 256 == 0 && F % 256 == 0) {
@@ -625,7 +685,6 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   }
   ra.tiles_up = h->tiles_up; ra.tiles_dn = h->tiles_dn;
   ra.err = h->err;
-  ra.cmask = dt == MOE_BF16 ? h->cmask : nullptr;
   ra.n_group = c.n_group; ra.topk_group = c.topk_group;
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
@@ -772,6 +831,11 @@ moe_status moe_get_routing(moe_handle* h, int32_t* counts, int32_t* offsets, int
   return cuda_status(e);
 }
 
+moe_status moe_get_expert_counts(moe_handle* h, int32_t* counts, void* stream) {
+  if (!h || !counts) return MOE_ERR_INVALID_ARG;
+  return moe_get_routing(h, counts, nullptr, nullptr, nullptr, stream);
+}
+
 moe_status moe_profile_enable(moe_handle* h, int on) {
   if (!h) return MOE_ERR_INVALID_ARG;
   if (on && !h->ev[0]) {
@@ -855,16 +919,17 @@ moe_status moe_selftest_nvfp4_convert(unsigned long long* mismatches_host, void*
 }
 
 moe_status moe_sync(moe_handle* h, void* stream) {
-  if (!h) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   int word = 0;
-  if (cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (word) {
-    cudaMemset(h->err, 0, sizeof(int));
-    return (word & DEV_ERR_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE_CHECK;
+  if (!h) {                      // the error word of moe_route_noalloc's fixed array
+    if (noalloc_take_error(&word) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    if (cudaMemcpy(&word, h->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (word) cudaMemset(h->err, 0, sizeof(int));
   }
+  if (word) return (word & DEV_ERR_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE_CHECK;
   return MOE_OK;
 }
 

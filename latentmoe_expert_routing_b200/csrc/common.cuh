@@ -12,6 +12,7 @@ namespace lmoe {
 enum : int {
   DEV_ERR_INDEX = 1,     // an expert / row index outside its range
   DEV_ERR_TIMEOUT = 2,   // a bounded wait gave up
+  DEV_ERR_NONFINITE = 4, // a router logit was NaN
 };
 
 struct bf16x8 { __nv_bfloat162 v[4]; };

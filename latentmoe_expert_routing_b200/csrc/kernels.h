@@ -29,7 +29,6 @@ struct RouteArgs {
   int mt_dn, nc_dn;
   int32_t* tiles_dn;    // [E + 1]
   int* err;
-  uint32_t* cmask;           // [T, ceil(E/32)] candidate bits (certified router) or NULL
   int n_group, topk_group;   // group routing (section 5.5); n_group <= 1: all experts compete
 };
 
@@ -99,6 +98,8 @@ namespace lmoe {
 // Selection-only launch (sigmoid, +bias, top-k, weights) over precomputed
 // logits; rank / blkcnt are written for a caller that goes on to group pairs.
 void launch_route_select(const RouteArgs& a, cudaStream_t st);
+// moe_route_noalloc's device error word: read, then cleared (synchronous).
+cudaError_t noalloc_take_error(int* word);
 }  // namespace lmoe
 
 #include <cuda.h>

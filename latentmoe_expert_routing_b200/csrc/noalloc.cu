@@ -74,6 +74,8 @@ extern "C" moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
     return MOE_ERR_INVALID_ARG;
   if (scratch_bytes(T, n_experts, top_k) > kScratchBytes)
     return MOE_ERR_INVALID_ARG;   // more tokens than the fixed scratch holds
+  // an error left pending by earlier work on this thread is not ours to clear
+  if (cudaPeekAtLastError() != cudaSuccess) return MOE_ERR_CUDA;
   unsigned char* base = nullptr;
   moe_status st = scratch_for_current_device(&base);
   if (st != MOE_OK) return st;
@@ -84,9 +86,8 @@ extern "C" moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
   int32_t* rank = reinterpret_cast<int32_t*>(base + kErrBytes + align256(size_t(T) * n_experts * 4));
   int32_t* blkcnt = reinterpret_cast<int32_t*>(
       reinterpret_cast<unsigned char*>(rank) + align256(size_t(T) * top_k * 4));
-  // logits, rank and blkcnt are fully rewritten by each call; only the error
-  // word accumulates (OR) and is cleared here.
-  if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  // logits, rank and blkcnt are fully rewritten by each call; the error word
+  // accumulates (OR) until moe_sync(NULL, stream) reads and clears it.
   lmoe::launch_router_logits(hidden, w_gate, logits, T, d_model, n_experts, dtype, s);
   lmoe::RouteArgs ra{};
   ra.logits = logits; ra.bias = gate_bias; ra.T = T; ra.E = n_experts; ra.k = top_k;
@@ -95,3 +96,25 @@ extern "C" moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
   lmoe::launch_route_select(ra, s);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+namespace lmoe {
+
+// The error word of the fixed array on the current device: copied out and then
+// cleared (both synchronous).  0 when no call has used the array on this device.
+cudaError_t noalloc_take_error(int* word) {
+  *word = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (dev >= 0 && dev < kMaxDevices) p = g_ptr[dev];
+  }
+  if (!p) return cudaSuccess;
+  e = cudaMemcpy(word, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && *word) e = cudaMemset(p, 0, sizeof(int));
+  return e;
+}
+
+}  // namespace lmoe

@@ -155,8 +155,7 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
              int n_tok, int E, int k, float rsf,
              int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
              int32_t* __restrict__ rank, int32_t* __restrict__ blkcnt, int nblk,
-             int* __restrict__ err, const uint32_t* __restrict__ cmask, int n_group,
-             int topk_group) {
+             int* __restrict__ err, int n_group, int topk_group) {
   extern __shared__ uint32_t mask[];                 // [E]
   __shared__ float rsel[32][kMaxTopK];
   __shared__ float gsc[32][kMaxGroups];
@@ -166,20 +165,21 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
   __syncthreads();
   if (t < n_tok) {
     float s[EPL], c[EPL];
+    bool nan = false;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      // cmask (optional): only these experts can be in the top-k; their
-      // logits have been recomputed exactly
-      const bool cand = cmask == nullptr || ((cmask[(size_t)t * EPL + i] >> lane) & 1u);
-      if (e < E && cand) {
-        s[i] = sigmoid_fixed(logits[(size_t)t * E + e]);
+      if (e < E) {
+        const float l = logits[(size_t)t * E + e];
+        nan |= l != l;
+        s[i] = sigmoid_fixed(l);
         c[i] = __fadd_rn(s[i], bias[e]);
       } else {
         s[i] = 0.f;
         c[i] = -INFINITY;
       }
     }
+    if (__any_sync(0xffffffffu, nan) && lane == 0) atomicOr(err, DEV_ERR_NONFINITE);
     if (n_group > 1) mask_groups_warp<EPL>(c, E, n_group, topk_group, lane, gsc[warp]);
     uint32_t taken = 0u;                             // bit i: expert lane+32i chosen
     for (int j = 0; j < k; ++j) {
@@ -228,8 +228,10 @@ route_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
   __syncthreads();
   if (t < n_tok) {
     for (int j = lane; j < k; j += 32) {
+      // a slot left unfilled (fewer than k choice scores above -inf) holds an
+      // out-of-range index, already reported in the error word
       const int e = topk_idx[(size_t)t * k + j];
-      rank[(size_t)t * k + j] = __popc(mask[e] & ((1u << warp) - 1u));
+      rank[(size_t)t * k + j] = (e >= 0 && e < E) ? __popc(mask[e] & ((1u << warp) - 1u)) : 0;
     }
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -314,12 +316,13 @@ __global__ void route_perm_kernel(const int32_t* __restrict__ topk_idx,
                                   const int32_t* __restrict__ rank,
                                   const int32_t* __restrict__ blkpre,
                                   const int32_t* __restrict__ offsets, int n_tok,
-                                  int k, int nblk, int32_t* __restrict__ perm,
+                                  int k, int nblk, int E, int32_t* __restrict__ perm,
                                   int32_t* __restrict__ pos) {
   const long p = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (p >= (long)n_tok * k) return;
   const int t = (int)(p / k);
   const int e = topk_idx[p];
+  if (e < 0 || e >= E) return;          // an unfilled slot, reported by the selection
   const int q = offsets[e] + blkpre[(size_t)e * nblk + (t >> 5)] + rank[p];
   pos[p] = q;
   perm[q] = (int32_t)p;
@@ -344,7 +347,7 @@ template <int EPL>
 static void route_launch_epl(const RouteArgs& a, cudaStream_t st) {
   route_kernel<EPL><<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(
       a.logits, a.bias, a.T, a.E, a.k, a.rsf, a.topk_idx, a.topk_w, a.rank,
-      a.blkcnt, a.nblk, a.err, a.cmask, a.n_group, a.topk_group);
+      a.blkcnt, a.nblk, a.err, a.n_group, a.topk_group);
 }
 
 void launch_route_select(const RouteArgs& a, cudaStream_t st) {
@@ -370,7 +373,7 @@ void launch_route(const RouteArgs& a, cudaStream_t st) {
                                         a.mt_dn, a.nc_dn, a.tiles_dn);
   const long P = (long)a.T * a.k;
   route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
-      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.E, a.perm, a.pos);
 }
 
 }  // namespace lmoe
@@ -740,7 +743,7 @@ void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st) 
                                         a.mt_dn, a.nc_dn, a.tiles_dn);
   const long P = (long)a.T * a.k;
   route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
-      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.perm, a.pos);
+      a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.E, a.perm, a.pos);
 }
 
 }  // namespace lmoe

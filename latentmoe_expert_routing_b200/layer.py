@@ -15,12 +15,23 @@ from . import binding as B
 _TORCH_DT = {"fp32": torch.float32, "bf16": torch.bfloat16}
 
 
+_DENSE_NAMES = ("w_gate", "gate_bias", "w_fc1", "w_fc2", "w_shared_up", "w_shared_down")
+_EXPERT_NAMES = ("w_up", "w_down")
+_NVFP4_NAMES = ("up_codes", "up_scales", "up_gscale", "down_codes", "down_scales",
+                "down_gscale")
+
+
 class LatentMoE:
-    """One LatentMoE layer bound to device weights (borrowed, not copied).
+    """One LatentMoE layer.
 
     weights: dict with w_gate [E,D], gate_bias [E] fp32, w_fc1 [L,D],
-    w_fc2 [D,L], w_shared_up [Fs,D], w_shared_down [D,Fs], w_up [E,F,L],
-    w_down [E,L,F], all contiguous cuda tensors in `dtype` (bias fp32)."""
+    w_fc2 [D,L], w_shared_up [Fs,D], w_shared_down [D,Fs] and either dense
+    experts w_up [E,F,L], w_down [E,L,F] or, for the NVFP4 formats, the
+    pre-quantised up_codes [E,F,L/2] / up_scales [E,F,L/16] / up_gscale [E]
+    and down_codes [E,L,F/2] / down_scales [E,L,F/16] / down_gscale [E]
+    (uint8, uint8, fp32).  All tensors contiguous and on one side: cuda
+    tensors are borrowed (the library keeps their pointers), cpu tensors are
+    copied by moe_init."""
 
     def __init__(self, D, L, E, k, F, Fs, weights, *, max_tokens, rsf=5.0,
                  dtype="bf16", expert_fmt="dense", out_dtype=None,
@@ -30,17 +41,20 @@ class LatentMoE:
         self.out_dtype = out_dtype or dtype
         self.max_tokens = max_tokens
         self._w = {n: t.contiguous() for n, t in weights.items()}
-        for n, t in self._w.items():
-            if not t.is_cuda:
-                raise ValueError(f"weight {n} must be a cuda tensor")
+        on_dev = {t.is_cuda for t in self._w.values()}
+        if len(on_dev) != 1:
+            raise ValueError("weights must all be cuda tensors or all cpu tensors")
+        on_dev = on_dev.pop()
         cfg = B.moe_config(D, L, E, k, F, Fs, n_group, topk_group, max_tokens,
                            float(rsf), B.DTYPE[dtype], B.EXPERT_FMT[expert_fmt],
                            B.DTYPE[self.out_dtype])
-        w = B.moe_weights(*(self._w[n].data_ptr() for n in (
-            "w_gate", "gate_bias", "w_fc1", "w_fc2", "w_shared_up",
-            "w_shared_down", "w_up", "w_down")), 1)
+        ptr = lambda n: self._w[n].data_ptr() if n in self._w else None
+        w = B.moe_weights(*(ptr(n) for n in _DENSE_NAMES + _EXPERT_NAMES), int(on_dev),
+                          *(ptr(n) for n in _NVFP4_NAMES), int(on_dev))
         self.cfg = cfg
         self.handle = B.moe_init(cfg, w, torch.cuda.current_stream().cuda_stream)
+        if not on_dev:
+            self._w = {}                      # copied by moe_init
 
     @property
     def stream(self) -> int:

@@ -52,7 +52,7 @@ def _cfg(B, **kw):
 
 
 def _w(B, ptr=4096):
-    return B.moe_weights(*([ptr] * 8), 1)
+    return B.moe_weights(*([ptr] * 8), 1, *([None] * 6), 1)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -82,7 +82,10 @@ def test_calls_on_null_handle(B):
     assert B.lib.moe_forward(None, None, 1, None, None, None, None) == 1
     assert B.lib.moe_forward_host(None, None, 1, None, None, None, None) == 1
     assert B.lib.moe_get_routing(None, None, None, None, None, None) == 1
-    assert B.lib.moe_sync(None, None) == 1
+    import torch
+    # NULL handle: drains the stream and reports the no-alloc router's error word
+    assert B.lib.moe_sync(None, None) == (0 if torch.cuda.is_available() else B.MOE_ERR_CUDA)
+    assert B.lib.moe_get_expert_counts(None, None, None) == 1
     B.lib.moe_destroy(None)
 
 
@@ -99,3 +102,23 @@ def test_block_entry_points_validate_before_any_launch(B):
     assert B.lib.moe_rmsnorm(p, p, -1, 64, 1e-5, B.MOE_BF16, p, None) == 1
     assert B.lib.moe_rmsnorm(p, p, 4, 0, 1e-5, B.MOE_BF16, p, None) == 1
     assert B.lib.moe_rmsnorm(p, p, 4, 64, 1e-5, 7, p, None) == 1
+
+
+def test_init_rejects_mixed_or_partial_expert_sources(B):
+    """Dense experts and pre-quantised NVFP4 tensors exclude each other, the
+    pre-quantised set must be complete and needs an NVFP4 format, and borrowed
+    weights must be device pointers: all answered before any device work."""
+    h = ctypes.c_void_p()
+    q = [4096] * 6
+    nv = _cfg(B, dtype=B.MOE_BF16, expert_fmt=B.MOE_EXPERT_NVFP4_W4A16)
+    cases = [
+        (nv, B.moe_weights(*([4096] * 8), 1, *q, 1)),                 # both sources
+        (nv, B.moe_weights(*([4096] * 6), None, None, 1, *q[:5], None, 1)),   # partial
+        (_cfg(B), B.moe_weights(*([4096] * 6), None, None, 1, *q, 1)),  # dense format
+        (nv, B.moe_weights(*([4096] * 6), None, None, 1, *q[:5], 4100, 1)),   # misaligned
+        (_cfg(B), B.moe_weights(*([4096] * 8), 1, *([None] * 6), 0)),   # borrow of host
+        (_cfg(B), B.moe_weights(*([4096] * 6), None, 4096, 1, *([None] * 6), 1)),
+    ]
+    for cfg, w in cases:
+        assert B.lib.moe_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(w), None) == 1
+        assert not h.value

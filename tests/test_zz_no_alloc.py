@@ -84,3 +84,36 @@ def test_noalloc_rejects_more_tokens_than_the_scratch_holds(mods):
     assert st == B.MOE_ERR_INVALID_ARG
     assert lib.moe_route_noalloc(p, p, p, 4, 8192, 512, 600, ctypes.c_float(5.0),
                                  B.MOE_BF16, p, p, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_reports_device_errors_through_moe_sync(mods):
+    """The no-alloc router cannot own an error flag in caller memory, so the
+    problems its kernels see are kept in the fixed array's error word:
+    moe_sync(NULL, stream) drains the stream and reports, then clears, it."""
+    B, LY = mods
+    cfg = I.CONFIGS["tiny_fp32"]
+    W = LY.weights_for(cfg, "cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    x = I.hidden(cfg, "cuda")
+    _noalloc(B, x, W, cfg, cfg.T)
+    assert B.lib.moe_sync(None, st) == B.MOE_OK            # a clean call
+    # NaN rows give NaN logits
+    xn = x.clone()
+    xn[3] = float("nan")
+    _noalloc(B, xn, W, cfg, cfg.T)
+    assert B.lib.moe_sync(None, st) == B.MOE_ERR_DEVICE_CHECK
+    assert B.lib.moe_sync(None, st) == B.MOE_OK            # read and cleared
+    # only k - 1 experts have a choice score above -inf: the last slot of
+    # every token cannot be filled
+    bias = W["gate_bias"].clone()
+    bias[cfg.k - 1:] = float("-inf")
+    idx, w = _noalloc(B, x, dict(W, gate_bias=bias), cfg, cfg.T)
+    assert B.lib.moe_sync(None, st) == B.MOE_ERR_DEVICE_CHECK
+    assert torch.all(idx[:, cfg.k - 1] == 0x7FFFFFFF)
+    assert torch.all((idx[:, :cfg.k - 1] >= 0) & (idx[:, :cfg.k - 1] < cfg.k - 1))
+    # the array works on after the errors
+    idx, w = _noalloc(B, x, W, cfg, cfg.T)
+    assert B.lib.moe_sync(None, st) == B.MOE_OK
+    _, ref_idx, ref_w = LY.layer_for(cfg, W, out_dtype="fp32")(x)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref_idx)
