@@ -198,6 +198,13 @@ moe_status moe_forward_host(moe_handle* handle, const void* hidden_host, int T,
 moe_status moe_get_routing(moe_handle* handle, int32_t* counts, int32_t* offsets,
                            int32_t* perm, int32_t* pos, void* stream);
 
+/* Router logits of the last forward: logits [T, E] fp32, device, async on
+ * `stream`.  fp32 layers: the defined (fixed-order fp64, rounded) logits.
+ * bf16 layers: the tensor-core logits the certified selection starts from,
+ * within its error bound of the defined ones (the experts it could not place
+ * by that bound were recomputed exactly; moe_get_router_stats counts them). */
+moe_status moe_get_router_logits(moe_handle* handle, float* logits, void* stream);
+
 /* Tokens per expert of the last forward: counts [E] int32, device, async on
  * `stream` (the same values moe_get_routing writes). */
 moe_status moe_get_expert_counts(moe_handle* handle, int32_t* counts, void* stream);

@@ -61,6 +61,7 @@ SIGNATURES = [
     ("moe_rmsnorm", _i, [_vp, _vp, _i, _i, ctypes.c_float, _i, _vp, _vp]),
     ("moe_get_routing", _i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     ("moe_get_expert_counts", _i, [_vp, _vp, _vp]),
+    ("moe_get_router_logits", _i, [_vp, _vp, _vp]),
     ("moe_profile_enable", _i, [_vp, _i]),
     ("moe_profile_read", _i, [_vp, _p(ctypes.c_float), _i]),
     ("moe_route_noalloc", _i, [_vp, _vp, _vp, _i, _i, _i, _i, ctypes.c_float, _i,
@@ -141,6 +142,10 @@ STAGES = ["router_logits", "route", "dense_in", "expert_up", "expert_down",
 
 def moe_get_expert_counts(h, counts, stream):
     _check(_lib.moe_get_expert_counts(h, counts, stream), "moe_get_expert_counts")
+
+
+def moe_get_router_logits(h, logits, stream):
+    _check(_lib.moe_get_router_logits(h, logits, stream), "moe_get_router_logits")
 
 
 def moe_profile_enable(h, on):

@@ -831,6 +831,14 @@ moe_status moe_get_routing(moe_handle* h, int32_t* counts, int32_t* offsets, int
   return cuda_status(e);
 }
 
+moe_status moe_get_router_logits(moe_handle* h, float* logits, void* stream) {
+  if (!h || !logits) return MOE_ERR_INVALID_ARG;
+  const size_t n = (size_t)h->last_T * h->cfg.n_experts;
+  if (!n) return MOE_OK;
+  return cuda_status(cudaMemcpyAsync(logits, h->logits, n * 4, cudaMemcpyDeviceToDevice,
+                                     (cudaStream_t)stream));
+}
+
 moe_status moe_get_expert_counts(moe_handle* h, int32_t* counts, void* stream) {
   if (!h || !counts) return MOE_ERR_INVALID_ARG;
   return moe_get_routing(h, counts, nullptr, nullptr, nullptr, stream);

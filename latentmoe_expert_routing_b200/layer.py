@@ -118,6 +118,13 @@ class LatentMoE:
                           perm.data_ptr(), pos.data_ptr(), self.stream)
         return counts, offsets, perm[:T * k], pos[:T * k]
 
+    def router_logits(self, T):
+        """[T, E] fp32 router logits of the last forward (tensor-core logits for
+        bf16 layers)."""
+        lg = torch.empty(T, self.dims["E"], dtype=torch.float32, device="cuda")
+        B.moe_get_router_logits(self.handle, lg.data_ptr(), self.stream)
+        return lg
+
     def router_stats(self) -> int:
         """Exactly recomputed (token, expert) logits since the last call."""
         return B.moe_get_router_stats(self.handle, self.stream)

@@ -379,11 +379,13 @@ def expert_weights_fp64(w: np.ndarray, fmt: str) -> np.ndarray:
 
 def forward(x, w_gate, bias, w_fc1, w_fc2, w_su, w_sd, get_up, get_down, *,
             k, rsf, expert_fmt="dense", n_group=1, topk_group=1,
-            norm_topk_prob=True):
+            norm_topk_prob=True, experts_prepared=False):
     """One LatentMoE layer on token rows x[T, D].
 
     get_up(e) -> up_proj[e] [F, L] and get_down(e) -> down_proj[e] [L, F] return
     the stored (bf16 / fp32) expert weights; NVFP4 formats quantise them here.
+    With experts_prepared they return instead what expert_weights_fp64 makes of
+    the stored weights (a caller may compute those once and reuse them).
     Returns a dict with out [T, D] fp64 and every routing intermediate."""
     x64 = np.asarray(x, dtype=np.float64)
     T = x64.shape[0]
@@ -397,8 +399,11 @@ def forward(x, w_gate, bias, w_fc1, w_fc2, w_su, w_sd, get_up, get_down, *,
     y = np.zeros((T, k, z.shape[1]), dtype=np.float64)                # step 6
     for e in np.nonzero(counts)[0]:
         tok, slot = np.nonzero(idx == e)
-        up = expert_weights_fp64(get_up(int(e)), expert_fmt)
-        down = expert_weights_fp64(get_down(int(e)), expert_fmt)
+        if experts_prepared:
+            up, down = get_up(int(e)), get_down(int(e))
+        else:
+            up = expert_weights_fp64(get_up(int(e)), expert_fmt)
+            down = expert_weights_fp64(get_down(int(e)), expert_fmt)
         h = relu2(z_in[tok] @ up.T)
         if expert_fmt == "w4a4":
             h = nvfp4_roundtrip_activation(h)

@@ -1,4 +1,7 @@
 """Helpers shared by the GPU parity tests: layer set-up, oracle runs, metrics."""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -55,3 +58,56 @@ def check_dispatch_properties(idx, counts, offsets, perm, pos, E):
     order = np.argsort(flat * (T * k) + np.arange(T * k), kind="stable")
     assert np.array_equal(np.asarray(perm), order)
     assert np.array_equal(np.asarray(perm)[np.asarray(pos)], np.arange(T * k))
+
+
+def prepared_oracle_rows(cfg, W, x_rows, rows):
+    """oracle_rows for sampled token rows of a full-size workload.  The oracle
+    walks the selected experts in ascending order; their matrices (the oracle's
+    own expert_weights_fp64, NVFP4 quantisation included) are made ahead of it
+    on host threads, a bounded window at a time."""
+    x = np32(x_rows[rows])
+    l = O.router_logits(x, np32(W["w_gate"]))
+    _, _, idx, _ = O.route(l, np32(W["gate_bias"]), cfg.k, cfg.rsf, cfg.n_group,
+                           cfg.topk_group)
+    need = sorted(set(idx.reshape(-1).tolist()))
+    nw = max(1, min(32, os.cpu_count() or 1))
+    jobs = [(name, e) for e in need for name in ("w_up", "w_down")]
+    make = lambda j: O.expert_weights_fp64(np32(W[j[0]][j[1]]), cfg.expert_fmt)
+    futs, nxt = {}, [0]
+    with ThreadPoolExecutor(max_workers=nw) as ex:
+        def get(name, e):
+            while nxt[0] < len(jobs) and len(futs) < 2 * nw:
+                futs[jobs[nxt[0]]] = ex.submit(make, jobs[nxt[0]])
+                nxt[0] += 1
+            return futs.pop((name, e)).result()
+        return O.forward(x, np32(W["w_gate"]), np32(W["gate_bias"]), np32(W["w_fc1"]),
+                         np32(W["w_fc2"]), np32(W["w_shared_up"]), np32(W["w_shared_down"]),
+                         lambda e: get("w_up", e), lambda e: get("w_down", e), k=cfg.k,
+                         rsf=cfg.rsf, expert_fmt=cfg.expert_fmt, n_group=cfg.n_group,
+                         topk_group=cfg.topk_group, experts_prepared=True)
+
+
+def ragged_tile_tokens(counts, offsets, perm, k, nt, n=4):
+    """Tokens of the last token tile (nt pairs per tile) of the most loaded
+    expert: that tile is ragged unless the count is a multiple of nt."""
+    counts, offsets, perm = (np.asarray(a) for a in (counts, offsets, perm))
+    e = int(np.argmax(counts))
+    c = int(counts[e])
+    start = int(offsets[e]) + (c - 1) // nt * nt
+    pairs = perm[start:int(offsets[e + 1])]
+    toks = sorted(set((pairs // k).tolist()))
+    return e, toks[:n // 2] + toks[-(n - n // 2):]
+
+
+def spread_rows(T, n, extra=(), seed=0):
+    """n distinct token rows: the first two and last two, `extra`, and evenly
+    spread others (sorted)."""
+    rows = {0, 1, T - 2, T - 1} | {int(r) for r in extra}
+    for r in np.linspace(0, T - 1, n + 2).astype(int):
+        if len(rows) >= n:
+            break
+        rows.add(int(r))
+    rng = np.random.RandomState(seed)
+    while len(rows) < n:
+        rows.add(int(rng.randint(T)))
+    return sorted(rows)

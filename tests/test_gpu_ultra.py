@@ -1,20 +1,29 @@
 """Ultra-shape parity at the full sizes and in the launch configuration the
-benchmark times: routing of every token (decode) or of sampled tokens
-(prefill) bit-exact against the oracle, the grouping checked by its defining
-properties at full size, and sampled output rows against the oracle."""
+benchmark times: routing of every token (decode) or of 512+ sampled tokens
+(prefill, every outlier row among them) bit-exact against the oracle, the
+grouping checked by its defining properties at full size, 16+ output rows
+against the oracle (first and last token tiles, the ragged last tile of the
+most loaded expert, outlier rows), and the tensor-core router logits against
+the error bound the certified selection relies on."""
 import numpy as np
 import pytest
 import torch
 
 from latentmoe_expert_routing_b200 import inputs as I
 from oracle import moe_oracle as O
-from tests.gpu_common import check_dispatch_properties, np32, oracle_rows, out_metrics
+from tests.gpu_common import (check_dispatch_properties, np32, prepared_oracle_rows,
+                              ragged_tile_tokens, spread_rows)
 from tests.test_gpu_parity import _assert_out
 
 pytestmark = pytest.mark.gpu
 
 DEC = I.CONFIGS["ultra_decode_bf16"]
 PRE = I.CONFIGS["ultra_prefill_bf16"]
+
+# the certified router's model of the tensor-core logit error (section on the
+# certified router in the library): |l~ - l| <= margin * gamma_K * ||x|| ||w||,
+# gamma_K = K u / (1 - K u), u = 2^-23, margin = 2
+MARGIN, U = 2.0, 2.0 ** -23
 
 
 @pytest.fixture(scope="module")
@@ -34,7 +43,7 @@ def _routing_oracle(cfg, W, x):
     return O.route(l, np32(W["gate_bias"]), cfg.k, cfg.rsf)
 
 
-def _check(cfg, ultra, sample_route, sample_out):
+def _check(cfg, ultra, route_rows, out_rows_fn, nt):
     L, W = ultra
     lay = L.layer_for(cfg, W, out_dtype="fp32")
     x = I.hidden(cfg, "cuda")
@@ -44,24 +53,61 @@ def _check(cfg, ultra, sample_route, sample_out):
     idx_h, w_h = idx.cpu().numpy(), np32(w)
     exact = lay.router_stats()           # certified router: every selected + band
     assert cfg.T * cfg.k <= exact <= cfg.T * cfg.E
-    check_dispatch_properties(idx_h, counts.cpu().numpy(), offsets.cpu().numpy(),
-                              perm.cpu().numpy(), pos.cpu().numpy(), cfg.E)
-    rows = sample_route
-    _, _, ridx, rw = _routing_oracle(cfg, W, x[rows])
-    assert np.array_equal(idx_h[rows], ridx)
-    assert np.array_equal(w_h[rows].view(np.int32), rw.view(np.int32))
-    r = oracle_rows(cfg, W, x, rows=sample_out)
-    _assert_out(out[sample_out], r["out"])
+    c_h, o_h, p_h = counts.cpu().numpy(), offsets.cpu().numpy(), perm.cpu().numpy()
+    check_dispatch_properties(idx_h, c_h, o_h, p_h, pos.cpu().numpy(), cfg.E)
+    _, _, ridx, rw = _routing_oracle(cfg, W, x[route_rows])
+    assert np.array_equal(idx_h[route_rows], ridx)
+    assert np.array_equal(w_h[route_rows].view(np.int32), rw.view(np.int32))
+    _, ragged = ragged_tile_tokens(c_h, o_h, p_h, cfg.k, nt)
+    rows = out_rows_fn(ragged)
+    assert len(rows) >= 16
+    r = prepared_oracle_rows(cfg, W, x, rows)
+    assert np.array_equal(idx_h[rows], r["topk_idx"])
+    _assert_out(out[rows], r["out"])
     lay.close()
-    return counts.cpu().numpy()
+    return c_h
 
 
 def test_ultra_decode_bf16(ultra):
-    counts = _check(DEC, ultra, list(range(DEC.T)), [0, 31, 63])
+    counts = _check(DEC, ultra, list(range(DEC.T)),
+                    lambda ragged: spread_rows(DEC.T, 16, extra=ragged), nt=16)
     assert counts.sum() == DEC.T * DEC.k
 
 
 def test_ultra_prefill_bf16(ultra):
     outl = I.outlier_rows(PRE)
-    rows = sorted(set([0, 1, 4095, 8191] + outl[:4] + list(range(3000, 3024))))
-    _check(PRE, ultra, rows, [0, outl[0], 8191])
+    rng = np.random.RandomState(5)
+    route = sorted(set(outl) | set(range(32)) | set(range(PRE.T - 32, PRE.T)) |
+                   set(rng.choice(PRE.T, 400, replace=False).tolist()))
+    assert len(route) >= 512 and set(outl) <= set(route)
+    _check(PRE, ultra, route,
+           lambda ragged: spread_rows(PRE.T, 18, extra=list(ragged) + outl[:6]), nt=256)
+
+
+def _logit_error_ratio(lt, x, W, K):
+    """max over (t, e) of |l~ - l| / (Delta / margin): the tensor-core logits'
+    error against the bound the certified router assumes, without its margin."""
+    xs, wg = np32(x).astype(np.float64), np32(W["w_gate"]).astype(np.float64)
+    l = O.router_logits(xs, wg).astype(np.float64)
+    gamma = K * U / (1 - K * U)
+    bound = gamma * np.linalg.norm(xs, axis=1)[:, None] * np.linalg.norm(wg, axis=1)[None, :]
+    return float(np.max(np.abs(lt.cpu().numpy().astype(np.float64) - l) / bound))
+
+
+def test_tensor_core_logits_within_the_certified_bound(ultra):
+    """The certified router assumes |l~ - l| <= margin * gamma_K ||x|| ||w||; the
+    observed error of the tensor-core logits must sit inside the bound even
+    without the margin, for the 64 decode tokens (split-K logits) and for 128
+    prefill tokens (one K pass per 256-token tile), outlier rows among them."""
+    L, W = ultra
+    ratios = {}
+    for cfg, rows in ((DEC, list(range(DEC.T))),
+                      (PRE, I.outlier_rows(PRE)[:64] + list(range(64)))):
+        lay = L.layer_for(cfg, W, out_dtype="fp32")
+        x = I.hidden(cfg, "cuda")
+        lay(x)
+        lay.sync()
+        ratios[cfg.name] = _logit_error_ratio(lay.router_logits(cfg.T)[rows], x[rows], W, cfg.D)
+        lay.close()
+    print("tensor-core logit error / bound:", ratios)
+    assert all(v <= 1.0 for v in ratios.values()), ratios

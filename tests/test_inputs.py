@@ -32,6 +32,16 @@ def test_cos_2pi_against_libm_and_quadrants():
     assert np.abs(got[-7] - math.sqrt(0.5)) <= 2e-16
 
 
+def test_sqrt_newton_against_libm():
+    rng = np.random.RandomState(2)
+    x = np.concatenate([rng.uniform(0, 50, 200000), 2.0 ** rng.uniform(-31, 6, 20000),
+                        [0.0, 1.0, 2.0, 0.25, 2.0 ** -31, 44.3614195558365]])
+    got = I.sqrt_newton(torch.from_numpy(x)).numpy()
+    ref = np.sqrt(x)
+    assert [got[-6], got[-5], got[-3]] == [0.0, 1.0, 0.5]        # exact squares
+    assert np.max(np.abs(got - ref) / np.spacing(np.maximum(ref, 1e-300))) <= 1
+
+
 def test_unit_normal_is_standard_normal():
     v = I.unit_normal(0, 1, 0, 1 << 22).numpy()
     assert abs(v.mean()) < 2e-3 and abs(v.var() - 1.0) < 3e-3
