@@ -20,17 +20,19 @@ constexpr int kUmmaK = 16;                // K per tcgen05.mma (kind::f16)
 constexpr int kWTileBytes = kBM * kBK * 2;
 constexpr int kTableBytes = 2 * 4 * 1025 + 16;     // tiles[E+1], offsets[E+1], E <= 1024
 
-constexpr int kWqRecordBytes = 4608;
+constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
 
 // 64-K slices per pipeline step of the NVFP4 kernel: up to 4 dividing the
 // tile's K, and few enough that TMEM (512 columns) holds a W slot of 32*KS
-// columns per dequant group (two) next to the two accumulators (2*nt columns).
-// The host picks the record TMA box with the same rule.
+// columns per dequant group (two) next to the accumulators (wq_acc_cols: a
+// double-buffered pair, 2*nt columns, or for 16-token tiles one pair per MMA
+// thread, four of them).  The host picks the record TMA box with the same rule.
+__host__ __device__ inline int wq_acc_cols(int nt) { return (nt == 16 ? 8 : 2) * nt; }
 __host__ __device__ inline int wq_slices_per_step(int kt_all, int nt) {
   int ks = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
-  while (ks > 1 && (512 - 2 * nt) / (32 * ks) < 2) ks >>= 1;
+  while (ks > 1 && (512 - wq_acc_cols(nt)) / (32 * ks) < 2) ks >>= 1;
   return ks;
-}      // NVFP4 weight record: 128 x 32 B codes + 128 x 4 B scales
+}
 
 template <int NT, int STAGES>
 struct UmmaSmem {

@@ -5,23 +5,28 @@
 // records and are expanded to exact bf16 rows directly in tensor memory, from
 // where the MMA reads its A operand ("TS" form).
 //
-// A 64-K slice of NVFP4 weights is only 4.6 KB, while the single issuing thread
-// pays ~100 cycles per barrier wait and ~60-100 per commit or MMA on a loaded
-// SM; so a pipeline step is a batch of KS = 4 slices (K = 256, 16 MMAs per
-// wait/commit pair).  The dequantised W tiles live in TMEM (slots of 32*KS
-// columns next to the accumulators), which leaves shared memory for the record
-// batches (covering HBM latency) and the activation tiles.
+// A 64-K slice of NVFP4 weights is only 4.6 KB, and every tcgen05 instruction
+// holds its issuing thread for ~55 cycles (more on a busy SM), so a pipeline
+// step is a batch of KS = 4 slices (K = 256) and each MMA thread pays one wait
+// and one commit per step: the dequant warps wait for the step's activation
+// tile as well as its records, so the MMA threads wait only for "W ready", and
+// one commit per step frees the step's A slot and W slot together.  The
+// dequantised W tiles live in TMEM (slots of 32*KS columns next to the
+// accumulators), which leaves shared memory for the record batches (covering
+// HBM latency) and the activation tiles.
 //
 // Warps (640 threads):
 //   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
 //   2      activation producer (TMA tiles into the A ring)
-//   3      16-token tiles: second MMA issuer (16-K steps 2-3 of every slice into
-//          a second accumulator); otherwise idle
-//   4-7    epilogue group 0 (even 8-column chunks of the accumulator)
+//   3, 16, 18  16-token tiles: further MMA issuers -- four threads, one per SM
+//          sub-partition, thread j issuing the j-th 16-K step of every slice
+//          into its own accumulator pair; otherwise idle
+//   4-7    epilogue group 0 (16-token tiles: every chunk, summing the four
+//          accumulators; otherwise the even 8-column chunks)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
 //          alternate steps; each thread expands its weight row's slices
-//   16-19  epilogue group 1 (odd chunks)
+//   16-19  epilogue group 1 (odd chunks) for 32-token and wider tiles
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
 //
@@ -39,19 +44,20 @@ namespace lmoe {
 
 constexpr int kMaxKS = 4;                    // 64-K slices per pipeline step
 
-template <int NT, int SA, int RAW>
+template <int NT, int RAW>
 struct WqSmem {
+  // 16-token tiles keep four accumulator pairs (four MMA threads)
+  static constexpr int kAccCols = (NT == 16 ? 8 : 2) * NT;
+  static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
+  static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
   static constexpr int kATileBytes = NT * kBK * 2;                     // one 64-K slice, multiple of 1024
-  static constexpr int kASlotBytes = kMaxKS * kATileBytes;             // one step
+  // one A slot per W slot: SW slots of KS tiles fit in kMaxSW tiles
+  static constexpr int kARegionBytes = kMaxSW * kATileBytes;
   static constexpr int kRawSlotBytes = kMaxKS * kWqRecordBytes;        // one step's records
-  static constexpr int kRawOffset = SA * kASlotBytes;
+  static constexpr int kRawOffset = kARegionBytes;
   static constexpr int kBarOffset = kRawOffset + RAW * kRawSlotBytes;
   static constexpr int kTableOffset = kBarOffset + 1024;               // 128 barrier slots
   static constexpr int kBytes = kTableOffset + kTableBytes + 1024;     // + alignment
-  // 16-token tiles keep two accumulator pairs (two MMA threads, section below)
-  static constexpr int kAccCols = (NT == 16 ? 4 : 2) * NT;
-  static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
-  static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
 };
 
 constexpr int kWqThreads = 640;
@@ -64,19 +70,27 @@ __device__ __forceinline__ int dq_group(int warp) {
   return (warp >= 8 && warp < 16) ? (warp - 8) >> 2 : -1;
 }
 
-template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA, bool F16>
+// MMA thread index of a warp (lane 0 issues): warp 1, and for 16-token tiles
+// warps 3, 16, 18 -- one per SM sub-partition (warp % 4); -1 otherwise
+template <bool SPLIT>
+__device__ __forceinline__ int mma_thread(int warp) {
+  if (warp == 1) return 0;
+  if (!SPLIT) return -1;
+  return warp == 3 ? 1 : warp == 16 ? 2 : warp == 18 ? 3 : -1;
+}
+
+template <int NT, int RAW, typename TO, bool RELU2, bool QA, bool F16>
 __global__ void __launch_bounds__(kWqThreads, 1)
 umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wqmap,
                const UmmaArgs a) {
-  using S = WqSmem<NT, SA, RAW>;
+  using S = WqSmem<NT, RAW>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset); // A tile landed
-  uint64_t* a_empty = a_full + SA;                                      // A slot free (MMA done)
-  uint64_t* w_ready = a_empty + SA;                                     // W slot written (TMEM)
-  uint64_t* w_empty = w_ready + S::kMaxSW;                              // W slot free (MMA done)
-  uint64_t* raw_full = w_empty + S::kMaxSW;                             // record batch landed
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset); // A tiles of slot landed
+  uint64_t* w_ready = a_full + S::kMaxSW;                               // W slot written (TMEM)
+  uint64_t* slot_free = w_ready + S::kMaxSW;                            // slot's MMAs done
+  uint64_t* raw_full = slot_free + S::kMaxSW;                           // record batch landed
   uint64_t* raw_empty = raw_full + RAW;                                 // record batch consumed
   uint64_t* acc_full = raw_empty + RAW;                                 // [2]
   uint64_t* acc_empty = acc_full + 2;                                   // [2]
@@ -87,12 +101,13 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 16-token tiles: two threads issue the MMAs (16-K steps 0-1 and 2-3 of every
-  // slice) into two accumulators that the epilogue adds; each tcgen05
-  // instruction holds its issuing thread for tens of cycles, and a 128 x 16 x 16
-  // MMA is far shorter than that
+  // 16-token tiles: four threads issue the MMAs (thread j the j-th 16-K step of
+  // every slice) into four accumulators that the epilogue adds; each tcgen05
+  // instruction holds its issuing thread for ~55 cycles, four times a
+  // 128 x 16 x 16 MMA's time on the tensor pipe
   constexpr bool SPLIT = NT == 16;
-  constexpr uint32_t NM = SPLIT ? 2 : 1;    // MMA threads
+  constexpr uint32_t NM = SPLIT ? 4 : 1;    // MMA threads
+  constexpr int kEpiThreads = SPLIT ? 128 : 256;
   const int kt_all = a.K0 / kBK;
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
   // tile has a multiple of KS slices
@@ -101,10 +116,13 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   const int SW = (512 - S::kWCol0) / (32 * KS);                        // W slots of 32*KS columns
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) { mbar_init(&a_full[s], 1); mbar_init(&a_empty[s], NM); }
-    for (int s = 0; s < SW; ++s) { mbar_init(&w_ready[s], kDqGroupThreads); mbar_init(&w_empty[s], NM); }
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&w_ready[s], kDqGroupThreads);
+      mbar_init(&slot_free[s], NM);
+    }
     for (int r = 0; r < RAW; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], kDqGroupThreads); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], NM); mbar_init(&acc_empty[b], 256); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], NM); mbar_init(&acc_empty[b], kEpiThreads); }
     mbar_init(mma_done, NM);
     *abort_flag = 0;
     fence_mbar_init();
@@ -156,53 +174,54 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     // ---------------- activation producer ----------------
     if (lane == 0) {
       uint32_t it = 0, sa = 0, pa = 1;
+      const int slot_bytes = KS * S::kATileBytes;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
         for (int st = 0; st < nsteps; ++st, ++it) {
-          if (!mbar_wait(&a_empty[sa], pa)) { fail(13); ok = false; break; }
-          mbar_arrive_expect_tx(&a_full[sa], KS * S::kATileBytes);
-          uint8_t* dst = smem + sa * S::kASlotBytes;
+          if (!mbar_wait(&slot_free[sa], pa)) { fail(13); ok = false; break; }
+          mbar_arrive_expect_tx(&a_full[sa], slot_bytes);
+          uint8_t* dst = smem + sa * slot_bytes;
           for (int ks = 0; ks < KS; ++ks)
             tma_load_2d(dst + ks * S::kATileBytes, &amap, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
-          if (++sa == SA) { sa = 0; pa ^= 1; }
+          if (++sa == (uint32_t)SW) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
       }
-      const uint32_t n = it < (uint32_t)SA ? it : (uint32_t)SA;
+      const uint32_t n = it < (uint32_t)SW ? it : (uint32_t)SW;
       for (uint32_t j = 0; j < n; ++j) {
         const uint32_t i = it - 1 - j;
-        if (!mbar_wait(&a_full[i % SA], (i / SA) & 1)) { fail(14); break; }
+        if (!mbar_wait(&a_full[i % SW], (i / SW) & 1)) { fail(14); break; }
       }
     }
-  } else if (warp == 1 || (SPLIT && warp == 3)) {
+  } else if (mma_thread<SPLIT>(warp) >= 0) {
     // ---------------- MMA issuer(s) (A from TMEM, B from shared memory) ----------------
-    const int half = warp == 3;               // SPLIT: 16-K steps 2 half .. 2 half + 1
+    const int j = mma_thread<SPLIT>(warp);    // SPLIT: the j-th 16-K step of every slice
     if (lane == 0) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
-      uint32_t sa = 0, pa = 0, sw = 0, pw = 0, lt = 0;
+      const uint32_t slot_desc = (uint32_t)((KS * S::kATileBytes) >> 4);
+      uint32_t s = 0, ps = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         const uint32_t buf = lt & 1, use = lt >> 1;
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(15); break; }
         tc_fence_after();
-        const uint32_t d = tmem + (2 * half + buf) * NT;
+        const uint32_t d = tmem + (2 * j + buf) * NT;
         // ragged tiles multiply only their valid rows, rounded up to N granularity 16
         const int n_eff = min(NT, (ti.valid + 15) & ~15);
         const uint32_t idesc = F16 ? idesc_f16_f32(kBM, n_eff) : idesc_bf16_f32(kBM, n_eff);
         bool ok = true;
         for (int st = 0; st < nsteps; ++st) {
-          if (!mbar_wait(&a_full[sa], pa) || !mbar_wait(&w_ready[sw], pw)) { fail(16); ok = false; break; }
+          // W ready implies the step's A tiles landed (the dequant warps waited for them)
+          if (!mbar_wait(&w_ready[s], ps)) { fail(16); ok = false; break; }
           tc_fence_after();
-          uint32_t wt = tmem + S::kWCol0 + sw * 32 * KS;
-          uint64_t bd = bdesc0 + (uint64_t)(sa * (S::kASlotBytes >> 4));
+          uint32_t wt = tmem + S::kWCol0 + s * 32 * KS;
+          uint64_t bd = bdesc0 + (uint64_t)(s * slot_desc);
           for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
             if (SPLIT) {
-              const int j = 2 * half;
               mma_bf16_ts(d, wt + 8 * j, bd + 2 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
-              mma_bf16_ts(d, wt + 8 * j + 8, bd + 2 * j + 2, idesc, 1u);
             } else {
               mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
               mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
@@ -210,10 +229,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
               mma_bf16_ts(d, wt + 24, bd + 6, idesc, 1u);
             }
           }
-          mma_commit(&a_empty[sa]);          // both slots free once these MMAs finish
-          mma_commit(&w_empty[sw]);
-          if (++sa == SA) { sa = 0; pa ^= 1; }
-          if (++sw == SW) { sw = 0; pw ^= 1; }
+          mma_commit(&slot_free[s]);          // A and W slot free once these MMAs finish
+          if (++s == (uint32_t)SW) { s = 0; ps ^= 1; }
         }
         if (!ok) break;
         mma_commit(&acc_full[buf]);
@@ -235,8 +252,10 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       for (int st = 0; st < nsteps; ++st, ++it) {
         if ((int)(it % kDqGroups) != g) continue;
         const int sw = it % SW, rr = it % RAW;
+        const uint32_t ph = (it / SW) & 1;
         if (!mbar_wait_sleep(&raw_full[rr], (it / RAW) & 1) ||
-            !mbar_wait_sleep(&w_empty[sw], ((it / SW) & 1) ^ 1)) { fail(18); ok = false; break; }
+            !mbar_wait_sleep(&slot_free[sw], ph ^ 1) ||
+            !mbar_wait_sleep(&a_full[sw], ph)) { fail(18); ok = false; break; }
         tc_fence_after();
         const uint8_t* rec = smem + S::kRawOffset + rr * S::kRawSlotBytes;
         for (int ks = 0; ks < KS; ++ks) {
@@ -252,10 +271,12 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       }
       if (!ok) break;
     }
-  } else if ((warp >= 4 && warp < 8) || (warp >= 16 && warp < 20)) {
-    // ---------------- epilogue (two groups split the accumulator's chunks) ----------------
+  } else if ((warp >= 4 && warp < 8) || (!SPLIT && warp >= 16 && warp < 20)) {
+    // ---------------- epilogue (two groups split the accumulator's chunks;
+    // 16-token tiles: group 0 alone) ----------------
     const int q = warp & 3;
     const int grp = warp >= 16 ? 1 : 0;
+    constexpr int kChunkStep = SPLIT ? 1 : 2;
     TO* out = reinterpret_cast<TO*>(a.out);
     uint32_t lt = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
@@ -268,17 +289,26 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       const bool col_ok = n < a.n_out;
       // gscale holds s_g * 2^26 (the bf16 expansion carries 2^-26); exact rescale for fp16
       const float gs = a.gscale ? (F16 ? a.gscale[ti.grp] * 0x1p-26f : a.gscale[ti.grp]) : 1.f;
-      for (int c = grp; c < NT / 8; c += 2) {
+      for (int c = grp; c < NT / 8; c += kChunkStep) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
-        uint32_t rg[8], rh[8];
-        tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * NT + c * 8, rg);
-        if (SPLIT) tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + (2 + buf) * NT + c * 8, rh);
+        const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;
+        uint32_t r0[8], r1[8], r2[8], r3[8];
+        tmem_ld8(row_base + buf * NT, r0);
+        if (SPLIT) {
+          tmem_ld8(row_base + (2 + buf) * NT, r1);
+          tmem_ld8(row_base + (4 + buf) * NT, r2);
+          tmem_ld8(row_base + (6 + buf) * NT, r3);
+        }
         tmem_ld_wait();
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float acc = SPLIT ? __fadd_rn(__uint_as_float(rg[j]), __uint_as_float(rh[j]))
-                                  : __uint_as_float(rg[j]);
+          // the four partial sums (16-K steps 0..3 of every slice), added in order
+          const float acc =
+              SPLIT ? __fadd_rn(__fadd_rn(__fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j])),
+                                          __uint_as_float(r2[j])),
+                                __uint_as_float(r3[j]))
+                    : __uint_as_float(r0[j]);
           v[j] = __fmul_rn(acc, gs);
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
@@ -315,18 +345,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   }
 }
 
-template <int NT, int SA, int RAW, typename TO, bool RELU2, bool QA, bool F16>
+template <int NT, int RAW, typename TO, bool RELU2, bool QA, bool F16>
 static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
-  using S = WqSmem<NT, SA, RAW>;
+  using S = WqSmem<NT, RAW>;
   static_assert(S::kBytes <= 232448, "shared memory budget");
   // dequant groups work on up to kDqGroups steps at once: each ring needs at
-  // least that many slots, or a waiter could target a phase two ahead (parity alias)
-  // dequant groups work on up to kDqGroups steps at once: each ring needs at
-  // least that many slots, or a waiter could target a phase two ahead (parity alias)
-  static_assert((512 - S::kWCol0) / 32 >= kDqGroups && RAW >= kDqGroups && SA >= 2,
-                "ring too shallow for the dequant groups");
-  static_assert(2 * SA + 2 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
-  auto kern = umma_wq_kernel<NT, SA, RAW, TO, RELU2, QA, F16>;
+  // least that many slots, or a waiter could target a phase two ahead (parity
+  // alias); wq_slices_per_step keeps at least two W slots
+  static_assert(S::kMaxSW >= kDqGroups && RAW >= kDqGroups, "ring too shallow for the dequant groups");
+  static_assert(3 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
+  auto kern = umma_wq_kernel<NT, RAW, TO, RELU2, QA, F16>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -342,19 +370,19 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int NT, int SA, int RAW>
+template <int NT, int RAW>
 static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
   if (L.a_f16) {                         // W4A4: fp16 operands, natural record order
     switch (L.epi) {
-      case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, SA, RAW, __half, true, true, true>(L, st);
-      case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false, true>(L, st);
+      case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, RAW, __half, true, true, true>(L, st);
+      case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false, true>(L, st);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (L.epi) {
-    case UMMA_EPI_BF16: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, false, false, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, SA, RAW, __nv_bfloat16, true, false, false>(L, st);
-    case UMMA_EPI_F32: return wq_launch_t<NT, SA, RAW, float, false, false, false>(L, st);
+    case UMMA_EPI_BF16: return wq_launch_t<NT, RAW, __nv_bfloat16, false, false, false>(L, st);
+    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, RAW, __nv_bfloat16, true, false, false>(L, st);
+    case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false, false>(L, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -362,9 +390,9 @@ static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st) {
   if (L.args.K1 != 0 || !L.args.wq) return cudaErrorInvalidValue;
   switch (L.nt) {
-    case 16: return wq_launch_nt<16, 6, 8>(L, st);          // A 48 KB + records 147 KB
-    case 64: return wq_launch_nt<64, 3, 6>(L, st);          // A 96 KB + records 110 KB
-    case 128: return wq_launch_nt<128, 2, 4>(L, st);        // A 128 KB + records 74 KB
+    case 16: return wq_launch_nt<16, 9>(L, st);             // A 24 KB + records 166 KB
+    case 64: return wq_launch_nt<64, 6>(L, st);             // A 96 KB + records 110 KB
+    case 128: return wq_launch_nt<128, 4>(L, st);           // A 128 KB + records 74 KB
   }
   return cudaErrorInvalidValue;
 }
