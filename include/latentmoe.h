@@ -143,6 +143,47 @@ typedef struct moe_handle moe_handle;
 moe_status moe_init(moe_handle** handle, const moe_config* cfg,
                     const moe_weights* weights, void* stream);
 
+/* Expert parallelism across n_ranks layers (one per GPU), written from the
+ * pages' LatentMoE remark: tokens reach their experts through the d_latent-wide
+ * latent, a quarter of d_model at the Ultra shape, so an expert-parallel layer
+ * needs to exchange only latent rows.
+ *   moe_init_ep      rank `rank` of `n_ranks` holds routed experts
+ *                    [rank*E/n_ranks, (rank+1)*E/n_ranks): the weights' expert
+ *                    tensors (w_up / w_down, or the pre-quantised NVFP4 set)
+ *                    cover those E/n_ranks experts only; everything else (gate,
+ *                    bias, fc1, fc2, shared expert) is the whole layer's.
+ *                    E % n_ranks != 0 or rank outside [0, n_ranks):
+ *                    MOE_ERR_INVALID_ARG; n_ranks > 1 needs dtype MOE_BF16
+ *                    (MOE_ERR_UNSUPPORTED otherwise).  moe_init is
+ *                    moe_init_ep(.., 0, 1, ..).  An expert-parallel handle
+ *                    (n_ranks > 1) rejects moe_forward / moe_forward_host /
+ *                    moe_block_forward with MOE_ERR_UNSUPPORTED.
+ *   moe_forward_ep_partial
+ *                    steps 1-6 on every rank for all T tokens: the router over
+ *                    all E experts (the same bits on every rank), fc1 and the
+ *                    shared expert's up projection, then the routed experts
+ *                    this rank holds, combined in slot order into
+ *                    zc_part[t] = sum of w[t,j] * y[t,j] over the slots j whose
+ *                    expert is held here   (fp32 [T, d_latent], device; rows of
+ *                    tokens with no held expert are zero).
+ *   (the caller gathers every rank's zc_part into parts [n_ranks, T, d_latent]
+ *    fp32, rank r's rows at parts + r*T*d_latent -- one all-gather)
+ *   moe_forward_ep_finish
+ *                    step 7 for the token shard [t0, t0 + Ts): zc = the parts
+ *                    summed in rank order (fp32, rank 0 first), rounded to the
+ *                    layer dtype, out[0..Ts) = zc W_fc2^T + the shared expert
+ *                    of those rows (activations kept from the partial call on
+ *                    this handle, which must be the last forward with the same
+ *                    T).  out [Ts, d_model] out_dtype, device.
+ * The result equals moe_forward's up to the order of the fp32 combine sums
+ * (slot order within a rank, then rank order); routing is identical. */
+moe_status moe_init_ep(moe_handle** handle, const moe_config* cfg, const moe_weights* weights,
+                       int rank, int n_ranks, void* stream);
+moe_status moe_forward_ep_partial(moe_handle* handle, const void* hidden, int T, float* zc_part,
+                                  int32_t* topk_idx, float* topk_w, void* stream);
+moe_status moe_forward_ep_finish(moe_handle* handle, const float* parts, int n_parts, int T,
+                                 int t0, int Ts, void* out, void* stream);
+
 /* One layer forward on T token rows (report section 5.6).
  *   hidden   [T, D] dtype, device, row-major, 16-byte aligned
  *   out      [T, D] out_dtype, device

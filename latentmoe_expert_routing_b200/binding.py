@@ -55,6 +55,9 @@ _vp, _i, _p = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER
 # (name, restype, argtypes) of every entry point declared in include/latentmoe.h
 SIGNATURES = [
     ("moe_init", _i, [_p(_vp), _p(moe_config), _p(moe_weights), _vp]),
+    ("moe_init_ep", _i, [_p(_vp), _p(moe_config), _p(moe_weights), _i, _i, _vp]),
+    ("moe_forward_ep_partial", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
+    ("moe_forward_ep_finish", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp]),
     ("moe_forward", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     ("moe_forward_host", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     ("moe_block_forward", _i, [_vp, _vp, _i, _vp, ctypes.c_float, _vp, _vp, _vp, _vp]),
@@ -107,6 +110,23 @@ def moe_init(cfg: moe_config, w: moe_weights, stream: int):
     _check(_lib.moe_init(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(w),
                          stream), "moe_init")
     return h
+
+
+def moe_init_ep(cfg: moe_config, w: moe_weights, rank: int, n_ranks: int, stream: int):
+    h = ctypes.c_void_p()
+    _check(_lib.moe_init_ep(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(w), rank, n_ranks,
+                            stream), "moe_init_ep")
+    return h
+
+
+def moe_forward_ep_partial(h, hidden_ptr, T, zc_part_ptr, topk_idx_ptr, topk_w_ptr, stream):
+    _check(_lib.moe_forward_ep_partial(h, hidden_ptr, T, zc_part_ptr, topk_idx_ptr, topk_w_ptr,
+                                       stream), "moe_forward_ep_partial")
+
+
+def moe_forward_ep_finish(h, parts_ptr, n_parts, T, t0, Ts, out_ptr, stream):
+    _check(_lib.moe_forward_ep_finish(h, parts_ptr, n_parts, T, t0, Ts, out_ptr, stream),
+           "moe_forward_ep_finish")
 
 
 def moe_forward(h, hidden_ptr, T, out_ptr, topk_idx_ptr, topk_w_ptr, stream):

@@ -15,6 +15,8 @@ using namespace lmoe;
 struct moe_handle {
   moe_config cfg;
   int device = 0;
+  // expert parallelism: this layer holds experts [e0, e0 + e_loc) of n_experts
+  int e0 = 0, e_loc = 0, ep_rank = 0, ep_ranks = 1;
   std::vector<void*> owned;          // device allocations to free
   // weights (borrowed or owned)
   const void *w_gate = nullptr, *w_fc1 = nullptr, *w_fc2 = nullptr;
@@ -216,7 +218,7 @@ struct TempBuf {
 
 moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s) {
   const moe_config& c = h->cfg;
-  const size_t E = c.n_experts, F = c.d_ff, L = c.d_latent;
+  const size_t E = h->e_loc, F = c.d_ff, L = c.d_latent;     // the experts this layer holds
   const size_t recs_up = E * ((F + 127) / 128) * (L / 64), recs_dn = E * ((L + 127) / 128) * (F / 64);
   if (!dev_alloc(h, &h->rec_up, recs_up * 4608) || !dev_alloc(h, &h->rec_dn, recs_dn * 4608) ||
       !dev_alloc(h, &h->gs_up, E * 4) || !dev_alloc(h, &h->gs_dn, E * 4))
@@ -318,10 +320,32 @@ bool use_mxf4_pair(const moe_config& c, long P) {
 // Tensor-core path for bf16 layers: G1 (fc1, shared up), row gather, grouped
 // up / down, combine, G5 (fc2 + shared down) -- all tcgen05 GEMMs but the gather
 // and the combine.
+// G5 on M token rows: out = zc W_fc2^T + h_sh W_sd^T, one accumulator over
+// K = L + Fs; zc / h_sh come through their maps (and 128-row half maps for SM pairs).
+moe_status launch_g5(moe_handle* h, int M, const CUtensorMap& zc_map, const CUtensorMap& zc_half,
+                     const CUtensorMap& hsh_map, const CUtensorMap& hsh_half, void* out,
+                     cudaStream_t s) {
+  const moe_config& c = h->cfg;
+  const int di = nt_index(M);
+  UmmaLaunch g{};
+  g.args.err = h->err;
+  g.args.E = 1;
+  g.args.M = M;
+  g.nt = kNT[di];
+  g.wmap0 = h->wm_fc2; g.amap0 = zc_map;
+  g.wmap1 = h->wm_sd; g.amap1 = hsh_map;
+  g.args.K0 = c.d_latent; g.args.K1 = c.d_ff_shared; g.args.n_out = c.d_model;
+  g.args.ldo = c.d_model;
+  g.args.dense_tiles = ceil_div(c.d_model, 128) * ceil_div(M, g.nt);
+  g.args.out = out; g.epi = c.out_dtype == MOE_BF16 ? UMMA_EPI_BF16 : UMMA_EPI_F32;
+  g.max_tiles = g.args.dense_tiles;
+  return launch_dense_umma(h, g, s, &zc_half, &hsh_half);
+}
+
 template <typename Mark>
 moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMap* xhalf, int T,
-                        void* out,
-                        const float* wts, Mark& mark, cudaStream_t s) {
+                        void* out, const int32_t* idx,
+                        const float* wts, Mark& mark, cudaStream_t s, float* zc_part) {
   const moe_config& c = h->cfg;
   const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
   const int F = c.d_ff, Fs = c.d_ff_shared;
@@ -372,7 +396,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     }
     UmmaLaunch u{};
     u.args.err = h->err;
-    u.args.E = E; u.args.offsets = h->offsets; u.nt = ntg;
+    u.args.E = E; u.args.offsets = h->offsets; u.nt = ntg; u.args.grp0 = h->e0;
     u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
     u.args.tiles = h->tiles_up; u.args.out = h->hq; u.args.gscale = h->gs_up;
     u.epi = UMMA_EPI_F16_RELU2_Q;
@@ -387,6 +411,10 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     e = mp ? launch_umma_mxf4_pair(u, h->mxp_dn, nullptr, s) : launch_umma_mxf4(u, h->mx_dn, nullptr, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     mark(MOE_STAGE_COMBINE);
+    if (zc_part) {
+      launch_combine_part(h->Y, wts, h->pos, idx, h->e0, h->e0 + h->e_loc, zc_part, T, k, L, s);
+      return MOE_OK;
+    }
     launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
     mark(MOE_STAGE_DENSE_OUT);
   } else {
@@ -396,7 +424,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   UmmaLaunch u{};
   u.a_f16 = w4a4;
   u.args.err = h->err;
-  u.args.E = E; u.args.offsets = h->offsets;
+  u.args.E = E; u.args.offsets = h->offsets; u.args.grp0 = h->e0;
   u.nt = ntg;
   u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
@@ -425,19 +453,16 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
   if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_COMBINE);
+  if (zc_part) {
+    launch_combine_part(h->Y, wts, h->pos, idx, h->e0, h->e0 + h->e_loc, zc_part, T, k, L, s);
+    return MOE_OK;
+  }
   launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
   mark(MOE_STAGE_DENSE_OUT);
   }
 
   // step 7: out = zc W_fc2^T + h_sh W_sd^T, one accumulator over K = L + Fs
-  g.wmap0 = h->wm_fc2; g.amap0 = h->am_zc[di];
-  g.wmap1 = h->wm_sd; g.amap1 = h->am_hsh[di];
-  g.args.K0 = L; g.args.K1 = Fs; g.args.n_out = D; g.args.ldo = D;
-  g.args.dense_tiles = ceil_div(D, 128) * ceil_div(T, ntd);
-  g.args.out = out; g.epi = c.out_dtype == MOE_BF16 ? UMMA_EPI_BF16 : UMMA_EPI_F32;
-  g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s, &h->am_zc[3], &h->am_hsh[3])) != MOE_OK) return st;
-  return MOE_OK;
+  return launch_g5(h, T, h->am_zc[di], h->am_zc[3], h->am_hsh[di], h->am_hsh[3], out, s);
 }
 
 }  // namespace
@@ -475,10 +500,18 @@ void moe_destroy(moe_handle* h) {
 
 moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* w,
                     void* stream) {
+  return moe_init_ep(out, cfg, w, 0, 1, stream);
+}
+
+moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weights* w, int rank,
+                       int n_ranks, void* stream) {
   if (!out || !w) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
+  if (n_ranks < 1 || rank < 0 || rank >= n_ranks || cfg->n_experts % n_ranks)
+    return MOE_ERR_INVALID_ARG;
+  if (n_ranks > 1 && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   const void* ptrs[] = {w->w_gate, w->gate_bias, w->w_fc1, w->w_fc2, w->w_shared_up,
                         w->w_shared_down};
   for (const void* p : ptrs)
@@ -512,9 +545,14 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
   moe_handle* h = new (std::nothrow) moe_handle();
   if (!h) return MOE_ERR_OOM;
   h->cfg = *cfg;
+  h->ep_rank = rank;
+  h->ep_ranks = n_ranks;
+  h->e_loc = cfg->n_experts / n_ranks;
+  h->e0 = rank * h->e_loc;
   cudaGetDevice(&h->device);
   const moe_config& c = h->cfg;
   const size_t D = c.d_model, L = c.d_latent, E = c.n_experts, F = c.d_ff, Fs = c.d_ff_shared;
+  const size_t El = h->e_loc;                     // routed experts held by this layer
   const size_t T = c.max_tokens, k = c.top_k, P = T * k, nblk = (T + 31) / 32;
   const size_t ds = dt_size(c.dtype);
   cudaStream_t s = (cudaStream_t)stream;
@@ -530,7 +568,7 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
         {w->w_gate, &h->w_gate, E * D * ds},    {w->w_fc1, &h->w_fc1, L * D * ds},
         {w->w_fc2, &h->w_fc2, D * L * ds},      {w->w_shared_up, &h->w_su, Fs * D * ds},
         {w->w_shared_down, &h->w_sd, D * Fs * ds}, {w->gate_bias, (const void**)&h->bias, E * 4},
-        {w->w_up, &h->w_up, E * F * L * ds},    {w->w_down, &h->w_down, E * L * F * ds}};
+        {w->w_up, &h->w_up, El * F * L * ds},   {w->w_down, &h->w_down, El * L * F * ds}};
     for (auto& q : cp) {
       if (!dense_experts && (q.dst == &h->w_up || q.dst == &h->w_down)) continue;
       void* d = nullptr;
@@ -574,8 +612,8 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
     bool m = make_tmap_bf16(&h->wm_gate, h->w_gate, E, D, 128) &&
              make_tmap_bf16(&h->wm_fc1, h->w_fc1, L, D, 128) &&
              make_tmap_bf16(&h->wm_su, h->w_su, Fs, D, 128) &&
-             (!dense_experts || (make_tmap_bf16(&h->wm_up, h->w_up, E * F, L, 128) &&
-                                 make_tmap_bf16(&h->wm_dn, h->w_down, E * L, F, 128))) &&
+             (!dense_experts || (make_tmap_bf16(&h->wm_up, h->w_up, El * F, L, 128) &&
+                                 make_tmap_bf16(&h->wm_dn, h->w_down, El * L, F, 128))) &&
              make_tmap_bf16(&h->wm_fc2, h->w_fc2, D, L, 128) &&
              make_tmap_bf16(&h->wm_sd, h->w_sd, D, Fs, 128);
     for (int i = 0; i < 4 && m; ++i)
@@ -631,13 +669,16 @@ moe_status moe_init(moe_handle** out, const moe_config* cfg, const moe_weights* 
   return MOE_OK;
 }
 
-moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
-                       int32_t* topk_idx, float* topk_w, void* stream) {
+// One forward; with zc_part (expert parallelism) it stops after the routed
+// experts and writes this layer's partial latent combine instead of `out`.
+static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* out,
+                               int32_t* topk_idx, float* topk_w, void* stream, float* zc_part) {
   if (!h) return MOE_ERR_INVALID_ARG;
   const moe_config& c = h->cfg;
   if (T < 0 || T > c.max_tokens) return MOE_ERR_INVALID_ARG;
   if (T == 0) { h->last_T = 0; return MOE_OK; }
-  if (!hidden || !out || !aligned16(hidden) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (!hidden || !aligned16(hidden)) return MOE_ERR_INVALID_ARG;
+  if (zc_part ? !aligned16(zc_part) : (!out || !aligned16(out))) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
   const int F = c.d_ff, Fs = c.d_ff_shared;
@@ -686,6 +727,7 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   ra.tiles_up = h->tiles_up; ra.tiles_dn = h->tiles_dn;
   ra.err = h->err;
   ra.n_group = c.n_group; ra.topk_group = c.topk_group;
+  ra.e_lo = h->e0; ra.e_hi = h->e0 + h->e_loc;
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
                 h->stats, h->wstat};
@@ -696,7 +738,8 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
   mark(MOE_STAGE_DENSE_IN);
 
   if (dt == MOE_BF16) {
-    moe_status us = forward_umma(h, xmap, wide ? &xhalf : nullptr, T, out, wts, mark, s);
+    moe_status us = forward_umma(h, xmap, wide ? &xhalf : nullptr, T, out, idx, wts, mark, s,
+                                 zc_part);
     if (us != MOE_OK) return us;
   } else {
     // step 5 and the shared expert's up projection: both read x
@@ -734,8 +777,43 @@ moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
     launch_dense(g5, s);
   }
   mark(MOE_NUM_STAGES);
-  h->prof_valid = h->prof;
+  h->prof_valid = h->prof && !zc_part;
   h->last_T = T;
+  return cuda_status(cudaGetLastError());
+}
+
+moe_status moe_forward(moe_handle* h, const void* hidden, int T, void* out,
+                       int32_t* topk_idx, float* topk_w, void* stream) {
+  if (h && h->ep_ranks > 1) return MOE_ERR_UNSUPPORTED;     // holds only some experts
+  return forward_impl(h, hidden, T, out, topk_idx, topk_w, stream, nullptr);
+}
+
+moe_status moe_forward_ep_partial(moe_handle* h, const void* hidden, int T, float* zc_part,
+                                  int32_t* topk_idx, float* topk_w, void* stream) {
+  if (!h || !zc_part) return MOE_ERR_INVALID_ARG;
+  return forward_impl(h, hidden, T, nullptr, topk_idx, topk_w, stream, zc_part);
+}
+
+moe_status moe_forward_ep_finish(moe_handle* h, const float* parts, int n_parts, int T, int t0,
+                                 int Ts, void* out, void* stream) {
+  if (!h || !parts || !aligned16(parts)) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (n_parts != h->ep_ranks || T != h->last_T || t0 < 0 || Ts < 0 || t0 + Ts > T)
+    return MOE_ERR_INVALID_ARG;
+  if (Ts == 0) return MOE_OK;
+  if (!out || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int L = c.d_latent, Fs = c.d_ff_shared;
+  // zc rows 0..Ts: the ranks' partial latents summed in rank order
+  launch_latent_reduce(parts, n_parts, (long)T * L, t0, Ts, L, h->zc, MOE_BF16, s);
+  // the shared expert's activations of rows t0..t0+Ts, from the partial forward
+  const __nv_bfloat16* hsh = static_cast<const __nv_bfloat16*>(h->h_sh) + (size_t)t0 * Fs;
+  CUtensorMap hmap, hhalf;
+  if (!make_tmap_bf16(&hmap, hsh, Ts, Fs, kNT[nt_index(Ts)]) ||
+      !make_tmap_bf16(&hhalf, hsh, Ts, Fs, 128))
+    return MOE_ERR_CUDA;
+  const moe_status st = launch_g5(h, Ts, h->am_zc[nt_index(Ts)], h->am_zc[3], hmap, hhalf, out, s);
+  if (st != MOE_OK) return st;
   return cuda_status(cudaGetLastError());
 }
 

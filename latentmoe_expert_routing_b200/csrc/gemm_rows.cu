@@ -223,6 +223,72 @@ __global__ void combine_kernel(const float* __restrict__ Y, const float* __restr
   store_val(o, acc.x); store_val(o + 1, acc.y); store_val(o + 2, acc.z); store_val(o + 3, acc.w);
 }
 
+// Expert-parallel partial combine: only the slots whose expert this layer holds
+// (e_lo <= idx < e_hi) contribute, in slot order, fp32 output.
+__global__ void combine_part_kernel(const float* __restrict__ Y, const float* __restrict__ w,
+                                    const int32_t* __restrict__ pos,
+                                    const int32_t* __restrict__ idx, int e_lo, int e_hi,
+                                    float* __restrict__ zc, int T, int k, int L) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_tok = L / 4;
+  if (i >= (long)T * per_tok) return;
+  const int t = (int)(i / per_tok), c = (int)(i - (long)t * per_tok) * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int e = idx[(size_t)t * k + j];
+    if (e < e_lo || e >= e_hi) continue;
+    const float wj = w[(size_t)t * k + j];
+    const float4 y = *reinterpret_cast<const float4*>(Y + (size_t)pos[(size_t)t * k + j] * L + c);
+    acc.x = fmaf(wj, y.x, acc.x);
+    acc.y = fmaf(wj, y.y, acc.y);
+    acc.z = fmaf(wj, y.z, acc.z);
+    acc.w = fmaf(wj, y.w, acc.w);
+  }
+  *reinterpret_cast<float4*>(zc + (size_t)t * L + c) = acc;
+}
+
+void launch_combine_part(const float* Y, const float* topk_w, const int32_t* pos,
+                         const int32_t* idx, int e_lo, int e_hi, float* zc, int T, int k, int L,
+                         cudaStream_t st) {
+  const long n = (long)T * (L / 4);
+  if (n == 0) return;
+  combine_part_kernel<<<ceil_div(n, 256), 256, 0, st>>>(Y, topk_w, pos, idx, e_lo, e_hi, zc, T, k, L);
+}
+
+// The exchanged partial latents summed in rank order: zc[t] = sum_g parts[g][t0 + t]
+// (fp32 adds, g ascending), rounded to the layer dtype.
+template <typename TO>
+__global__ void latent_reduce_kernel(const float* __restrict__ parts, int n_parts, long part_stride,
+                                     int t0, int Ts, int L, TO* __restrict__ zc) {
+  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_tok = L / 4;
+  if (i >= (long)Ts * per_tok) return;
+  const int t = (int)(i / per_tok), c = (int)(i - (long)t * per_tok) * 4;
+  const float* src = parts + (size_t)(t0 + t) * L + c;
+  float4 acc = *reinterpret_cast<const float4*>(src);
+  for (int g = 1; g < n_parts; ++g) {
+    const float4 v = *reinterpret_cast<const float4*>(src + g * part_stride);
+    acc.x = __fadd_rn(acc.x, v.x);
+    acc.y = __fadd_rn(acc.y, v.y);
+    acc.z = __fadd_rn(acc.z, v.z);
+    acc.w = __fadd_rn(acc.w, v.w);
+  }
+  TO* o = zc + (size_t)t * L + c;
+  store_val(o, acc.x); store_val(o + 1, acc.y); store_val(o + 2, acc.z); store_val(o + 3, acc.w);
+}
+
+void launch_latent_reduce(const float* parts, int n_parts, long part_stride, int t0, int Ts, int L,
+                          void* zc, moe_dtype out_dt, cudaStream_t st) {
+  const long n = (long)Ts * (L / 4);
+  if (n == 0) return;
+  if (out_dt == MOE_BF16)
+    latent_reduce_kernel<__nv_bfloat16><<<ceil_div(n, 256), 256, 0, st>>>(
+        parts, n_parts, part_stride, t0, Ts, L, (__nv_bfloat16*)zc);
+  else
+    latent_reduce_kernel<float><<<ceil_div(n, 256), 256, 0, st>>>(parts, n_parts, part_stride, t0,
+                                                                   Ts, L, (float*)zc);
+}
+
 void launch_combine(const float* Y, const float* topk_w, const int32_t* pos, void* zc,
                     int T, int k, int L, moe_dtype out_dt, cudaStream_t st) {
   const long n = (long)T * (L / 4);

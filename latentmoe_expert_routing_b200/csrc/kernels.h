@@ -30,6 +30,8 @@ struct RouteArgs {
   int32_t* tiles_dn;    // [E + 1]
   int* err;
   int n_group, topk_group;   // group routing (section 5.5); n_group <= 1: all experts compete
+  int e_lo, e_hi;            // experts held (expert parallelism): tiles only for
+                             // e_lo <= e < e_hi; e_hi <= 0: all experts
 };
 
 void launch_router_logits(const void* x, const void* wg, float* logits, int T,
@@ -82,6 +84,11 @@ struct GroupedArgs {
 void launch_grouped(const GroupedArgs& a, int max_tiles, cudaStream_t st);
 
 // zc[t, :] = sum_j w[t, j] * Y[pos[t, j], :], fixed slot order, fp32 math.
+void launch_combine_part(const float* Y, const float* topk_w, const int32_t* pos,
+                         const int32_t* idx, int e_lo, int e_hi, float* zc, int T, int k, int L,
+                         cudaStream_t st);
+void launch_latent_reduce(const float* parts, int n_parts, long part_stride, int t0, int Ts, int L,
+                          void* zc, moe_dtype out_dt, cudaStream_t st);
 void launch_combine(const float* Y, const float* topk_w, const int32_t* pos,
                     void* zc, int T, int k, int L, moe_dtype out_dt, cudaStream_t st);
 
@@ -110,6 +117,8 @@ struct UmmaArgs {
   int n_out;                // output columns = weight rows per group
   int ldo;                  // output row stride (elements)
   int w_group_rows;         // row offset between groups in the weight maps
+  int grp0;                 // group held first in the weights (expert parallelism:
+                            // weights, records and gscale cover groups grp0..)
   int E;                    // groups (grouped mode)
   const int32_t* offsets;   // [E+1] A-row offsets (grouped) or NULL (dense)
   const int32_t* tiles;     // [E+1] tile offsets (grouped)
@@ -119,7 +128,7 @@ struct UmmaArgs {
   int* err;
   const uint8_t* wq;        // NVFP4 weight records (GEMM layout) or NULL: weights via wmap0
   int wq_mblks;             // 128-row blocks per weight matrix (NVFP4)
-  const float* gscale;      // [E] per-group output scale (NVFP4 global scale) or NULL
+  const float* gscale;      // [held groups] per-group output scale (NVFP4 global scale) or NULL
   int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
                             // fp32 partials out[slice][row][n] (slice stride below)
   long split_stride;        // elements between slices of the partial output

@@ -279,7 +279,7 @@ route_scan_kernel(const int32_t* __restrict__ blkcnt, int nblk, int E,
                   int32_t* __restrict__ blkpre, int32_t* __restrict__ counts,
                   int32_t* __restrict__ offsets, int mt_up, int nc_up,
                   int32_t* __restrict__ tiles_up, int mt_dn, int nc_dn,
-                  int32_t* __restrict__ tiles_dn) {
+                  int32_t* __restrict__ tiles_dn, int e_lo, int e_hi) {
   __shared__ int tot[1024];
   __shared__ int wt[33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -301,11 +301,13 @@ route_scan_kernel(const int32_t* __restrict__ blkcnt, int nblk, int E,
   const int off = block_excl_scan(c, wt, &all);
   if (e < E) { counts[e] = c; offsets[e] = off; }
   if (e == 0) offsets[E] = all;
-  const int tu = e < E ? (c + mt_up - 1) / mt_up * nc_up : 0;
+  // the grouped GEMMs run tiles only for the experts this layer holds
+  const bool held = e < E && e >= e_lo && (e_hi <= 0 || e < e_hi);
+  const int tu = held ? (c + mt_up - 1) / mt_up * nc_up : 0;
   const int ou = block_excl_scan(tu, wt, &all);
   if (e < E) tiles_up[e] = ou;
   if (e == 0) tiles_up[E] = all;
-  const int td = e < E ? (c + mt_dn - 1) / mt_dn * nc_dn : 0;
+  const int td = held ? (c + mt_dn - 1) / mt_dn * nc_dn : 0;
   const int od = block_excl_scan(td, wt, &all);
   if (e < E) tiles_dn[e] = od;
   if (e == 0) tiles_dn[E] = all;
@@ -370,7 +372,7 @@ void launch_route(const RouteArgs& a, cudaStream_t st) {
   else route_launch_epl<32>(a, st);
   route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
                                         a.offsets, a.mt_up, a.nc_up, a.tiles_up,
-                                        a.mt_dn, a.nc_dn, a.tiles_dn);
+                                        a.mt_dn, a.nc_dn, a.tiles_dn, a.e_lo, a.e_hi);
   const long P = (long)a.T * a.k;
   route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
       a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.E, a.perm, a.pos);
@@ -740,7 +742,7 @@ void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st) 
   route_ranks_kernel<<<a.nblk, 1024, a.E * sizeof(uint32_t), st>>>(a);
   route_scan_kernel<<<1, 1024, 0, st>>>(a.blkcnt, a.nblk, a.E, a.blkpre, a.counts,
                                         a.offsets, a.mt_up, a.nc_up, a.tiles_up,
-                                        a.mt_dn, a.nc_dn, a.tiles_dn);
+                                        a.mt_dn, a.nc_dn, a.tiles_dn, a.e_lo, a.e_hi);
   const long P = (long)a.T * a.k;
   route_perm_kernel<<<ceil_div(P, 256), 256, 0, st>>>(
       a.topk_idx, a.rank, a.blkpre, a.offsets, a.T, a.k, a.nblk, a.E, a.perm, a.pos);

@@ -46,6 +46,7 @@ struct UmmaSmem {
 
 struct TileInfo {
   int grp;         // group (expert) index, 0 in dense mode
+  int wgrp;        // the group's index among the groups the weights hold (grp - grp0)
   int mblk;        // 128-row block of the weight matrix
   int w_row0;      // first weight row (row of the weight tensor map)
   int n0;          // first output column (weight row within the group)
@@ -94,9 +95,10 @@ __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, const int32_t* s_
   const int mblk = local / nnb, nb = local - mblk * nnb;
   if (mblk >= nmb) return false;
   ti.grp = e;
+  ti.wgrp = e - a.grp0;
   ti.mblk = mblk;
   ti.n0 = mblk * kBM;
-  ti.w_row0 = e * a.w_group_rows + ti.n0;
+  ti.w_row0 = ti.wgrp * a.w_group_rows + ti.n0;
   ti.a_row0 = base + nb * NT;
   ti.valid = min(NT, cnt - nb * NT);
   return true;
@@ -128,9 +130,10 @@ __device__ __forceinline__ bool decode_pair_tile(const UmmaArgs& a, const int32_
   const int mblk = local / nnb, nb = local - mblk * nnb;
   if (mblk >= nmb) return false;
   ti.grp = e;
+  ti.wgrp = e - a.grp0;
   ti.mblk = mblk;
   ti.n0 = mblk * kPairBM;
-  ti.w_row0 = e * a.w_group_rows + ti.n0;
+  ti.w_row0 = ti.wgrp * a.w_group_rows + ti.n0;
   ti.a_row0 = base + nb * kPairNT;
   ti.valid = min(kPairNT, cnt - nb * kPairNT);
   ti.kb = 0;

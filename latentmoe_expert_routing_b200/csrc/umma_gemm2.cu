@@ -186,7 +186,7 @@ umma_pair_kernel(const __grid_constant__ CUtensorMap wmap0,
       tc_fence_after();
       const int n = ti.n0 + (int)rank * kBM + 32 * q + lane;   // output column of this thread
       const bool col_ok = n < a.n_out;
-      const float gs = a.gscale ? a.gscale[ti.grp] : 1.f;
+      const float gs = a.gscale ? a.gscale[ti.wgrp] : 1.f;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * kPairNT;
       auto emit = [&](const uint32_t* r, int c) {
         float v[8];

@@ -154,7 +154,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
-        int rec = (ti.grp * a.wq_mblks + ti.mblk) * kt_all;     // first record of the tile
+        int rec = (ti.wgrp * a.wq_mblks + ti.mblk) * kt_all;     // first record of the tile
         bool ok = true;
         for (int st = 0; st < nsteps; ++st, ++it, rec += KS) {
           if (!mbar_wait(&raw_empty[rs], pr)) { fail(11); ok = false; break; }
@@ -288,7 +288,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
       // gscale holds s_g * 2^26 (the bf16 expansion carries 2^-26); exact rescale for fp16
-      const float gs = a.gscale ? (F16 ? a.gscale[ti.grp] * 0x1p-26f : a.gscale[ti.grp]) : 1.f;
+      const float gs = a.gscale ? (F16 ? a.gscale[ti.wgrp] * 0x1p-26f : a.gscale[ti.wgrp]) : 1.f;
       for (int c = grp; c < NT / 8; c += kChunkStep) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
         const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;

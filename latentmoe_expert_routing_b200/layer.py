@@ -35,7 +35,7 @@ class LatentMoE:
 
     def __init__(self, D, L, E, k, F, Fs, weights, *, max_tokens, rsf=5.0,
                  dtype="bf16", expert_fmt="dense", out_dtype=None,
-                 n_group=1, topk_group=1):
+                 n_group=1, topk_group=1, ep_rank=0, ep_ranks=1):
         self.dims = dict(D=D, L=L, E=E, k=k, F=F, Fs=Fs)
         self.dtype = dtype
         self.out_dtype = out_dtype or dtype
@@ -52,7 +52,10 @@ class LatentMoE:
         w = B.moe_weights(*(ptr(n) for n in _DENSE_NAMES + _EXPERT_NAMES), int(on_dev),
                           *(ptr(n) for n in _NVFP4_NAMES), int(on_dev))
         self.cfg = cfg
-        self.handle = B.moe_init(cfg, w, torch.cuda.current_stream().cuda_stream)
+        self.ep = (ep_rank, ep_ranks)
+        st = torch.cuda.current_stream().cuda_stream
+        self.handle = (B.moe_init(cfg, w, st) if ep_ranks == 1 else
+                       B.moe_init_ep(cfg, w, ep_rank, ep_ranks, st))
         if not on_dev:
             self._w = {}                      # copied by moe_init
 
@@ -75,6 +78,37 @@ class LatentMoE:
         B.moe_forward(self.handle, x.data_ptr(), T, out.data_ptr(),
                       topk_idx.data_ptr(), topk_w.data_ptr(), self.stream)
         return out, topk_idx, topk_w
+
+    def ep_partial(self, x, zc_part=None, topk_idx=None, topk_w=None):
+        """Expert parallelism, steps 1-6: (zc_part [T, L] fp32, topk_idx, topk_w)
+        with zc_part the slot-ordered combine of the experts this layer holds."""
+        T = x.shape[0]
+        L, k = self.dims["L"], self.dims["k"]
+        if x.dtype != _TORCH_DT[self.dtype] or not x.is_cuda or x.shape[1] != self.dims["D"]:
+            raise ValueError("x must be a cuda [T, d_model] tensor in the layer dtype")
+        x = x.contiguous()
+        if zc_part is None:
+            zc_part = torch.empty(T, L, dtype=torch.float32, device=x.device)
+        if topk_idx is None:
+            topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+        B.moe_forward_ep_partial(self.handle, x.data_ptr(), T, zc_part.data_ptr(),
+                                 topk_idx.data_ptr(), topk_w.data_ptr(), self.stream)
+        self._ep_T = T
+        return zc_part, topk_idx, topk_w
+
+    def ep_finish(self, parts, t0, Ts, out=None):
+        """Expert parallelism, step 7 on token rows [t0, t0 + Ts): parts
+        [n_ranks, T, L] fp32 (every rank's zc_part, rank order)."""
+        parts = parts.contiguous()
+        n, T = parts.shape[0], parts.shape[1]
+        if out is None:
+            out = torch.empty(Ts, self.dims["D"], dtype=_TORCH_DT[self.out_dtype],
+                              device=parts.device)
+        B.moe_forward_ep_finish(self.handle, parts.data_ptr(), n, T, t0, Ts,
+                                out.data_ptr() if Ts else None, self.stream)
+        return out
 
     def block(self, x, norm_weight, eps=1e-5, out=None, topk_idx=None, topk_w=None):
         """The block around the layer: out = x + layer(RMSNorm(x)); norm_weight [D]
@@ -158,8 +192,19 @@ def weights_for(cfg, device="cuda"):
                 w_shared_down=I.w_shared_down(cfg, device), w_up=up, w_down=down)
 
 
-def layer_for(cfg, weights, max_tokens=None, out_dtype=None):
+def layer_for(cfg, weights, max_tokens=None, out_dtype=None, ep_rank=0, ep_ranks=1):
+    """A layer for config `cfg`; with ep_ranks > 1 the rank's slice of the
+    experts is taken from the full expert tensors in `weights`."""
+    if ep_ranks > 1:
+        from .dist import ep_expert_range
+        e0, e1 = ep_expert_range(ep_rank, ep_ranks, cfg.E)
+        weights = dict(weights)
+        for n in ("w_up", "w_down", "up_codes", "up_scales", "up_gscale", "down_codes",
+                  "down_scales", "down_gscale"):
+            if n in weights:
+                weights[n] = weights[n][e0:e1]
     return LatentMoE(cfg.D, cfg.L, cfg.E, cfg.k, cfg.F, cfg.Fs, weights,
                      max_tokens=max_tokens or cfg.T, rsf=cfg.rsf, dtype=cfg.dtype,
                      expert_fmt=cfg.expert_fmt, out_dtype=out_dtype,
-                     n_group=cfg.n_group, topk_group=cfg.topk_group)
+                     n_group=cfg.n_group, topk_group=cfg.topk_group,
+                     ep_rank=ep_rank, ep_ranks=ep_ranks)
