@@ -98,7 +98,7 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
                              const CUtensorMap* half0 = nullptr,
                              const CUtensorMap* half1 = nullptr) {
   const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
-  const int steps = (g.args.K0 + g.args.K1) / 64;
+  const int steps = (g.args.K0 + g.args.K1 + 63) / 64;
   // Pick the K split with the least modelled time: waves of the persistent grid
   // times (steps per slice + a fixed per-tile cost of about two steps).
   int S = 1;
@@ -106,6 +106,7 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
   for (int c = 1; c <= 64 && c <= steps; ++c) {
     if (steps % c || (c > 1 && steps / c < 2)) continue;
     if (c > 1 && (size_t)c * g.args.M * g.args.n_out > h->splitws_elems) continue;
+    if (c > 1 && g.args.n_out % 16) continue;       // the reduce works in 16-column blocks
     const int waves = ceil_div((long)tiles * c, h->sms);
     const double cost = waves * (steps / (double)c + 2.0) + (c > 1 ? 1.0 : 0.0);
     if (cost < best - 1e-9) { best = cost; S = c; }
@@ -594,7 +595,12 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
        dev_alloc(h, &h->err, 16);
   if (!ok) { moe_destroy(h); return MOE_ERR_OOM; }
   if (c.dtype == MOE_BF16) {
-    if (c.d_model % 64 || c.d_latent % 64 || c.d_ff % 64 || c.d_ff_shared % 64) {
+    // tensor-core tiles: d_model and d_latent in whole 64-wide K steps (a GEMM's
+    // first K segment and the exact-logit order); the expert and shared widths
+    // may end in a partial step (zero-filled TMA boxes, masked output columns),
+    // except for NVFP4 experts, whose records hold whole 64-wide slices
+    if (c.d_model % 64 || c.d_latent % 64 ||
+        (c.expert_fmt != MOE_EXPERT_DENSE && c.d_ff % 64)) {
       moe_destroy(h);
       return MOE_ERR_UNSUPPORTED;
     }

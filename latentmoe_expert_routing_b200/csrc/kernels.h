@@ -113,7 +113,7 @@ cudaError_t noalloc_take_error(int* word);
 namespace lmoe {
 // Tensor-core GEMM (umma_gemm.cu): out[a_row, n] = epi(sum_s A_s[a_row, :] . W_s[w_row, :])
 struct UmmaArgs {
-  int K0, K1;               // K of segment 0 and 1 (multiples of 64; K1 = 0: none)
+  int K0, K1;               // K of segment 0 (a multiple of 64 when K1 > 0) and 1 (K1 = 0: none)
   int n_out;                // output columns = weight rows per group
   int ldo;                  // output row stride (elements)
   int w_group_rows;         // row offset between groups in the weight maps

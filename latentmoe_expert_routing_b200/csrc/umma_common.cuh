@@ -73,7 +73,9 @@ __device__ __forceinline__ bool decode_tile(const UmmaArgs& a, const int32_t* s_
                                             const int32_t* s_off, int tile, TileInfo& ti) {
   const int nmb = (a.n_out + kBM - 1) / kBM;
   const int S = a.offsets ? 1 : (a.ksplit > 1 ? a.ksplit : 1);
-  const int kt_all = (a.K0 + a.K1) / kBK;
+  // a K that is not a multiple of 64 ends in a partial step: the TMA boxes
+  // past the tensor's K are zero-filled (only the last segment may be ragged)
+  const int kt_all = (a.K0 + a.K1 + kBK - 1) / kBK;
   ti.slice = tile % S;
   ti.kb = ti.slice * (kt_all / S);
   ti.ke = ti.kb + kt_all / S;
@@ -137,7 +139,7 @@ __device__ __forceinline__ bool decode_pair_tile(const UmmaArgs& a, const int32_
   ti.a_row0 = base + nb * kPairNT;
   ti.valid = min(kPairNT, cnt - nb * kPairNT);
   ti.kb = 0;
-  ti.ke = (a.K0 + a.K1) / kBK;
+  ti.ke = (a.K0 + a.K1 + kBK - 1) / kBK;
   ti.slice = 0;
   return true;
 }

@@ -49,7 +49,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt0 = a.K0 / kBK;
+  const int kt0 = (a.K0 + kBK - 1) / kBK;      // first step of segment 1
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

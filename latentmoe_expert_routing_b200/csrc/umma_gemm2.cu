@@ -67,7 +67,7 @@ umma_pair_kernel(const __grid_constant__ CUtensorMap wmap0,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = pair2::cluster_rank();
   const bool leader = rank == 0;
-  const int kt0 = a.K0 / kBK;
+  const int kt0 = (a.K0 + kBK - 1) / kBK;      // first step of segment 1
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {

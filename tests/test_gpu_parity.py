@@ -188,3 +188,15 @@ def test_group_routing(L, dtype, E, k, n_group, topk_group, T):
     _assert_out(g[0], r["out"])
     G = E // n_group
     assert all(len(set((row // G).tolist())) <= topk_group for row in g[1].cpu().numpy())
+
+
+@pytest.mark.parametrize("T", [3, 64, 300])
+def test_ragged_expert_and_shared_widths(L, T):
+    """Expert and shared intermediate widths that are not multiples of 64 (the
+    Super shape's 7688 is one): the expert up / shared up GEMMs end in a partial
+    block of output columns, the expert down / fc2 + shared down GEMMs in a
+    partial K step.  T spans the 16-, 64- and 256-token tiles."""
+    cfg = TINY.replace(dtype="bf16", E=16, k=4, D=256, L=64, F=200, Fs=136)
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    _assert_out(g[0], r["out"])
