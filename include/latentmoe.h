@@ -75,6 +75,18 @@ typedef enum {
   MOE_EXPERT_NVFP4_W4A4 = 2    /* NVFP4 weights and NVFP4 expert activations  */
 } moe_expert_fmt;
 
+/* Global scale of the W4A4 latent activations z (NVFP4's second-level FP32
+ * scale; the format fixes it per tensor, the pages say nothing of how it is
+ * chosen for activations). */
+typedef enum {
+  MOE_ACT_SCALE_UNIT = 0,     /* 1.0: the E4M3 block scales alone             */
+  MOE_ACT_SCALE_TENSOR = 1    /* amax(|z|) / (6 * 448) of the forward's latent  */
+                              /* tensor z [T, d_latent], computed on the device */
+                              /* every forward (the weights' rule).  The ReLU^2 */
+                              /* activations keep 1.0: their tensor maximum is  */
+                              /* known only after the whole up projection.      */
+} moe_act_scale;
+
 typedef struct {
   int d_model;        /* D: 8192 for the Ultra shape                         */
   int d_latent;       /* L: moe_latent_size, 2048                            */
@@ -90,6 +102,7 @@ typedef struct {
   moe_dtype dtype;               /* activations and dense weights            */
   moe_expert_fmt expert_fmt;
   moe_dtype out_dtype;           /* dtype of `out`                           */
+  moe_act_scale act_scale;       /* W4A4 only; other formats ignore it       */
 } moe_config;
 
 /* Weights, row-major [out, in] (report section 2.3.4).  Pointers are device

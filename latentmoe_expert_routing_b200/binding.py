@@ -20,6 +20,8 @@ MOE_EXPERT_DENSE, MOE_EXPERT_NVFP4_W4A16, MOE_EXPERT_NVFP4_W4A4 = 0, 1, 2
 EXPERT_FMT = {"dense": MOE_EXPERT_DENSE, "w4a16": MOE_EXPERT_NVFP4_W4A16,
               "w4a4": MOE_EXPERT_NVFP4_W4A4}
 DTYPE = {"fp32": MOE_FP32, "bf16": MOE_BF16}
+MOE_ACT_SCALE_UNIT, MOE_ACT_SCALE_TENSOR = 0, 1
+ACT_SCALE = {"unit": MOE_ACT_SCALE_UNIT, "tensor": MOE_ACT_SCALE_TENSOR}
 
 
 class moe_config(ctypes.Structure):
@@ -30,7 +32,7 @@ class moe_config(ctypes.Structure):
                 ("max_tokens", ctypes.c_int),
                 ("routed_scaling_factor", ctypes.c_float),
                 ("dtype", ctypes.c_int), ("expert_fmt", ctypes.c_int),
-                ("out_dtype", ctypes.c_int)]
+                ("out_dtype", ctypes.c_int), ("act_scale", ctypes.c_int)]
 
 
 class moe_weights(ctypes.Structure):

@@ -59,6 +59,8 @@ struct moe_handle {
   uint8_t *zq = nullptr, *zs = nullptr, *zq_perm = nullptr, *zs_perm = nullptr;
   uint8_t *hq = nullptr, *hs = nullptr;
   float* one = nullptr;                          // activations' global scale (1.0)
+  float* act_gs = nullptr;                       // W4A4 dynamic latent global scale
+  unsigned* act_amax = nullptr;                  // ... and the amax it is made from
   Mxf4Maps mx_up{}, mx_dn{};
   // SM-pair block-scaled GEMMs: scales as atoms (weights [row block][K/64],
   // tokens [token tile][2][K/64]); codes shared with the maps above
@@ -190,6 +192,8 @@ moe_status validate(const moe_config* c) {
     return MOE_ERR_INVALID_ARG;
   if (c->expert_fmt != MOE_EXPERT_DENSE && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  if (c->act_scale != MOE_ACT_SCALE_UNIT && c->act_scale != MOE_ACT_SCALE_TENSOR)
+    return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -368,9 +372,10 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
   const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
   const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
-  const bool mx = use_mxf4(c, P) && h->z32;   // W4A4 on the block-scaled FP4 tensor cores
-  g.args.out = mx ? (void*)h->z32 : h->z;
-  g.epi = mx ? UMMA_EPI_F32 : w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
+  const bool mx = use_mxf4(c, P) && h->zq;    // W4A4 on the block-scaled FP4 tensor cores
+  const bool dyn = w4a4 && h->act_gs;         // the latent's per-tensor global scale
+  g.args.out = (mx || dyn) ? (void*)h->z32 : h->z;
+  g.epi = (mx || dyn) ? UMMA_EPI_F32 : w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
   g.max_tiles = g.args.dense_tiles;
   if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   g.wmap0 = h->wm_su;
@@ -379,12 +384,15 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
   if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   mark(MOE_STAGE_EXPERT_UP);
+  if (dyn && launch_tensor_gscale(h->z32, (long)T * L, h->act_amax, h->act_gs, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   // step 6: routed experts on permuted latent rows (grouped by expert)
   if (mx) {
-    // z rounded to NVFP4 (global scale 1) as codes / scales, gathered per pair;
-    // up: ReLU^2 rounded to NVFP4 as codes / scales; down: fp32
-    if ((e = launch_quantize_rows_nvfp4(h->z32, T, L, h->one, h->zq, h->zs, s)) != cudaSuccess)
+    // z rounded to NVFP4 (global scale 1, or the tensor's) as codes / scales,
+    // gathered per pair; up: ReLU^2 rounded to NVFP4 as codes / scales; down: fp32
+    if ((e = launch_quantize_rows_nvfp4(h->z32, T, L, dyn ? h->act_gs : h->one, h->zq, h->zs,
+                                        s)) != cudaSuccess)
       return MOE_ERR_CUDA;
     const bool mp = use_mxf4_pair(c, P);    // SM pairs: 256-token tiles, 256-row weight blocks
     launch_gather_bytes(h->zq, h->perm, h->zq_perm, P, k, L / 2, s);
@@ -400,6 +408,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     u.args.E = E; u.args.offsets = h->offsets; u.nt = ntg; u.args.grp0 = h->e0;
     u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
     u.args.tiles = h->tiles_up; u.args.out = h->hq; u.args.gscale = h->gs_up;
+    u.args.act_gscale = dyn ? h->act_gs : nullptr;
     u.epi = UMMA_EPI_F16_RELU2_Q;
     u.max_tiles = mp ? (int)((P / 256 + E) * (F / 256)) : (int)((P / ntg + E) * ceil_div(F, 128));
     e = mp ? launch_umma_mxf4_pair(u, h->mxp_up, h->hs_t, s) : launch_umma_mxf4(u, h->mx_up, h->hs, s);
@@ -407,6 +416,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     mark(MOE_STAGE_EXPERT_DOWN);
     u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
     u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.args.gscale = h->gs_dn;
+    u.args.act_gscale = nullptr;                // ReLU^2 activations: global scale 1
     u.epi = UMMA_EPI_F32;
     u.max_tiles = mp ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
     e = mp ? launch_umma_mxf4_pair(u, h->mxp_dn, nullptr, s) : launch_umma_mxf4(u, h->mx_dn, nullptr, s);
@@ -419,7 +429,11 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     launch_combine(h->Y, wts, h->pos, h->zc, T, k, L, MOE_BF16, s);
     mark(MOE_STAGE_DENSE_OUT);
   } else {
-  // (W4A4: z holds NVFP4 round-trip values, exact in fp16, the experts' operand type)
+  // (W4A4: z holds NVFP4 round-trip values, exact in fp16, the experts' operand
+  // type; with the tensor's global scale, values q * s_b and the scale goes to
+  // the up GEMM's epilogue)
+  if (dyn && launch_roundtrip_rows(h->z32, T, L, h->act_gs, h->z, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (w4a4) launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, s);
   else launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
   UmmaLaunch u{};
@@ -437,6 +451,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   };
   if (wq) {
     u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up;
+    u.args.act_gscale = dyn ? h->act_gs : nullptr;
     u.wqmap = h->rm_up[batch_idx(L / 64)];
   }
   const bool pg = grouped_pair(c, P);     // SM pairs: 256-row weight blocks, half-token boxes
@@ -449,6 +464,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
   if (wq) {
     u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn;
+    u.args.act_gscale = nullptr;
     u.wqmap = h->rm_dn[batch_idx(F / 64)];
   }
   u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
@@ -666,6 +682,15 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
       }
     }
   }
+  if (c.dtype == MOE_BF16 && c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 &&
+      c.act_scale == MOE_ACT_SCALE_TENSOR) {
+    // the latent's per-tensor global scale: fc1 writes fp32 z, its amax gives the scale
+    if ((!h->z32 && !dev_alloc(h, &h->z32, T * L * 4)) || !dev_alloc(h, &h->act_gs, 16) ||
+        !dev_alloc(h, &h->act_amax, 16)) {
+      moe_destroy(h);
+      return MOE_ERR_OOM;
+    }
+  }
   if (cudaMemsetAsync(h->err, 0, 16, s) != cudaSuccess ||
       cudaStreamSynchronize(s) != cudaSuccess) {
     moe_destroy(h);
@@ -721,7 +746,7 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
   ra.blkcnt = h->blkcnt; ra.blkpre = h->blkpre; ra.nblk = (T + 31) / 32;
   ra.counts = h->counts; ra.offsets = h->offsets; ra.perm = h->perm; ra.pos = h->pos;
   if (dt == MOE_BF16) {           // tensor-core tiles: 128 (SM pairs: 256) weight rows x NT pairs
-    const bool mp = use_mxf4_pair(c, (long)T * k) && h->z32;   // as forward_umma decides
+    const bool mp = use_mxf4_pair(c, (long)T * k) && h->zq;    // as forward_umma decides
     const int nt = mp ? 256 : kNT[grouped_nt_index(c, (long)T * k)];
     const int bm = (mp || grouped_pair(c, (long)T * k)) ? 256 : 128;
     ra.mt_up = nt; ra.nc_up = ceil_div(F, bm);

@@ -129,6 +129,7 @@ struct UmmaArgs {
   const uint8_t* wq;        // NVFP4 weight records (GEMM layout) or NULL: weights via wmap0
   int wq_mblks;             // 128-row blocks per weight matrix (NVFP4)
   const float* gscale;      // [held groups] per-group output scale (NVFP4 global scale) or NULL
+  const float* act_gscale;  // W4A4: the activations' global scale (one fp32 on the device) or NULL
   int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
                             // fp32 partials out[slice][row][n] (slice stride below)
   long split_stride;        // elements between slices of the partial output
@@ -191,6 +192,10 @@ cudaError_t launch_gather_sf_tiles(const uint8_t* plain, const int32_t* perm,
                                    long P, int k, int K, uint8_t* atoms, cudaStream_t st);
 // NVFP4 codes / scales of fp32 rows [rows, K] with global scale *gscale (1 for
 // activations): the quantiser's encoding, plain layout
+cudaError_t launch_tensor_gscale(const float* x, long n, unsigned* amax, float* gscale,
+                                 cudaStream_t st);
+cudaError_t launch_roundtrip_rows(const float* x, int rows, int K, const float* gscale,
+                                  void* out, cudaStream_t st);
 cudaError_t launch_quantize_rows_nvfp4(const float* x, int rows, int K, const float* gscale,
                                        uint8_t* codes, uint8_t* scales, cudaStream_t st);
 // dst[p] = src[perm[p] / k], rows of row_bytes bytes (multiple of 16)

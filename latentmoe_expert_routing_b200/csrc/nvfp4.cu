@@ -202,6 +202,61 @@ cudaError_t launch_nvfp4_convert_check(unsigned long long* bad, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// Per-tensor global scale of an activation tensor: gscale = amax(|x|) / (6 * 448)
+// (the weights' rule), amax over n fp32 values; `amax` is a device word this
+// call clears first.
+cudaError_t launch_tensor_gscale(const float* x, long n, unsigned* amax, float* gscale,
+                                 cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  if (n > 0) {
+    const long want = (n + 2047) / 2048;           // about 8 values per thread, 2 CTAs per SM at most
+    matrix_amax_kernel<float><<<dim3((unsigned)(want < 296 ? want : 296), 1), 256, 0, st>>>(x, n, amax);
+  }
+  global_scale_kernel<<<1, 32, 0, st>>>(amax, gscale, 1);
+  return cudaGetLastError();
+}
+
+// NVFP4 round trip of fp32 rows [rows, K] in 16-element blocks with the global
+// scale *gscale (the quantiser's arithmetic), written as value(q) * value(s_b):
+// at most 6 significant bits, exact in bf16 and in fp16 (the W4A4 GEMM's operand
+// type, converted by the row gather); the global scale is left to the consumer's
+// epilogue.
+__global__ void roundtrip_rows_kernel(const float* __restrict__ x, long nb,
+                                      const float* __restrict__ gscale,
+                                      __nv_bfloat16* __restrict__ out) {
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= nb) return;
+  const float sg = *gscale;
+  const float* p = x + b * 16;
+  float v[16], amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) { v[i] = p[i]; amax = fmaxf(amax, fabsf(v[i])); }
+  const float den = __fmul_rn(6.0f, sg);
+  const float ratio = den > 0.f ? __fdiv_rn(amax, den) : 0.f;
+  const uint32_t sb = e4m3_encode_pos(ratio);
+  const float sbv = e4m3_value(sb);
+  const float scale = __fmul_rn(sbv, sg);
+  __nv_bfloat16 h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = scale > 0.f ? e2m1_encode(__fdiv_rn(v[i], scale)) : 0u;
+    h[i] = __float2bfloat16_rn(e2m1_value(q) * sbv);   // exact: <= 6 significant bits
+  }
+  uint4* o = reinterpret_cast<uint4*>(out + b * 16);
+  o[0] = *reinterpret_cast<const uint4*>(&h[0]);
+  o[1] = *reinterpret_cast<const uint4*>(&h[8]);
+}
+
+cudaError_t launch_roundtrip_rows(const float* x, int rows, int K, const float* gscale,
+                                  void* out, cudaStream_t st) {
+  if (K % 16) return cudaErrorInvalidValue;
+  const long nb = (long)rows * (K / 16);
+  if (nb == 0) return cudaSuccess;
+  roundtrip_rows_kernel<<<ceil_div(nb, 256), 256, 0, st>>>(x, nb, gscale, (__nv_bfloat16*)out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize_rows_nvfp4(const float* x, int rows, int K, const float* gscale,
                                        uint8_t* codes, uint8_t* scales, cudaStream_t st) {
   if (K % 16) return cudaErrorInvalidValue;

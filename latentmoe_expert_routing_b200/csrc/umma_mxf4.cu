@@ -243,7 +243,9 @@ umma_mxf4_kernel(const __grid_constant__ CUtensorMap wcode_map,
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;              // output column of this thread
       const bool col_ok = n < a.n_out;
-      const float gs = a.gscale[ti.wgrp] * 0x1p-26f;    // weights' global scale s_g
+      // weights' global scale s_g, times the activations' when they have one
+      const float gs = a.act_gscale ? __fmul_rn(a.gscale[ti.wgrp] * 0x1p-26f, *a.act_gscale)
+                                    : a.gscale[ti.wgrp] * 0x1p-26f;
       for (int c = grp; c < kNT / 8 && c * 8 < ti.valid; c += kEpiGroups) {
         uint32_t rg[8];
         tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + buf * kNT + c * 8, rg);

@@ -305,7 +305,9 @@ umma_mxf4_pair_kernel(const __grid_constant__ CUtensorMap wcode_map,
       __syncwarp();
       if (lane == 0) pair2::arrive_remote(empty_leader);
       if (!active) continue;
-      const float gs = a.gscale[ti.wgrp] * 0x1p-26f;    // weights' global scale s_g
+      // weights' global scale s_g, times the activations' when they have one
+      const float gs = a.act_gscale ? __fmul_rn(a.gscale[ti.wgrp] * 0x1p-26f, *a.act_gscale)
+                                    : a.gscale[ti.wgrp] * 0x1p-26f;
       if constexpr (UP) {
         const int row = (int)rank * 128 + 32 * q + lane;       // token row within the pair tile
         if (row >= ti.valid) continue;

@@ -288,7 +288,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
       // gscale holds s_g * 2^26 (the bf16 expansion carries 2^-26); exact rescale for fp16
-      const float gs = a.gscale ? (F16 ? a.gscale[ti.wgrp] * 0x1p-26f : a.gscale[ti.wgrp]) : 1.f;
+      float gs = a.gscale ? (F16 ? a.gscale[ti.wgrp] * 0x1p-26f : a.gscale[ti.wgrp]) : 1.f;
+      if (a.act_gscale) gs = __fmul_rn(gs, *a.act_gscale);   // W4A4 activations' global scale
       for (int c = grp; c < NT / 8; c += kChunkStep) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
         const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;

@@ -35,7 +35,7 @@ class LatentMoE:
 
     def __init__(self, D, L, E, k, F, Fs, weights, *, max_tokens, rsf=5.0,
                  dtype="bf16", expert_fmt="dense", out_dtype=None,
-                 n_group=1, topk_group=1, ep_rank=0, ep_ranks=1):
+                 n_group=1, topk_group=1, ep_rank=0, ep_ranks=1, act_scale="unit"):
         self.dims = dict(D=D, L=L, E=E, k=k, F=F, Fs=Fs)
         self.dtype = dtype
         self.out_dtype = out_dtype or dtype
@@ -47,7 +47,7 @@ class LatentMoE:
         on_dev = on_dev.pop()
         cfg = B.moe_config(D, L, E, k, F, Fs, n_group, topk_group, max_tokens,
                            float(rsf), B.DTYPE[dtype], B.EXPERT_FMT[expert_fmt],
-                           B.DTYPE[self.out_dtype])
+                           B.DTYPE[self.out_dtype], B.ACT_SCALE[act_scale])
         ptr = lambda n: self._w[n].data_ptr() if n in self._w else None
         w = B.moe_weights(*(ptr(n) for n in _DENSE_NAMES + _EXPERT_NAMES), int(on_dev),
                           *(ptr(n) for n in _NVFP4_NAMES), int(on_dev))
@@ -207,4 +207,4 @@ def layer_for(cfg, weights, max_tokens=None, out_dtype=None, ep_rank=0, ep_ranks
                      max_tokens=max_tokens or cfg.T, rsf=cfg.rsf, dtype=cfg.dtype,
                      expert_fmt=cfg.expert_fmt, out_dtype=out_dtype,
                      n_group=cfg.n_group, topk_group=cfg.topk_group,
-                     ep_rank=ep_rank, ep_ranks=ep_ranks)
+                     ep_rank=ep_rank, ep_ranks=ep_ranks, act_scale=cfg.act_scale)

@@ -342,12 +342,13 @@ def nvfp4_dequantize(codes: np.ndarray, scales: np.ndarray, s_g) -> np.ndarray:
     return (q * E4M3_TABLE[scales][..., None] * float(s_g)).reshape(rows, K)
 
 
-def nvfp4_roundtrip_activation(a: np.ndarray) -> np.ndarray:
+def nvfp4_roundtrip_activation(a: np.ndarray, s_g=np.float32(1.0)) -> np.ndarray:
     """W4A4 activation path: round to fp32, quantise along the last axis with
-    global scale 1.0, dequantise (fp64)."""
+    global scale s_g (1.0 unless the layer uses the tensor's own scale),
+    dequantise (fp64)."""
     a32 = np.asarray(a, dtype=np.float32)
-    q, sb = nvfp4_quantize(a32, np.float32(1.0))
-    return nvfp4_dequantize(q, sb, np.float32(1.0))
+    q, sb = nvfp4_quantize(a32, s_g)
+    return nvfp4_dequantize(q, sb, s_g)
 
 
 def pack_e2m1(codes: np.ndarray) -> np.ndarray:
@@ -379,13 +380,16 @@ def expert_weights_fp64(w: np.ndarray, fmt: str) -> np.ndarray:
 
 def forward(x, w_gate, bias, w_fc1, w_fc2, w_su, w_sd, get_up, get_down, *,
             k, rsf, expert_fmt="dense", n_group=1, topk_group=1,
-            norm_topk_prob=True, experts_prepared=False):
+            norm_topk_prob=True, experts_prepared=False, act_scale="unit"):
     """One LatentMoE layer on token rows x[T, D].
 
     get_up(e) -> up_proj[e] [F, L] and get_down(e) -> down_proj[e] [L, F] return
     the stored (bf16 / fp32) expert weights; NVFP4 formats quantise them here.
     With experts_prepared they return instead what expert_weights_fp64 makes of
     the stored weights (a caller may compute those once and reuse them).
+    W4A4 rounds the latent z with global scale 1.0 (act_scale "unit") or with
+    the tensor's own, amax(z) / (6 * 448) over all of z in fp32 ("tensor"), and
+    each expert's ReLU^2 activations with global scale 1.0.
     Returns a dict with out [T, D] fp64 and every routing intermediate."""
     x64 = np.asarray(x, dtype=np.float64)
     T = x64.shape[0]
@@ -395,7 +399,11 @@ def forward(x, w_gate, bias, w_fc1, w_fc2, w_su, w_sd, get_up, get_down, *,
                               n_group, topk_group, norm_topk_prob)   # steps 2-4
     counts, offsets, perm, pos = dispatch(idx, E)
     z = x64 @ np.asarray(w_fc1, dtype=np.float64).T                   # step 5
-    z_in = nvfp4_roundtrip_activation(z) if expert_fmt == "w4a4" else z
+    if expert_fmt == "w4a4":
+        zg = nvfp4_global_scale(z) if act_scale == "tensor" else np.float32(1.0)
+        z_in = nvfp4_roundtrip_activation(z, zg)
+    else:
+        z_in = z
     y = np.zeros((T, k, z.shape[1]), dtype=np.float64)                # step 6
     for e in np.nonzero(counts)[0]:
         tok, slot = np.nonzero(idx == e)

@@ -35,7 +35,7 @@ def oracle_rows(cfg, W, x_rows, rows=None):
                      np32(W["w_fc2"]), np32(W["w_shared_up"]), np32(W["w_shared_down"]),
                      lambda e: get(up, e), lambda e: get(down, e), k=cfg.k, rsf=cfg.rsf,
                      expert_fmt=cfg.expert_fmt, n_group=cfg.n_group,
-                     topk_group=cfg.topk_group)
+                     topk_group=cfg.topk_group, act_scale=cfg.act_scale)
 
 
 def out_metrics(gpu_out, ref):
@@ -84,7 +84,8 @@ def prepared_oracle_rows(cfg, W, x_rows, rows):
                          np32(W["w_fc2"]), np32(W["w_shared_up"]), np32(W["w_shared_down"]),
                          lambda e: get("w_up", e), lambda e: get("w_down", e), k=cfg.k,
                          rsf=cfg.rsf, expert_fmt=cfg.expert_fmt, n_group=cfg.n_group,
-                         topk_group=cfg.topk_group, experts_prepared=True)
+                         topk_group=cfg.topk_group, experts_prepared=True,
+                         act_scale=cfg.act_scale)
 
 
 def ragged_tile_tokens(counts, offsets, perm, k, nt, n=4):

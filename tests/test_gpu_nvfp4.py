@@ -101,6 +101,20 @@ def test_nvfp4_mid_layer(L, fmt, T):
         assert rel <= 1e-2, rel
 
 
+@pytest.mark.parametrize("T", [3, 64, 600, 1200])
+def test_w4a4_latent_tensor_scale(L, T):
+    """W4A4 with the latent's own per-tensor global scale (amax(z) / 2688,
+    computed on the device every forward): the fp16-operand path (16- and
+    64-token tiles), the block-scaled FP4 GEMMs on one SM (~150 pairs per
+    expert) and on SM pairs (~300), against the oracle's tensor-scale layer."""
+    cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt="w4a4", E=16, k=4, D=512,
+                                         L=256, F=512, Fs=512, act_scale="tensor")
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    rel, nmax, raw = out_metrics(g[0], r["out"])
+    assert rel <= REL_L2_NVFP4, (rel, nmax)
+
+
 @pytest.fixture(scope="module")
 def ultra_bf16_weights(L):
     W = L.weights_for(I.CONFIGS["ultra_decode_bf16"])

@@ -231,9 +231,9 @@ def _pins():
 def _z_then_h(fz, fh):
     """fz on the first activation rounding of a forward (the latent z), fh on
     the later ones (each expert's relu(h)^2)."""
-    def wrapped(a):
+    def wrapped(a, *scale):
         _CALLS["n"] += 1
-        return fz(a) if _CALLS["n"] == 1 else fh(a)
+        return fz(a, *scale) if _CALLS["n"] == 1 else fh(a, *scale)
     return wrapped
 
 
@@ -246,14 +246,14 @@ def test_pins_hold_for_the_oracle():
     ("shared_gscale", "w4a16"), ("round_before_relu2", "hand")])
 def test_planted_mistakes_break_a_pin(monkeypatch, mistake, caught_by):
     rt = O.nvfp4_roundtrip_activation
-    ident = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
+    ident = lambda a, *scale: np.asarray(a, dtype=np.float32).astype(np.float64)
     if mistake == "no_h_rounding":
         monkeypatch.setattr(O, "nvfp4_roundtrip_activation", _z_then_h(rt, ident))
     elif mistake == "no_z_rounding":
         monkeypatch.setattr(O, "nvfp4_roundtrip_activation", _z_then_h(ident, rt))
     elif mistake == "z_wrong_axis":           # blocks of 16 tokens instead of 16 latents
         monkeypatch.setattr(O, "nvfp4_roundtrip_activation",
-                            _z_then_h(lambda a: rt(np.asarray(a).T).T, rt))
+                            _z_then_h(lambda a, *scale: rt(np.asarray(a).T, *scale).T, rt))
     elif mistake == "shared_gscale":          # the first matrix's s_g for every matrix
         first = {}
         g = O.nvfp4_global_scale
@@ -263,3 +263,71 @@ def test_planted_mistakes_break_a_pin(monkeypatch, mistake, caught_by):
         monkeypatch.setattr(O, "nvfp4_roundtrip_activation", _z_then_h(rt, ident))
         monkeypatch.setattr(O, "relu2", lambda v: r2(rt(v)))
     assert not _pins()[caught_by]
+
+
+# ---------------------------------------------------------------------------
+# The latent's per-tensor global scale (act_scale "tensor"): s_g = amax(z) /
+# (6 * 448) in fp32, the weights' rule applied to the activation tensor.
+# ---------------------------------------------------------------------------
+
+
+def _quantise_with_own_scale(z):
+    sg = O.nvfp4_global_scale(z)
+    return O.nvfp4_quantize(np.asarray(z, np.float32), sg), sg
+
+
+@pytest.mark.parametrize("j", [-7, -1, 3, 9])
+def test_tensor_scale_codes_invariant_under_power_of_two_scaling(j):
+    """Scaling a tensor by 2^j scales its amax, hence its global scale and every
+    block's ratio, by 2^j exactly: the codes and E4M3 scales do not change."""
+    rng = np.random.RandomState(20 + j)
+    z = (rng.standard_normal((24, 128)) * np.exp(rng.uniform(-3, 3, (24, 1)))).astype(np.float32)
+    (q0, s0), g0 = _quantise_with_own_scale(z)
+    (q1, s1), g1 = _quantise_with_own_scale(z * np.float32(2.0 ** j))
+    assert g1 == np.float32(g0 * np.float32(2.0 ** j))
+    assert np.array_equal(q0, q1) and np.array_equal(s0, s1)
+
+
+def test_tensor_scale_keeps_what_unit_scale_saturates():
+    """A block maximum of 10000 exceeds what global scale 1 can represent
+    (6 * 448 = 2688): with the tensor's own scale it survives up to the fp32
+    rounding of that scale."""
+    z = np.zeros((1, 16), np.float32)
+    z[0, 0], z[0, 1] = 10000.0, 1.0
+    unit = O.nvfp4_roundtrip_activation(z)
+    assert unit[0, 0] == 2688.0
+    sg = O.nvfp4_global_scale(z)
+    tens = O.nvfp4_roundtrip_activation(z, sg)
+    assert abs(tens[0, 0] - 10000.0) <= 10000.0 * 2.0 ** -22
+    assert tens[0, 1] == 0.0          # 1 / (448 * s_g) = 0.27 rounds to code 0 next to 10000
+
+
+def test_tensor_scale_equals_unit_scale_when_it_is_a_power_of_two():
+    """With amax(z) = 2688 * 2^-10 the tensor's scale is exactly 2^-10; every
+    block's E4M3 scale is then the unit-scale one times 2^10 (both normal) and
+    the codes agree, so the two W4A4 layers are equal bit for bit."""
+    rng = np.random.RandomState(31)
+    T, L, E, k, F, Fs = 8, 32, 4, 2, 32, 16
+    z = rng.uniform(-1, 1, (T, L)) * 2.0
+    z[:, ::16] = 0.25 * np.sign(z[:, ::16])          # every block's amax >= 0.25
+    z[0, 5] = 2688.0 * 2.0 ** -10                     # the tensor's amax, 2.625
+    x = z.astype(np.float32)
+    f32 = lambda *s: (rng.standard_normal(s) / np.sqrt(s[-1])).astype(np.float32)
+    up, down = f32(E, F, L), f32(E, L, F)
+    args = (x, f32(E, L), (0.1 * rng.standard_normal(E)).astype(np.float32),
+            np.eye(L, dtype=np.float32), f32(L, L), f32(Fs, L), f32(L, Fs), up, down, k)
+    assert O.nvfp4_global_scale(x) == np.float32(2.0 ** -10)
+    unit = O.forward(*args[:7], lambda e: up[e].astype(np.float64),
+                     lambda e: down[e].astype(np.float64), k=k, rsf=5.0, expert_fmt="w4a4")
+    tens = O.forward(*args[:7], lambda e: up[e].astype(np.float64),
+                     lambda e: down[e].astype(np.float64), k=k, rsf=5.0, expert_fmt="w4a4",
+                     act_scale="tensor")
+    assert np.array_equal(unit["out"], tens["out"])
+    # and a tensor whose scale is not a power of two gives a different layer
+    x2 = x * np.float32(1.5)
+    a2 = (x2,) + args[1:7]
+    u2 = O.forward(*a2, lambda e: up[e].astype(np.float64), lambda e: down[e].astype(np.float64),
+                   k=k, rsf=5.0, expert_fmt="w4a4")
+    t2 = O.forward(*a2, lambda e: up[e].astype(np.float64), lambda e: down[e].astype(np.float64),
+                   k=k, rsf=5.0, expert_fmt="w4a4", act_scale="tensor")
+    assert not np.array_equal(u2["out"], t2["out"])
