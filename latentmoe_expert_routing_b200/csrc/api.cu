@@ -61,6 +61,8 @@ struct moe_handle {
   float* one = nullptr;                          // activations' global scale (1.0)
   float* act_gs = nullptr;                       // W4A4 dynamic latent global scale
   unsigned* act_amax = nullptr;                  // ... and the amax it is made from
+  float* zp2 = nullptr;                          // W4A16: z's power of two and its inverse
+  unsigned* zp2_amax = nullptr;
   Mxf4Maps mx_up{}, mx_dn{};
   // SM-pair block-scaled GEMMs: scales as atoms (weights [row block][K/64],
   // tokens [token tile][2][K/64]); codes shared with the maps above
@@ -241,8 +243,6 @@ moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s)
     return MOE_ERR_OOM;
   }
   if (!pre && (!amax.alloc(E * 4) || (!dev && !dense.alloc(n * 2)))) return MOE_ERR_OOM;
-  // W4A4 streams fp16 operands: its records keep the plain nibble order
-  const int natural = w4a4;
   struct Proj {
     int rows, K;
     const void* dense;
@@ -276,7 +276,7 @@ moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s)
         e = launch_quantize_nvfp4(src, MOE_BF16, (int)E, q.rows, q.K, cu, su, q.gs,
                                   static_cast<unsigned*>(amax.p), s);
     }
-    if (e == cudaSuccess) e = launch_repack_gemm(cu, su, (int)E, q.rows, q.K, q.rec, natural, s);
+    if (e == cudaSuccess) e = launch_repack_gemm(cu, su, (int)E, q.rows, q.K, q.rec, s);
     if (e == cudaSuccess) e = launch_gemm_gscale(q.gs, q.gs, (int)E, s);
     if (e != cudaSuccess) break;
   }
@@ -434,24 +434,36 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   // the up GEMM's epilogue)
   if (dyn && launch_roundtrip_rows(h->z32, T, L, h->act_gs, h->z, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (w4a4) launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, s);
-  else launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
+  // NVFP4 experts take fp16 activations: W4A4's are NVFP4 round-trip values;
+  // W4A16's bf16 z is scaled by the power of two that puts its maximum in
+  // [2^13, 2^14) (exact; the inverse comes back in the up GEMM's epilogue)
+  if (w4a4) {
+    launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, nullptr, h->err, s);
+  } else if (wq) {
+    if (launch_pow2_scale(h->z, (long)T * L, h->zp2_amax, h->zp2, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    launch_gather_rows_f16(h->z, h->perm, h->z_perm, P, k, L, h->zp2, h->err, s);
+  } else {
+    launch_gather_rows(h->z, h->perm, h->z_perm, P, k, L, s);
+  }
   UmmaLaunch u{};
-  u.a_f16 = w4a4;
   u.args.err = h->err;
   u.args.E = E; u.args.offsets = h->offsets; u.args.grp0 = h->e0;
   u.nt = ntg;
   u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
   u.args.tiles = h->tiles_up; u.args.out = h->H;
-  u.epi = w4a4 ? UMMA_EPI_F16_RELU2_Q : UMMA_EPI_BF16_RELU2;
+  u.epi = w4a4 ? UMMA_EPI_F16_RELU2_Q : wq ? UMMA_EPI_F16_RELU2 : UMMA_EPI_BF16_RELU2;
   auto batch_idx = [ntg](int kt) {      // record map box = slices per step of the kernel
     const int ks = wq_slices_per_step(kt, ntg);
     return ks == 4 ? 2 : (ks == 2 ? 1 : 0);
   };
   if (wq) {
     u.args.wq = h->rec_up; u.args.wq_mblks = ceil_div(F, 128); u.args.gscale = h->gs_up;
-    u.args.act_gscale = dyn ? h->act_gs : nullptr;
+    // W4A4: the latent's global scale (if any); W4A16: undo z's power of two,
+    // and write relu^2 scaled by 2^-8 (relu^2(v 2^-4) = relu^2(v) 2^-8) into fp16 H
+    u.args.act_gscale = w4a4 ? (dyn ? h->act_gs : nullptr) : h->zp2 + 1;
+    u.args.acc_mul = w4a4 ? 0.f : 0x1p-4f;
     u.wqmap = h->rm_up[batch_idx(L / 64)];
   }
   const bool pg = grouped_pair(c, P);     // SM pairs: 256-row weight blocks, half-token boxes
@@ -465,6 +477,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   if (wq) {
     u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn;
     u.args.act_gscale = nullptr;
+    u.args.acc_mul = w4a4 ? 0.f : 0x1p8f;         // W4A16: H was stored times 2^-8
     u.wqmap = h->rm_dn[batch_idx(F / 64)];
   }
   u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
@@ -681,6 +694,11 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
         return MOE_ERR_CUDA;
       }
     }
+  }
+  if (c.dtype == MOE_BF16 && c.expert_fmt == MOE_EXPERT_NVFP4_W4A16 &&
+      (!dev_alloc(h, &h->zp2, 16) || !dev_alloc(h, &h->zp2_amax, 16))) {
+    moe_destroy(h);
+    return MOE_ERR_OOM;
   }
   if (c.dtype == MOE_BF16 && c.expert_fmt == MOE_EXPERT_NVFP4_W4A4 &&
       c.act_scale == MOE_ACT_SCALE_TENSOR) {

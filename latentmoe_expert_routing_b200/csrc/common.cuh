@@ -1,6 +1,7 @@
 // Shared device helpers of the LatentMoE CUDA library (sm_100a).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,6 +14,7 @@ enum : int {
   DEV_ERR_INDEX = 1,     // an expert / row index outside its range
   DEV_ERR_TIMEOUT = 2,   // a bounded wait gave up
   DEV_ERR_NONFINITE = 4, // a router logit was NaN
+  DEV_ERR_RANGE = 8,     // a value outside the fp16 range of an fp16 GEMM operand
 };
 
 struct bf16x8 { __nv_bfloat162 v[4]; };
@@ -56,6 +58,7 @@ __device__ __forceinline__ void load8_stream(const float* p, float (&f)[8]) {
 
 __device__ __forceinline__ void store_val(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 __device__ __forceinline__ void store_val(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_val(__half* p, float v) { *p = __float2half_rn(v); }
 
 __device__ __forceinline__ double to_f64(__nv_bfloat16 v) { return (double)__bfloat162float(v); }
 __device__ __forceinline__ double to_f64(float v) { return (double)v; }

@@ -129,7 +129,9 @@ struct UmmaArgs {
   const uint8_t* wq;        // NVFP4 weight records (GEMM layout) or NULL: weights via wmap0
   int wq_mblks;             // 128-row blocks per weight matrix (NVFP4)
   const float* gscale;      // [held groups] per-group output scale (NVFP4 global scale) or NULL
-  const float* act_gscale;  // W4A4: the activations' global scale (one fp32 on the device) or NULL
+  const float* act_gscale;  // the activations' scale (one fp32 on the device: W4A4's global
+                            // scale, or the inverse power of two W4A16 scaled them by) or NULL
+  float acc_mul;            // NVFP4: a power of two the accumulator is multiplied by (0: 1)
   int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
                             // fp32 partials out[slice][row][n] (slice stride below)
   long split_stride;        // elements between slices of the partial output
@@ -137,7 +139,8 @@ struct UmmaArgs {
 // epilogues; _Q variants round the output through NVFP4 in 16-column blocks
 // (F16_RELU2_Q writes fp16: NVFP4 round-trip values are exact fp16 numbers)
 enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2,
-               UMMA_EPI_BF16_Q = 3, UMMA_EPI_BF16_RELU2_Q = 4, UMMA_EPI_F16_RELU2_Q = 5 };
+               UMMA_EPI_BF16_Q = 3, UMMA_EPI_BF16_RELU2_Q = 4, UMMA_EPI_F16_RELU2_Q = 5,
+               UMMA_EPI_F16_RELU2 = 6 };
 struct UmmaLaunch {
   CUtensorMap wmap0, amap0, wmap1, amap1;
   CUtensorMap wqmap;        // NVFP4 records as [records][36][128 B] (see make_tmap_records)
@@ -145,8 +148,6 @@ struct UmmaLaunch {
   int nt;                   // token rows per tile: 16, 64 or 256
   UmmaEpi epi;
   int max_tiles;            // upper bound of the tile count (grid clamp)
-  int a_f16;                // NVFP4 only: activations are fp16 and the records use the
-                            // natural nibble order (both operands exact fp16 values)
 };
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
 // NVFP4 GEMM records (4608 B each) as a 3-D uint8 tensor, box = `batch` records
@@ -205,17 +206,21 @@ cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int ro
                                   uint8_t* codes, uint8_t* scales, float* gscale,
                                   unsigned* amax_tmp, cudaStream_t st);
 cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t st);
-// natural = 0: pairs of a code word 16 bits apart (bf16 expansion by shifts);
-// natural = 1: element 2i in the low nibble of byte i (hardware fp16 conversion)
+// plain layout -> GEMM records (codes in the plain nibble order, element 2i in
+// the low nibble of byte i: the hardware E2M1 -> fp16 conversion reads it)
 cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
-                               int K, uint8_t* out, int natural, cudaStream_t st);
+                               int K, uint8_t* out, cudaStream_t st);
 // adds to *bad the disagreements between the hardware NVFP4 conversions and
 // the format-definition encoders / decoders (see moe_selftest_nvfp4_convert)
 cudaError_t launch_nvfp4_convert_check(unsigned long long* bad, cudaStream_t st);
-// zp[p] = z[perm[p] / k] for each permuted pair, bf16 -> fp16 (exact for values
-// that fp16 represents, such as NVFP4 round-trip outputs)
+// zp[p] = z[perm[p] / k] * mul for each permuted pair, bf16 -> fp16; mul (a
+// power of two on the device, or NULL for 1) keeps the values inside fp16's
+// range; a value that leaves it sets DEV_ERR_RANGE in *err
 void launch_gather_rows_f16(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
-                            cudaStream_t st);
+                            const float* mul, int* err, cudaStream_t st);
+// mul2[0] = 2^s with amax(|z|) * 2^s in [2^13, 2^14) (1 for an all-zero z) and
+// mul2[1] = 2^-s, over the n bf16 values of z; amax is a device word (cleared here)
+cudaError_t launch_pow2_scale(const void* z, long n, unsigned* amax, float* mul2, cudaStream_t st);
 void launch_gather_rows(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
                         cudaStream_t st);
 }  // namespace lmoe

@@ -8,12 +8,9 @@
 // GEMM layout (library internal): per (matrix, 128-row block, 64-K stage) one
 // contiguous 4608-byte record: codes as [half 0..1][row 0..127][16 bytes] (row r's
 // elements 32h..32h+31 at h*2048 + r*16), then 128 rows x 4 scale bytes; rows
-// past the matrix are zero.  Within a row, 32-bit word i holds
-// elements k = 8i..8i+7 with element 8i+2j in bits 4j..4j+3 and element
-// 8i+2j+1 in bits 16+4j..19+4j, so that one shift pair turns the word into a
-// bf16 pair (see the dequant in umma_common.cuh).  The W4A4 layout ("natural")
-// keeps the plain byte order instead (element 2i in the low nibble of byte i),
-// which the hardware E2M1 -> f16x2 conversion reads directly.
+// past the matrix are zero.  The codes keep the plain byte order (element 2i in
+// the low nibble of byte i), which the hardware E2M1 -> f16x2 conversion reads
+// directly.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -75,8 +72,7 @@ __global__ void quantize_blocks_kernel(const T* __restrict__ w, int n_mat, int r
 
 // plain layout -> GEMM layout
 __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-                                   int n_mat, int rows, int K, int natural,
-                                   uint8_t* __restrict__ out) {
+                                   int n_mat, int rows, int K, uint8_t* __restrict__ out) {
   const int nmb = (rows + 127) / 128, nks = K / 64;
   const long rec = (long)blockIdx.x;                 // one record per block, 128 threads = rows
   if (rec >= (long)n_mat * nmb * nks) return;
@@ -90,17 +86,7 @@ __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint
   uint32_t s = 0;
   if (row < rows) {
     const uint8_t* cp = codes + ((size_t)m * rows + row) * (K / 2) + ks * 32;
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t b4 = *reinterpret_cast<const uint32_t*>(cp + 4 * i);   // bytes B0..B3
-      if (natural) { wd[i] = b4; continue; }
-      uint32_t w = 0;
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t bj = (b4 >> (8 * j)) & 0xFFu;
-        w |= (bj & 0xFu) << (4 * j);          // element 8i+2j
-        w |= (bj >> 4) << (16 + 4 * j);       // element 8i+2j+1
-      }
-      wd[i] = w;
-    }
+    for (int i = 0; i < 8; ++i) wd[i] = *reinterpret_cast<const uint32_t*>(cp + 4 * i);
     s = *reinterpret_cast<const uint32_t*>(scales + ((size_t)m * rows + row) * (K / 16) + ks * 4);
   }
   *reinterpret_cast<uint4*>(o + r * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
@@ -143,9 +129,9 @@ cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t 
 }
 
 cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
-                               int K, uint8_t* out, int natural, cudaStream_t st) {
+                               int K, uint8_t* out, cudaStream_t st) {
   const long recs = (long)n_mat * ((rows + 127) / 128) * (K / 64);
-  repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, natural, out);
+  repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, out);
   return cudaGetLastError();
 }
 
@@ -352,28 +338,58 @@ cudaError_t launch_gather_sf_tiles(const uint8_t* plain, const int32_t* perm,
 
 // one thread per 8 elements of a permuted row
 __global__ void gather_rows_f16_kernel(const uint4* __restrict__ z, const int32_t* __restrict__ perm,
-                                       uint4* __restrict__ zp, long P, int k, int row_vecs) {
+                                       uint4* __restrict__ zp, long P, int k, int row_vecs,
+                                       const float* __restrict__ mul, int* __restrict__ err) {
   const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= P * row_vecs) return;
   const long p = i / row_vecs;
   const int c = (int)(i - p * row_vecs);
   const uint4 u = z[(long)(perm[p] / k) * row_vecs + c];
+  const float m = mul ? *mul : 1.f;
   uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  bool bad = false;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-    const __half2 h = __floats2half2_rn(f.x, f.y);
+    const float a = __fmul_rn(f.x, m), b = __fmul_rn(f.y, m);
+    bad |= fabsf(a) > 65504.f || fabsf(b) > 65504.f;
+    const __half2 h = __floats2half2_rn(a, b);
     w[j] = *reinterpret_cast<const uint32_t*>(&h);
   }
+  if (bad && err) atomicOr(err, DEV_ERR_RANGE);
   zp[i] = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 2^s such that amax * 2^s lies in [2^13, 2^14): with amax = 1.f * 2^(E - 127)
+// (E its exponent field) s = 140 - E, kept within [-126, 126] so that both 2^s
+// and 2^-s are normal fp32 numbers, built from their exponent bits
+__global__ void pow2_scale_kernel(const unsigned* __restrict__ amax, float* __restrict__ mul2) {
+  const unsigned bits = *amax;
+  int s = bits ? 140 - (int)(bits >> 23) : 0;
+  s = s < -126 ? -126 : (s > 126 ? 126 : s);
+  mul2[0] = __uint_as_float((unsigned)(s + 127) << 23);
+  mul2[1] = __uint_as_float((unsigned)(127 - s) << 23);
+}
+
+cudaError_t launch_pow2_scale(const void* z, long n, unsigned* amax, float* mul2, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  if (n > 0) {
+    const long want = (n + 2047) / 2048;
+    matrix_amax_kernel<__nv_bfloat16><<<dim3((unsigned)(want < 296 ? want : 296), 1), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(z), n, amax);
+  }
+  pow2_scale_kernel<<<1, 1, 0, st>>>(amax, mul2);
+  return cudaGetLastError();
+}
+
 void launch_gather_rows_f16(const void* z, const int32_t* perm, void* zp, long P, int k, int L,
-                            cudaStream_t st) {
+                            const float* mul, int* err, cudaStream_t st) {
   const int rv = L / 8;
   const long n = P * rv;
   if (n == 0) return;
-  gather_rows_f16_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)z, perm, (uint4*)zp, P, k, rv);
+  gather_rows_f16_kernel<<<ceil_div(n, 256), 256, 0, st>>>((const uint4*)z, perm, (uint4*)zp, P, k, rv,
+                                                           mul, err);
 }
 
 }  // namespace lmoe

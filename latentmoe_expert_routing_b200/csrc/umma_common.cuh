@@ -163,81 +163,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// NVFP4 record -> bf16 W tile.  Record codes are half-major ([half][row][16 B]),
-// so a warp expanding 32 consecutive rows of one half reads 512 contiguous
-// bytes and its swizzled stores hit every bank evenly.
-// Thread (r, half) expands chunks 4*half ..
-// 4*half+3 of row r (k = 8c..8c+7 each) into the 128-byte-swizzled tile: chunk c
-// lands at 16-byte slot c ^ (r & 7).  A record word holds the pair (8c+2j,
-// 8c+2j+1) at bits 4j and 16+4j; shifting the 3 magnitude bits of each code
-// into bf16 bits 6-8 (sign into bit 15) gives exactly q * 2^-126 (code 1 is the
-// bf16 subnormal 2^-127), and one bf16x2 multiply by value(s_b) * 2^100 gives
-// q * s_b * 2^-26 exactly (at most 6 significant bits, normal range).  The
-// epilogue multiplies the accumulator by s_g * 2^26.
-template <int J>
-__device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t x) {
-  constexpr int sa = 6 - 4 * J, sb = 12 - 4 * J;
-  const uint32_t a = sa >= 0 ? (x << sa) : (x >> -sa);
-  const uint32_t b = x << sb;
-  return (a & 0x01C001C0u) | (b & 0x80008000u);
-}
-
-__device__ __forceinline__ void dequant_half(const uint8_t* rec, uint8_t* wtile, int r, int half) {
-  const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
-  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
-  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
-    const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
-    const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 4 * half + 2 * b + cc;
-      const uint32_t x = words[2 * b + cc];
-      uint32_t o[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
-                       e2m1_pair_bits<3>(x)};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&o[j]);
-        v = __hmul2(v, s2);
-        o[j] = *reinterpret_cast<uint32_t*>(&v);
-      }
-      *reinterpret_cast<uint4*>(wtile + r * 128 + ((c ^ (r & 7)) << 4)) =
-          make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-}
-
-// NVFP4 record row r (both halves, k = 0..63) -> 32 packed bf16x2 words in k
-// order, each exactly q * s_b * 2^-26 (see dequant_half).
-__device__ __forceinline__ void dequant_row_regs(const uint8_t* rec, int r, uint32_t (&o)[32]) {
-  const uint32_t sc = reinterpret_cast<const uint32_t*>(rec + 4096)[r];
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const uint4 cw = *reinterpret_cast<const uint4*>(rec + half * 2048 + r * 16);
-    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const uint32_t code = (sc >> (8 * (2 * half + b))) & 0xFFu;
-      const __nv_bfloat16 sv = __float2bfloat16_rn(e4m3_value(code) * 0x1p100f);
-      const __nv_bfloat162 s2 = __halves2bfloat162(sv, sv);
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const uint32_t x = words[2 * b + cc];
-        const int c = 4 * half + 2 * b + cc;            // chunk: k = 8c .. 8c+7
-        uint32_t p[4] = {e2m1_pair_bits<0>(x), e2m1_pair_bits<1>(x), e2m1_pair_bits<2>(x),
-                         e2m1_pair_bits<3>(x)};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&p[j]);
-          v = __hmul2(v, s2);
-          o[4 * c + j] = *reinterpret_cast<uint32_t*>(&v);
-        }
-      }
-    }
-  }
-}
 
 // NVFP4 round trip (global scale 1) of this lane's 8 token values within the
 // 16-lane block of rows it belongs to, as f16x2 pairs (tokens 2p, 2p+1 in

@@ -229,7 +229,9 @@ static EncodeTiledFn encode_fn() {
 // Row-major bf16 matrix [rows, K], box = box_rows x 64 elements, 128-B swizzle.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn || !base || rows <= 0 || K <= 0 || (K % kBK) != 0) return false;
+  // K a multiple of 8 (16-byte row stride); a K that is not a multiple of the
+  // 64-wide box ends in a partial box, whose columns past K read as zeros
+  if (!fn || !base || rows <= 0 || K <= 0 || (K % 8) != 0) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
   cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};

@@ -1,8 +1,8 @@
 // Tensor-core grouped GEMM with NVFP4 expert weights (report section 8.1 /
 // NVFP4 format details; section 5.6 step 6).  Same tiling and orientation as
-// umma_gemm_kernel (128 weight rows x NT token rows, bf16 kind::f16 MMA into a
+// umma_gemm_kernel (128 weight rows x NT token rows, fp16 kind::f16 MMA into a
 // double-buffered TMEM accumulator); the weights arrive as 4608-byte NVFP4
-// records and are expanded to exact bf16 rows directly in tensor memory, from
+// records and are expanded to exact fp16 rows directly in tensor memory, from
 // where the MMA reads its A operand ("TS" form).
 //
 // A 64-K slice of NVFP4 weights is only 4.6 KB, and every tcgen05 instruction
@@ -30,11 +30,17 @@
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
 //
-// W4A4 runs the same pipeline on fp16 operands (F16): the activations are
-// NVFP4 round-trip values and the dequantised weights are q * s_b, all exact
-// fp16 numbers, so the hardware E2M1 -> f16x2 conversion expands the weights
-// (about one instruction per element instead of seven) and the MMA computes
-// the same exact products as in bf16.
+// Both operands are fp16.  The dequantised weights q * s_b (at most 6
+// significant bits, magnitudes in [2^-10, 2688]) are exact fp16 numbers, so the
+// hardware E2M1 -> f16x2 conversion expands a pair of codes in one instruction
+// (the expansion is integer-ALU bound otherwise) and one fp16x2 multiply
+// applies the block scale; the epilogue multiplies by the global scale.  W4A4
+// activations are NVFP4 round-trip values, exact in fp16.  W4A16 activations
+// are bf16 values scaled by a power of two into fp16's range (exact for every
+// value within 2^31 of the tensor's maximum; the inverse power of two comes
+// back in the epilogue), and the up projection writes its ReLU^2 output as
+// fp16 scaled by 2^-8 (acc_mul), which the down projection undoes; a value
+// outside fp16's range sets DEV_ERR_RANGE.
 #include <cuda_fp16.h>
 #include <stdlib.h>
 
@@ -79,7 +85,7 @@ __device__ __forceinline__ int mma_thread(int warp) {
   return warp == 3 ? 1 : warp == 16 ? 2 : warp == 18 ? 3 : -1;
 }
 
-template <int NT, int RAW, typename TO, bool RELU2, bool QA, bool F16>
+template <int NT, int RAW, typename TO, bool RELU2, bool QA>
 __global__ void __launch_bounds__(kWqThreads, 1)
 umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wqmap,
                const UmmaArgs a) {
@@ -211,7 +217,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const uint32_t d = tmem + (2 * j + buf) * NT;
         // ragged tiles multiply only their valid rows, rounded up to N granularity 16
         const int n_eff = min(NT, (ti.valid + 15) & ~15);
-        const uint32_t idesc = F16 ? idesc_f16_f32(kBM, n_eff) : idesc_bf16_f32(kBM, n_eff);
+        const uint32_t idesc = idesc_f16_f32(kBM, n_eff);
         bool ok = true;
         for (int st = 0; st < nsteps; ++st) {
           // W ready implies the step's A tiles landed (the dequant warps waited for them)
@@ -260,8 +266,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const uint8_t* rec = smem + S::kRawOffset + rr * S::kRawSlotBytes;
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t o[32];
-          if (F16) dequant_row_f16(rec + ks * kWqRecordBytes, r, o);
-          else dequant_row_regs(rec + ks * kWqRecordBytes, r, o);
+          dequant_row_f16(rec + ks * kWqRecordBytes, r, o);
           tmem_st32(lane_base + sw * 32 * KS + ks * 32, o);
         }
         tmem_st_wait();
@@ -287,9 +292,11 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
-      // gscale holds s_g * 2^26 (the bf16 expansion carries 2^-26); exact rescale for fp16
-      float gs = a.gscale ? (F16 ? a.gscale[ti.wgrp] * 0x1p-26f : a.gscale[ti.wgrp]) : 1.f;
-      if (a.act_gscale) gs = __fmul_rn(gs, *a.act_gscale);   // W4A4 activations' global scale
+      // gscale holds s_g * 2^26: exact rescale by 2^-26; then the activations'
+      // scale and the accumulator's power of two
+      float gs = a.gscale ? a.gscale[ti.wgrp] * 0x1p-26f : 1.f;
+      if (a.act_gscale) gs = __fmul_rn(gs, *a.act_gscale);
+      if (a.acc_mul != 0.f) gs = __fmul_rn(gs, a.acc_mul);
       for (int c = grp; c < NT / 8; c += kChunkStep) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
         const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;
@@ -314,7 +321,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
         }
-        if constexpr (QA && F16) {
+        if constexpr (QA) {
           uint32_t hq[4];
           nvfp4_roundtrip16x8_h(v, hq);
           unsigned short* o16 = reinterpret_cast<unsigned short*>(a.out);
@@ -325,7 +332,12 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
               o16[(size_t)(ti.a_row0 + row) * a.ldo + n] = (unsigned short)(hq[j >> 1] >> (16 * (j & 1)));
           }
         } else {
-          if (QA) nvfp4_roundtrip16x8(v);
+          if constexpr (sizeof(TO) == 2) {    // fp16 activations for the next GEMM
+            bool bad = false;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) bad |= (c * 8 + j < ti.valid) && fabsf(v[j]) > 65504.f;
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(a.err, DEV_ERR_RANGE);
+          }
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int row = c * 8 + j;
@@ -346,7 +358,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   }
 }
 
-template <int NT, int RAW, typename TO, bool RELU2, bool QA, bool F16>
+template <int NT, int RAW, typename TO, bool RELU2, bool QA>
 static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   using S = WqSmem<NT, RAW>;
   static_assert(S::kBytes <= 232448, "shared memory budget");
@@ -355,7 +367,7 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   // alias); wq_slices_per_step keeps at least two W slots
   static_assert(S::kMaxSW >= kDqGroups && RAW >= kDqGroups, "ring too shallow for the dequant groups");
   static_assert(3 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
-  auto kern = umma_wq_kernel<NT, RAW, TO, RELU2, QA, F16>;
+  auto kern = umma_wq_kernel<NT, RAW, TO, RELU2, QA>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -373,17 +385,10 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
 
 template <int NT, int RAW>
 static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
-  if (L.a_f16) {                         // W4A4: fp16 operands, natural record order
-    switch (L.epi) {
-      case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, RAW, __half, true, true, true>(L, st);
-      case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false, true>(L, st);
-      default: return cudaErrorInvalidValue;
-    }
-  }
   switch (L.epi) {
-    case UMMA_EPI_BF16: return wq_launch_t<NT, RAW, __nv_bfloat16, false, false, false>(L, st);
-    case UMMA_EPI_BF16_RELU2: return wq_launch_t<NT, RAW, __nv_bfloat16, true, false, false>(L, st);
-    case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false, false>(L, st);
+    case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, RAW, __half, true, true>(L, st);    // W4A4 up
+    case UMMA_EPI_F16_RELU2: return wq_launch_t<NT, RAW, __half, true, false>(L, st);     // W4A16 up
+    case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false>(L, st);           // down
     default: return cudaErrorInvalidValue;
   }
 }
