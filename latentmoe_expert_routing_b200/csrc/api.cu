@@ -45,6 +45,7 @@ struct moe_handle {
   float* wnorm = nullptr;                        // ||w_gate[e]||_2 (certified router)
   float* wstat = nullptr;                        // max / min nonzero |w_gate[e]|
   float* splitws = nullptr;                      // split-K partials of the dense GEMMs
+  float* logit_parts = nullptr;                  // the router GEMM's split-K partial logits
   size_t splitws_elems = 0;
   int sms = 148;
   // NVFP4 experts: GEMM-layout records and per-expert global scales
@@ -139,6 +140,25 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
 }
 
 int nt_index(long rows_per_group) { return rows_per_group <= 16 ? 0 : rows_per_group <= 64 ? 1 : 2; }
+
+// K slices of the router GEMM (bf16 layers): its logits come out as fp32 partial
+// sums over D / S consecutive k each, which the certified router adds in fp64.
+// A slice's accumulation error bound scales with its length, so more slices
+// mean fewer experts whose logit has to be recomputed exactly; decode-sized
+// batches take 32 slices (they also fill the GPU), larger ones 8 (partials of
+// 8 T E floats).  S divides the D / 64 K steps.
+int router_splits(int D, int T) {
+  const int kt = D / 64;
+  for (int c = T <= 256 ? 32 : 8; c > 1; c >>= 1)
+    if (kt % c == 0) return c;
+  return 1;
+}
+
+size_t router_parts_elems(int D, int E, int max_tokens) {
+  const size_t small = (size_t)router_splits(D, 1) * (max_tokens < 256 ? max_tokens : 256);
+  const size_t large = max_tokens > 256 ? (size_t)router_splits(D, max_tokens) * max_tokens : 0;
+  return (small > large ? small : large) * E;
+}
 
 // Token rows per grouped-GEMM tile: NVFP4 experts keep their dequantised
 // weights in TMEM next to the accumulators, so their widest tile is 128 rows.
@@ -636,6 +656,7 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
     cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
     h->splitws_elems = kSplitWsElems;
     if (!dev_alloc(h, &h->splitws, h->splitws_elems * 4) ||
+        !dev_alloc(h, &h->logit_parts, router_parts_elems((int)D, (int)E, (int)T) * 4) ||
         !dev_alloc(h, &h->z_perm, P * L * 2) || !dev_alloc(h, &h->wnorm, E * 4) ||
         !dev_alloc(h, &h->wstat, E * 8) ||
         !dev_alloc(h, &h->stats, 16)) {
@@ -750,10 +771,11 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
     g.wmap0 = h->wm_gate; g.amap0 = xmap; g.nt = kNT[nt_index(T)];
     g.args.err = h->err; g.args.E = 1; g.args.M = T;
     g.args.K0 = D; g.args.n_out = E; g.args.ldo = E;
-    g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt);
-    g.args.out = h->logits; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
-    moe_status ls = launch_dense_umma(h, g, s, wide ? &xhalf : nullptr);
-    if (ls != MOE_OK) return ls;
+    g.args.ksplit = router_splits(D, T);          // partials [S][T][E], no reduce
+    g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt) * g.args.ksplit;
+    g.args.split_stride = (long)T * E;
+    g.args.out = h->logit_parts; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
+    if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
   }
@@ -779,7 +801,8 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
   ra.e_lo = h->e0; ra.e_hi = h->e0 + h->e_loc;
   if (dt == MOE_BF16) {
     CertArgs ca{(const __nv_bfloat16*)hidden, (const __nv_bfloat16*)h->w_gate, h->wnorm, D,
-                h->stats, h->wstat};
+                h->stats, h->wstat, h->logit_parts, router_splits(D, T), (long)T * E,
+                h->logits};
     launch_route_fused(ra, ca, s);
   } else {
     launch_route(ra, s);

@@ -46,6 +46,14 @@ struct CertArgs {
   int D;
   unsigned long long* stats;  // += number of exactly recomputed logits (or NULL)
   const float* wstat;       // [E][2] max |w_e|, min nonzero |w_e| (or NULL: double path)
+  // the tensor-core logits as `splits` fp32 partial sums over D / splits
+  // consecutive k each, parts[s][t][e]; the kernel adds them in fp64, rounds to
+  // fp32 and writes the result to logits_out.  NULL: RouteArgs::logits holds
+  // fp32 logits over the whole K.
+  const float* parts;
+  int splits;
+  long part_stride;
+  float* logits_out;
 };
 void launch_route_fused(const RouteArgs& a, const CertArgs& c, cudaStream_t st);
 void launch_row_norms(const void* w, int rows, int D, float* out, float* stat, cudaStream_t st);

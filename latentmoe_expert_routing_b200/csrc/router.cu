@@ -584,12 +584,25 @@ route_fused_kernel(RouteArgs a, CertArgs ca) {
     xmax = fmaxf(xmax, s_mx[w]);
     xmin = fminf(xmin, s_mn[w]);
   }
-  const double u = 0x1p-23, Ku = D * u;
-  const double g = kCertMargin * Ku / (1.0 - Ku);
+  // each fp32 accumulation covers D / splits terms; with partial sums, their
+  // fp64 total rounded to fp32 adds at most 2^-24 |l~| <= 2^-24 ||x|| ||w|| more
+  const int Kacc = ca.parts ? D / ca.splits : D;
+  const double u = 0x1p-23, Ku = Kacc * u;
+  const double g = kCertMargin * Ku / (1.0 - Ku) + (ca.parts ? 0x1p-23 : 0.0);
   const double dscale = 0.25 * g * sqrt((double)tot) * (1.0 + 0x1p-9);
   double cu = -INFINITY, lo = -INFINITY;
   if (e < E) {
-    const double c = (double)__fadd_rn(sigmoid_fixed(a.logits[(size_t)t * E + e]), a.bias[e]);
+    float lt;
+    if (ca.parts) {
+      const float* p = ca.parts + (size_t)t * E + e;
+      double acc = 0.0;
+      for (int s = 0; s < ca.splits; ++s) acc += (double)p[s * ca.part_stride];
+      lt = __double2float_rn(acc);
+      ca.logits_out[(size_t)t * E + e] = lt;
+    } else {
+      lt = a.logits[(size_t)t * E + e];
+    }
+    const double c = (double)__fadd_rn(sigmoid_fixed(lt), a.bias[e]);
     const double d = dscale * ca.wnorm[e] + kCertEps;
     cu = c + d;
     lo = c - d;
