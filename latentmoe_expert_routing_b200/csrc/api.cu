@@ -70,7 +70,7 @@ struct moe_handle {
   uint8_t *wa_up = nullptr, *wa_dn = nullptr, *zs_t = nullptr, *hs_t = nullptr;
   Mxf4Maps mxp_up{}, mxp_dn{};
   CUtensorMap wm_gate, wm_fc1, wm_su, wm_up, wm_dn, wm_fc2, wm_sd;
-  CUtensorMap am_zp[4], am_H[4], am_zc[4], am_hsh[4];   // token boxes of 16, 64, 256, 128 rows
+  CUtensorMap am_zp[5], am_H[5], am_zc[5], am_hsh[5];   // token boxes of 16, 64, 256, 128, 32 rows
   int prof = 0, prof_valid = 0;                    // stage timing (moe_profile_*)
   cudaEvent_t ev[MOE_NUM_STAGES + 1] = {};
 };
@@ -92,7 +92,7 @@ __global__ void selftest_wait_kernel(const volatile int* flag, long long cycles,
   }
 }
 
-const int kNT[4] = {16, 64, 256, 128};
+const int kNT[5] = {16, 64, 256, 128, 32};
 const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K partials
 
 // Dense tensor-core GEMM with split-K when its output tiles cannot fill the
@@ -162,9 +162,14 @@ size_t router_parts_elems(int D, int E, int max_tokens) {
 
 // Token rows per grouped-GEMM tile: NVFP4 experts keep their dequantised
 // weights in TMEM next to the accumulators, so their widest tile is 128 rows.
+// NVFP4 experts expand their weights once per token tile, so their decode
+// tiles grow with the pairs per expert: 16 tokens up to 8 pairs per expert on
+// average, 32 up to 32 (an expert of a decode batch rarely needs a second
+// tile), 64, then 128.
 int grouped_nt_index(const moe_config& c, long P) {
-  const int i = nt_index(P / c.n_experts);
-  return (c.expert_fmt != MOE_EXPERT_DENSE && i == 2) ? 3 : i;
+  const long per = P / c.n_experts;
+  if (c.expert_fmt == MOE_EXPERT_DENSE) return nt_index(per);
+  return per <= 8 ? 0 : per <= 32 ? 4 : per <= 64 ? 1 : 3;
 }
 
 // Grouped bf16 GEMMs with 256-token tiles run on SM pairs (256-row weight
@@ -672,7 +677,7 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
                                  make_tmap_bf16(&h->wm_dn, h->w_down, El * L, F, 128))) &&
              make_tmap_bf16(&h->wm_fc2, h->w_fc2, D, L, 128) &&
              make_tmap_bf16(&h->wm_sd, h->w_sd, D, Fs, 128);
-    for (int i = 0; i < 4 && m; ++i)
+    for (int i = 0; i < 5 && m; ++i)
       m = make_tmap_bf16(&h->am_zp[i], h->z_perm, P, L, kNT[i]) &&
           make_tmap_bf16(&h->am_H[i], h->H, P, F, kNT[i]) &&
           make_tmap_bf16(&h->am_zc[i], h->zc, T, L, kNT[i]) &&

@@ -19,10 +19,10 @@
 //   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
 //   2      activation producer (TMA tiles into the A ring)
-//   3, 16, 18  16-token tiles: further MMA issuers -- four threads, one per SM
+//   3, 16, 18  16- and 32-token tiles: further MMA issuers -- four threads, one per SM
 //          sub-partition, thread j issuing the j-th 16-K step of every slice
 //          into its own accumulator pair; otherwise idle
-//   4-7    epilogue group 0 (16-token tiles: every chunk, summing the four
+//   4-7    epilogue group 0 (16-/32-token tiles: every chunk, summing the four
 //          accumulators; otherwise the even 8-column chunks)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
 //          alternate steps; each thread expands its weight row's slices
@@ -52,8 +52,8 @@ constexpr int kMaxKS = 4;                    // 64-K slices per pipeline step
 
 template <int NT, int RAW>
 struct WqSmem {
-  // 16-token tiles keep four accumulator pairs (four MMA threads)
-  static constexpr int kAccCols = (NT == 16 ? 8 : 2) * NT;
+  // 16- and 32-token tiles keep four accumulator pairs (four MMA threads)
+  static constexpr int kAccCols = (NT <= 32 ? 8 : 2) * NT;
   static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
   static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
   static constexpr int kATileBytes = NT * kBK * 2;                     // one 64-K slice, multiple of 1024
@@ -76,7 +76,7 @@ __device__ __forceinline__ int dq_group(int warp) {
   return (warp >= 8 && warp < 16) ? (warp - 8) >> 2 : -1;
 }
 
-// MMA thread index of a warp (lane 0 issues): warp 1, and for 16-token tiles
+// MMA thread index of a warp (lane 0 issues): warp 1, and for 16-/32-token tiles
 // warps 3, 16, 18 -- one per SM sub-partition (warp % 4); -1 otherwise
 template <bool SPLIT>
 __device__ __forceinline__ int mma_thread(int warp) {
@@ -107,11 +107,11 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 16-token tiles: four threads issue the MMAs (thread j the j-th 16-K step of
+  // 16-/32-token tiles: four threads issue the MMAs (thread j the j-th 16-K step of
   // every slice) into four accumulators that the epilogue adds; each tcgen05
   // instruction holds its issuing thread for ~55 cycles, four times a
   // 128 x 16 x 16 MMA's time on the tensor pipe
-  constexpr bool SPLIT = NT == 16;
+  constexpr bool SPLIT = NT <= 32;
   constexpr uint32_t NM = SPLIT ? 4 : 1;    // MMA threads
   constexpr int kEpiThreads = SPLIT ? 128 : 256;
   const int kt_all = a.K0 / kBK;
@@ -278,7 +278,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     }
   } else if ((warp >= 4 && warp < 8) || (!SPLIT && warp >= 16 && warp < 20)) {
     // ---------------- epilogue (two groups split the accumulator's chunks;
-    // 16-token tiles: group 0 alone) ----------------
+    // 16-/32-token tiles: group 0 alone) ----------------
     const int q = warp & 3;
     const int grp = warp >= 16 ? 1 : 0;
     constexpr int kChunkStep = SPLIT ? 1 : 2;
@@ -397,6 +397,7 @@ cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st) {
   if (L.args.K1 != 0 || !L.args.wq) return cudaErrorInvalidValue;
   switch (L.nt) {
     case 16: return wq_launch_nt<16, 9>(L, st);             // A 24 KB + records 166 KB
+    case 32: return wq_launch_nt<32, 9>(L, st);             // A 32 KB + records 166 KB
     case 64: return wq_launch_nt<64, 6>(L, st);             // A 96 KB + records 110 KB
     case 128: return wq_launch_nt<128, 4>(L, st);           // A 128 KB + records 74 KB
   }
