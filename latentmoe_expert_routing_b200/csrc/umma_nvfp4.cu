@@ -13,16 +13,19 @@
 // one commit per step frees the step's A slot and W slot together.  The
 // dequantised W tiles live in TMEM (slots of 32*KS columns next to the
 // accumulators), which leaves shared memory for the record batches (covering
-// HBM latency) and the activation tiles.
+// HBM latency) and the activation tiles.  A slot is reused only after the
+// MMAs of the step before last that used it completed, so the pipeline depth
+// is the slot count: 16- and 32-token tiles keep two accumulator pairs (two
+// MMA threads) and three slots -- measured faster than four threads with two
+// slots, or two threads with six half-size slots.
 //
 // Warps (640 threads):
 //   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
 //   2      activation producer (TMA tiles into the A ring)
-//   3, 16, 18  16- and 32-token tiles: further MMA issuers -- four threads, one per SM
-//          sub-partition, thread j issuing the j-th 16-K step of every slice
-//          into its own accumulator pair; otherwise idle
-//   4-7    epilogue group 0 (16-/32-token tiles: every chunk, summing the four
+//   3      16- and 32-token tiles: the second MMA issuer (16-K steps 2-3 of
+//          every slice into its own accumulator pair); otherwise idle
+//   4-7    epilogue group 0 (16-/32-token tiles: every chunk, summing the two
 //          accumulators; otherwise the even 8-column chunks)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
 //          alternate steps; each thread expands its weight row's slices
@@ -52,8 +55,8 @@ constexpr int kMaxKS = 4;                    // 64-K slices per pipeline step
 
 template <int NT, int RAW>
 struct WqSmem {
-  // 16- and 32-token tiles keep four accumulator pairs (four MMA threads)
-  static constexpr int kAccCols = (NT <= 32 ? 8 : 2) * NT;
+  // 16- and 32-token tiles keep two accumulator pairs (two MMA threads)
+  static constexpr int kAccCols = (NT <= 32 ? 4 : 2) * NT;
   static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
   static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
   static constexpr int kATileBytes = NT * kBK * 2;                     // one 64-K slice, multiple of 1024
@@ -77,12 +80,11 @@ __device__ __forceinline__ int dq_group(int warp) {
 }
 
 // MMA thread index of a warp (lane 0 issues): warp 1, and for 16-/32-token tiles
-// warps 3, 16, 18 -- one per SM sub-partition (warp % 4); -1 otherwise
+// warp 3 as well; -1 otherwise
 template <bool SPLIT>
 __device__ __forceinline__ int mma_thread(int warp) {
   if (warp == 1) return 0;
-  if (!SPLIT) return -1;
-  return warp == 3 ? 1 : warp == 16 ? 2 : warp == 18 ? 3 : -1;
+  return (SPLIT && warp == 3) ? 1 : -1;
 }
 
 template <int NT, int RAW, typename TO, bool RELU2, bool QA>
@@ -107,12 +109,12 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 16-/32-token tiles: four threads issue the MMAs (thread j the j-th 16-K step of
-  // every slice) into four accumulators that the epilogue adds; each tcgen05
-  // instruction holds its issuing thread for ~55 cycles, four times a
-  // 128 x 16 x 16 MMA's time on the tensor pipe
+  // 16-/32-token tiles: two threads issue the MMAs (thread j the 16-K steps 2j and
+  // 2j+1 of every slice) into two accumulators that the epilogue adds; each
+  // tcgen05 instruction holds its issuing thread for ~55 cycles (more on a
+  // loaded SM), several times a 128 x 32 x 16 MMA's time on the tensor pipe
   constexpr bool SPLIT = NT <= 32;
-  constexpr uint32_t NM = SPLIT ? 4 : 1;    // MMA threads
+  constexpr uint32_t NM = SPLIT ? 2 : 1;    // MMA threads
   constexpr int kEpiThreads = SPLIT ? 128 : 256;
   const int kt_all = a.K0 / kBK;
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
@@ -203,7 +205,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     }
   } else if (mma_thread<SPLIT>(warp) >= 0) {
     // ---------------- MMA issuer(s) (A from TMEM, B from shared memory) ----------------
-    const int j = mma_thread<SPLIT>(warp);    // SPLIT: the j-th 16-K step of every slice
+    const int j = mma_thread<SPLIT>(warp);    // SPLIT: 16-K steps 2j, 2j+1 of every slice
     if (lane == 0) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
       const uint32_t slot_desc = (uint32_t)((KS * S::kATileBytes) >> 4);
@@ -227,7 +229,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
           uint64_t bd = bdesc0 + (uint64_t)(s * slot_desc);
           for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
             if (SPLIT) {
-              mma_bf16_ts(d, wt + 8 * j, bd + 2 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(d, wt + 16 * j, bd + 4 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
+              mma_bf16_ts(d, wt + 16 * j + 8, bd + 4 * j + 2, idesc, 1u);
             } else {
               mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
               mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
@@ -300,23 +303,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       for (int c = grp; c < NT / 8; c += kChunkStep) {
         if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
         const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;
-        uint32_t r0[8], r1[8], r2[8], r3[8];
+        uint32_t r0[8], r1[8];
         tmem_ld8(row_base + buf * NT, r0);
-        if (SPLIT) {
-          tmem_ld8(row_base + (2 + buf) * NT, r1);
-          tmem_ld8(row_base + (4 + buf) * NT, r2);
-          tmem_ld8(row_base + (6 + buf) * NT, r3);
-        }
+        if (SPLIT) tmem_ld8(row_base + (2 + buf) * NT, r1);
         tmem_ld_wait();
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          // the four partial sums (16-K steps 0..3 of every slice), added in order
-          const float acc =
-              SPLIT ? __fadd_rn(__fadd_rn(__fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j])),
-                                          __uint_as_float(r2[j])),
-                                __uint_as_float(r3[j]))
-                    : __uint_as_float(r0[j]);
+          // the two partial sums (16-K steps 0-1 and 2-3 of every slice)
+          const float acc = SPLIT ? __fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]))
+                                  : __uint_as_float(r0[j]);
           v[j] = __fmul_rn(acc, gs);
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
