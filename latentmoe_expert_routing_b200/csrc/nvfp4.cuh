@@ -78,8 +78,11 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
   return d;
 }
 
-// v / s for the E2M1 decision from r = RN(1 / s): one multiply and one
-// FMA-refined correction (the residual v - y0 s is exact); 0 when r = 0.
+// v / s for the E2M1 decision from r = RN(1 / s): the quotient y0 = RN(v r)
+// followed by one Markstein correction step y1 = y0 + r (v - y0 s), whose
+// residual v - y0 s one FMA forms exactly (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990); 0 when r = 0.
 __device__ __forceinline__ float nvfp4_div(float v, float s, float r) {
   const float y0 = __fmul_rn(v, r);
   return __fmaf_rn(__fmaf_rn(-y0, s, v), r, y0);
