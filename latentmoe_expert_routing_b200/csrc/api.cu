@@ -476,6 +476,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   u.args.E = E; u.args.offsets = h->offsets; u.args.grp0 = h->e0;
   u.nt = ntg;
   u.wmap0 = h->wm_up; u.amap0 = h->am_zp[gi];
+  u.amap1 = h->am_zp[0];                  // NVFP4: 16-row boxes for tiles of <= 16 tokens
   u.args.K0 = L; u.args.n_out = F; u.args.ldo = F; u.args.w_group_rows = F;
   u.args.tiles = h->tiles_up; u.args.out = h->H;
   u.epi = w4a4 ? UMMA_EPI_F16_RELU2_Q : wq ? UMMA_EPI_F16_RELU2 : UMMA_EPI_BF16_RELU2;
@@ -496,7 +497,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   u.max_tiles = pg ? (int)((P / 256 + E) * (F / 256)) : (int)((P / ntg + E) * ceil_div(F, 128));
   if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(MOE_STAGE_EXPERT_DOWN);
-  u.wmap0 = h->wm_dn; u.amap0 = h->am_H[pg ? 3 : gi];
+  u.wmap0 = h->wm_dn; u.amap0 = h->am_H[pg ? 3 : gi]; u.amap1 = h->am_H[0];
   u.args.K0 = F; u.args.n_out = L; u.args.ldo = L; u.args.w_group_rows = L;
   u.args.tiles = h->tiles_dn; u.args.out = h->Y; u.epi = UMMA_EPI_F32;
   if (wq) {

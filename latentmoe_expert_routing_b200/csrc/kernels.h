@@ -150,7 +150,7 @@ enum UmmaEpi { UMMA_EPI_BF16 = 0, UMMA_EPI_BF16_RELU2 = 1, UMMA_EPI_F32 = 2,
                UMMA_EPI_BF16_Q = 3, UMMA_EPI_BF16_RELU2_Q = 4, UMMA_EPI_F16_RELU2_Q = 5,
                UMMA_EPI_F16_RELU2 = 6 };
 struct UmmaLaunch {
-  CUtensorMap wmap0, amap0, wmap1, amap1;
+  CUtensorMap wmap0, amap0, wmap1, amap1;   // NVFP4 experts: amap1 = the token rows in 16-row boxes
   CUtensorMap wqmap;        // NVFP4 records as [records][36][128 B] (see make_tmap_records)
   UmmaArgs args;
   int nt;                   // token rows per tile: 16, 64 or 256

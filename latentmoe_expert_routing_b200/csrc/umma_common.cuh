@@ -25,9 +25,10 @@ constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B cod
 // 64-K slices per pipeline step of the NVFP4 kernel: up to 4 dividing the
 // tile's K, and few enough that TMEM (512 columns) holds a W slot of 32*KS
 // columns per dequant group (two) next to the accumulators (wq_acc_cols: a
-// double-buffered pair, 2*nt columns, or for 16-/32-token tiles one pair per
-// MMA thread, two of them).  The host picks the record TMA box with the same rule.
-__host__ __device__ inline int wq_acc_cols(int nt) { return (nt <= 32 ? 4 : 2) * nt; }
+// double-buffered accumulator, 2*nt columns, or for 16-/32-token tiles one
+// accumulator per MMA thread, four of them, double-buffered for 16 tokens and
+// single for 32: 128 columns).  The host picks the record TMA box with the same rule.
+__host__ __device__ inline int wq_acc_cols(int nt) { return nt <= 32 ? 128 : 2 * nt; }
 __host__ __device__ inline int wq_slices_per_step(int kt_all, int nt) {
   int ks = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
   while (ks > 1 && (512 - wq_acc_cols(nt)) / (32 * ks) < 2) ks >>= 1;

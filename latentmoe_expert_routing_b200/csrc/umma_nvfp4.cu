@@ -5,31 +5,33 @@
 // records and are expanded to exact fp16 rows directly in tensor memory, from
 // where the MMA reads its A operand ("TS" form).
 //
-// A 64-K slice of NVFP4 weights is only 4.6 KB, and every tcgen05 instruction
-// holds its issuing thread for ~55 cycles (more on a busy SM), so a pipeline
-// step is a batch of KS = 4 slices (K = 256) and each MMA thread pays one wait
-// and one commit per step: the dequant warps wait for the step's activation
-// tile as well as its records, so the MMA threads wait only for "W ready", and
-// one commit per step frees the step's A slot and W slot together.  The
-// dequantised W tiles live in TMEM (slots of 32*KS columns next to the
-// accumulators), which leaves shared memory for the record batches (covering
-// HBM latency) and the activation tiles.  A slot is reused only after the
-// MMAs of the step before last that used it completed, so the pipeline depth
-// is the slot count: 16- and 32-token tiles keep two accumulator pairs (two
-// MMA threads) and three slots -- measured faster than four threads with two
-// slots, or two threads with six half-size slots.
+// A 64-K slice of NVFP4 weights is only 4.6 KB and each tcgen05.mma holds its
+// issuing thread ~123 cycles (measured, whatever the operands), so a pipeline
+// step is a batch of KS = 4 slices (K = 256) and 16- and 32-token tiles issue
+// from four threads (one per SM sub-partition, each into its own accumulator;
+// the 32-token tiles' accumulators are single-buffered and the epilogue
+// releases them as soon as it has read them into registers).  Each MMA thread
+// commits once per step, to the step's barrier done[step % NA], which frees
+// both the step's activation slot (ring of NA slots, reloaded NA steps later)
+// and its W slot (TMEM, ring of SW <= NA slots of 32*KS columns next to the
+// accumulators, rewritten SW steps later).  The activation ring is deeper than
+// the W ring so that a tile's load latency is off the critical path: the
+// producer runs NA steps ahead, and the dequant warps wait only for their
+// records and for the W slot.  Shared memory holds the record batches (covering
+// HBM latency) and the activation tiles.
 //
 // Warps (640 threads):
 //   0      record producer (3-D TMA, batches of up to four records)
 //   1      TMEM allocation, MMA issue (one lane)
 //   2      activation producer (TMA tiles into the A ring)
-//   3      16- and 32-token tiles: the second MMA issuer (16-K steps 2-3 of
-//          every slice into its own accumulator pair); otherwise idle
-//   4-7    epilogue group 0 (16-/32-token tiles: every chunk, summing the two
+//   3      16- and 32-token tiles: MMA issuer 1; otherwise idle
+//   4-7    epilogue group 0 (16-/32-token tiles: every chunk, summing the four
 //          accumulators; otherwise the even 8-column chunks)
 //   8-15   dequant: two groups of four warps (one per TMEM lane quarter) take
 //          alternate steps; each thread expands its weight row's slices
-//   16-19  epilogue group 1 (odd chunks) for 32-token and wider tiles
+//   16-19  16-/32-token tiles: warps 16 and 18 are MMA issuers 2 and 3 (issuer
+//          j takes the 16-K step j of every 64-K slice); otherwise epilogue
+//          group 1 (odd chunks)
 // Every wait is bounded; on timeout the kernel records DEV_ERR_TIMEOUT, unwinds,
 // waits for its own copies and MMAs and frees TMEM.
 //
@@ -53,15 +55,17 @@ namespace lmoe {
 
 constexpr int kMaxKS = 4;                    // 64-K slices per pipeline step
 
-template <int NT, int RAW>
+template <int NT, int RAW, int NA>
 struct WqSmem {
-  // 16- and 32-token tiles keep two accumulator pairs (two MMA threads)
-  static constexpr int kAccCols = (NT <= 32 ? 4 : 2) * NT;
+  // 16- and 32-token tiles: one accumulator per MMA thread (four), double-
+  // buffered for 16 tokens, single for 32; wider tiles: one, double-buffered
+  static constexpr int kAccBufs = NT == 32 ? 1 : 2;
+  static constexpr int kAccCols = (NT <= 32 ? 4 : 1) * kAccBufs * NT;
   static constexpr int kWCol0 = kAccCols;                              // W slots after the accumulators
   static constexpr int kMaxSW = (512 - kWCol0) / 32;                   // with one slice per step
   static constexpr int kATileBytes = NT * kBK * 2;                     // one 64-K slice, multiple of 1024
-  // one A slot per W slot: SW slots of KS tiles fit in kMaxSW tiles
-  static constexpr int kARegionBytes = kMaxSW * kATileBytes;
+  // the activation ring: NA slots of up to kMaxKS tiles
+  static constexpr int kARegionBytes = NA * kMaxKS * kATileBytes;
   static constexpr int kRawSlotBytes = kMaxKS * kWqRecordBytes;        // one step's records
   static constexpr int kRawOffset = kARegionBytes;
   static constexpr int kBarOffset = kRawOffset + RAW * kRawSlotBytes;
@@ -80,25 +84,26 @@ __device__ __forceinline__ int dq_group(int warp) {
 }
 
 // MMA thread index of a warp (lane 0 issues): warp 1, and for 16-/32-token tiles
-// warp 3 as well; -1 otherwise
+// warps 3, 16 and 18 as well (one issuer per SM sub-partition); -1 otherwise
 template <bool SPLIT>
 __device__ __forceinline__ int mma_thread(int warp) {
   if (warp == 1) return 0;
-  return (SPLIT && warp == 3) ? 1 : -1;
+  if (!SPLIT) return -1;
+  return warp == 3 ? 1 : warp == 16 ? 2 : warp == 18 ? 3 : -1;
 }
 
-template <int NT, int RAW, typename TO, bool RELU2, bool QA>
+template <int NT, int RAW, int NA, typename TO, bool RELU2, bool QA>
 __global__ void __launch_bounds__(kWqThreads, 1)
-umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wqmap,
-               const UmmaArgs a) {
-  using S = WqSmem<NT, RAW>;
+umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap amap16,
+               const __grid_constant__ CUtensorMap wqmap, const UmmaArgs a) {
+  using S = WqSmem<NT, RAW, NA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset); // A tiles of slot landed
-  uint64_t* w_ready = a_full + S::kMaxSW;                               // W slot written (TMEM)
-  uint64_t* slot_free = w_ready + S::kMaxSW;                            // slot's MMAs done
-  uint64_t* raw_full = slot_free + S::kMaxSW;                           // record batch landed
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + S::kBarOffset); // [NA] A tiles of slot landed
+  uint64_t* done = a_full + NA;                                         // [NA] a step's MMAs completed
+  uint64_t* w_ready = done + NA;                                        // W slot written (TMEM)
+  uint64_t* raw_full = w_ready + S::kMaxSW;                             // record batch landed
   uint64_t* raw_empty = raw_full + RAW;                                 // record batch consumed
   uint64_t* acc_full = raw_empty + RAW;                                 // [2]
   uint64_t* acc_empty = acc_full + 2;                                   // [2]
@@ -109,32 +114,38 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   int32_t* s_off = s_tiles + 1025;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // 16-/32-token tiles: two threads issue the MMAs (thread j the 16-K steps 2j and
-  // 2j+1 of every slice) into two accumulators that the epilogue adds; each
-  // tcgen05 instruction holds its issuing thread for ~55 cycles (more on a
-  // loaded SM), several times a 128 x 32 x 16 MMA's time on the tensor pipe
+  // 16-/32-token tiles: four threads issue the MMAs (thread j the 16-K step j
+  // of every slice) into four accumulators that the epilogue adds; each
+  // tcgen05.mma holds its issuing thread for ~123 cycles, many times a
+  // 128 x 32 x 16 MMA's time on the tensor pipe
   constexpr bool SPLIT = NT <= 32;
-  constexpr uint32_t NM = SPLIT ? 2 : 1;    // MMA threads
+  constexpr uint32_t NM = SPLIT ? 4 : 1;    // MMA threads
+  constexpr int NB = S::kAccBufs;           // accumulator buffers per thread
   constexpr int kEpiThreads = SPLIT ? 128 : 256;
   const int kt_all = a.K0 / kBK;
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
   // tile has a multiple of KS slices
   const int KS = wq_slices_per_step(kt_all, NT);
   const int nsteps = kt_all / KS;
-  const int SW = (512 - S::kWCol0) / (32 * KS);                        // W slots of 32*KS columns
+  // W slots of 32*KS columns, at most NA: step `it` completes barrier done[it % NA],
+  // which frees its A slot for step it + NA and its W slot for step it + SW
+  const int SW = min((512 - S::kWCol0) / (32 * KS), NA);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SW; ++s) {
+    for (int s = 0; s < NA; ++s) {
       mbar_init(&a_full[s], 1);
-      mbar_init(&w_ready[s], kDqGroupThreads);
-      mbar_init(&slot_free[s], NM);
+      mbar_init(&done[s], NM);
     }
-    for (int r = 0; r < RAW; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], kDqGroupThreads); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], NM); mbar_init(&acc_empty[b], kEpiThreads); }
+    // one arrival per warp (after __syncwarp): a barrier phase completes after
+    // 4 or 8 arrivals instead of 128 or 256 serialised shared-memory updates
+    for (int s = 0; s < SW; ++s) mbar_init(&w_ready[s], kDqGroupThreads / 32);
+    for (int r = 0; r < RAW; ++r) { mbar_init(&raw_full[r], 1); mbar_init(&raw_empty[r], kDqGroupThreads / 32); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], NM); mbar_init(&acc_empty[b], kEpiThreads / 32); }
     mbar_init(mma_done, NM);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&amap);
+    if (NT > 16) tma_prefetch_desc(&amap16);
     tma_prefetch_desc(&wqmap);
   }
   if (warp == 1) {
@@ -182,55 +193,59 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     // ---------------- activation producer ----------------
     if (lane == 0) {
       uint32_t it = 0, sa = 0, pa = 1;
-      const int slot_bytes = KS * S::kATileBytes;
+      const int slot_bytes = KS * S::kATileBytes;   // slot stride: tiles of one step
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
+        // the MMA reads the tile's first n_eff rows: a tile of at most 16 valid
+        // rows loads 16-row boxes (half or less of the bytes)
+        const bool short_tile = NT > 16 && ti.valid <= 16;
+        const CUtensorMap* map = short_tile ? &amap16 : &amap;
+        const uint32_t step_bytes = KS * (short_tile ? 16 * kBK * 2 : S::kATileBytes);
         for (int st = 0; st < nsteps; ++st, ++it) {
-          if (!mbar_wait(&slot_free[sa], pa)) { fail(13); ok = false; break; }
-          mbar_arrive_expect_tx(&a_full[sa], slot_bytes);
+          if (!mbar_wait(&done[sa], pa)) { fail(13); ok = false; break; }
+          mbar_arrive_expect_tx(&a_full[sa], step_bytes);
           uint8_t* dst = smem + sa * slot_bytes;
           for (int ks = 0; ks < KS; ++ks)
-            tma_load_2d(dst + ks * S::kATileBytes, &amap, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
-          if (++sa == (uint32_t)SW) { sa = 0; pa ^= 1; }
+            tma_load_2d(dst + ks * S::kATileBytes, map, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
+          if (++sa == (uint32_t)NA) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
       }
-      const uint32_t n = it < (uint32_t)SW ? it : (uint32_t)SW;
+      const uint32_t n = it < (uint32_t)NA ? it : (uint32_t)NA;
       for (uint32_t j = 0; j < n; ++j) {
         const uint32_t i = it - 1 - j;
-        if (!mbar_wait(&a_full[i % SW], (i / SW) & 1)) { fail(14); break; }
+        if (!mbar_wait(&a_full[i % NA], (i / NA) & 1)) { fail(14); break; }
       }
     }
   } else if (mma_thread<SPLIT>(warp) >= 0) {
     // ---------------- MMA issuer(s) (A from TMEM, B from shared memory) ----------------
-    const int j = mma_thread<SPLIT>(warp);    // SPLIT: 16-K steps 2j, 2j+1 of every slice
+    const int j = mma_thread<SPLIT>(warp);    // SPLIT: 16-K step j of every slice
     if (lane == 0) {
       const uint64_t bdesc0 = sw128_desc(smem_u32(smem));
       const uint32_t slot_desc = (uint32_t)((KS * S::kATileBytes) >> 4);
-      uint32_t s = 0, ps = 0, lt = 0;
+      uint32_t s = 0, ps = 0, sa = 0, pa = 0, lt = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
-        const uint32_t buf = lt & 1, use = lt >> 1;
+        const uint32_t buf = lt % NB, use = lt / NB;
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1)) { fail(15); break; }
         tc_fence_after();
-        const uint32_t d = tmem + (2 * j + buf) * NT;
+        const uint32_t d = tmem + (j * NB + buf) * NT;
         // ragged tiles multiply only their valid rows, rounded up to N granularity 16
         const int n_eff = min(NT, (ti.valid + 15) & ~15);
         const uint32_t idesc = idesc_f16_f32(kBM, n_eff);
         bool ok = true;
         for (int st = 0; st < nsteps; ++st) {
-          // W ready implies the step's A tiles landed (the dequant warps waited for them)
-          if (!mbar_wait(&w_ready[s], ps)) { fail(16); ok = false; break; }
+          // the step's A tiles (normally landed long before) and its W slot
+          if (!mbar_wait(&a_full[sa], pa) || !mbar_wait(&w_ready[s], ps)) { fail(16); ok = false; break; }
           tc_fence_after();
           uint32_t wt = tmem + S::kWCol0 + s * 32 * KS;
-          uint64_t bd = bdesc0 + (uint64_t)(s * slot_desc);
+          uint64_t bd = bdesc0 + (uint64_t)(sa * slot_desc);
           for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
             if (SPLIT) {
-              mma_bf16_ts(d, wt + 16 * j, bd + 4 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
-              mma_bf16_ts(d, wt + 16 * j + 8, bd + 4 * j + 2, idesc, 1u);
+              mma_bf16_ts(d, wt + 8 * j, bd + 2 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
             } else {
               mma_bf16_ts(d, wt, bd, idesc, (st > 0 || ks > 0) ? 1u : 0u);
               mma_bf16_ts(d, wt + 8, bd + 2, idesc, 1u);
@@ -238,8 +253,9 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
               mma_bf16_ts(d, wt + 24, bd + 6, idesc, 1u);
             }
           }
-          mma_commit(&slot_free[s]);          // A and W slot free once these MMAs finish
+          mma_commit(&done[sa]);              // A slot (and W slot) free once these MMAs finish
           if (++s == (uint32_t)SW) { s = 0; ps ^= 1; }
+          if (++sa == (uint32_t)NA) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
         mma_commit(&acc_full[buf]);
@@ -261,10 +277,17 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       for (int st = 0; st < nsteps; ++st, ++it) {
         if ((int)(it % kDqGroups) != g) continue;
         const int sw = it % SW, rr = it % RAW;
-        const uint32_t ph = (it / SW) & 1;
-        if (!mbar_wait_sleep(&raw_full[rr], (it / RAW) & 1) ||
-            !mbar_wait_sleep(&slot_free[sw], ph ^ 1) ||
-            !mbar_wait_sleep(&a_full[sw], ph)) { fail(18); ok = false; break; }
+        // the W slot's previous step (it - SW) must have completed its MMAs; its
+        // barrier cannot have moved on (step it - SW + NA >= it needs this W)
+        const uint32_t prev = it - SW;
+        // the warp leaves together (its lanes meet at __syncwarp below)
+        const bool w_ok = mbar_wait_sleep(&raw_full[rr], (it / RAW) & 1) &&
+                          (it < (uint32_t)SW || mbar_wait_sleep(&done[prev % NA], (prev / NA) & 1));
+        if (!__all_sync(0xffffffffu, w_ok)) {
+          if (!w_ok) fail(18);
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint8_t* rec = smem + S::kRawOffset + rr * S::kRawSlotBytes;
         for (int ks = 0; ks < KS; ++ks) {
@@ -274,8 +297,11 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&raw_empty[rr]);
-        mbar_arrive(&w_ready[sw]);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&raw_empty[rr]);
+          mbar_arrive(&w_ready[sw]);
+        }
       }
       if (!ok) break;
     }
@@ -284,14 +310,17 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     // 16-/32-token tiles: group 0 alone) ----------------
     const int q = warp & 3;
     const int grp = warp >= 16 ? 1 : 0;
-    constexpr int kChunkStep = SPLIT ? 1 : 2;
     TO* out = reinterpret_cast<TO*>(a.out);
     uint32_t lt = 0;
     for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
       TileInfo ti;
       if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
-      const uint32_t buf = lt & 1, use = lt >> 1;
-      if (!mbar_wait_sleep(&acc_full[buf], use & 1)) { fail(19); break; }
+      const uint32_t buf = lt % NB, use = lt / NB;
+      const bool w_ok = mbar_wait_sleep(&acc_full[buf], use & 1);
+      if (!__all_sync(0xffffffffu, w_ok)) {   // the warp leaves together
+        if (!w_ok) fail(19);
+        break;
+      }
       tc_fence_after();
       const int n = ti.n0 + 32 * q + lane;
       const bool col_ok = n < a.n_out;
@@ -300,20 +329,12 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
       float gs = a.gscale ? a.gscale[ti.wgrp] * 0x1p-26f : 1.f;
       if (a.act_gscale) gs = __fmul_rn(gs, *a.act_gscale);
       if (a.acc_mul != 0.f) gs = __fmul_rn(gs, a.acc_mul);
-      for (int c = grp; c < NT / 8; c += kChunkStep) {
-        if (c * 8 >= ti.valid) break;        // uniform: no valid rows left
-        const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;
-        uint32_t r0[8], r1[8];
-        tmem_ld8(row_base + buf * NT, r0);
-        if (SPLIT) tmem_ld8(row_base + (2 + buf) * NT, r1);
-        tmem_ld_wait();
+      // one 8-column chunk (token rows c*8 .. c*8+7 of output column n)
+      auto emit = [&](const float (&acc8)[8], int c) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          // the two partial sums (16-K steps 0-1 and 2-3 of every slice)
-          const float acc = SPLIT ? __fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]))
-                                  : __uint_as_float(r0[j]);
-          v[j] = __fmul_rn(acc, gs);
+          v[j] = __fmul_rn(acc8[j], gs);
           if (RELU2) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
         }
@@ -340,9 +361,46 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
           }
         }
+      };
+      if constexpr (SPLIT) {
+        // read the four partial sums (16-K step t of every slice in accumulator
+        // t) of the valid chunks, release the accumulators, then finish
+        float acc[NT / 8][8];
+#pragma unroll
+        for (int c = 0; c < NT / 8; ++c) {
+          if (c * 8 < ti.valid) {            // uniform across the warp
+            const uint32_t row_base = tmem + ((uint32_t)(32 * q) << 16) + c * 8;
+            uint32_t r[4][8];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) tmem_ld8(row_base + (t * NB + buf) * NT, r[t]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              acc[c][j] = __fadd_rn(__fadd_rn(__uint_as_float(r[0][j]), __uint_as_float(r[1][j])),
+                                    __fadd_rn(__uint_as_float(r[2][j]), __uint_as_float(r[3][j])));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int c = 0; c < NT / 8; ++c)
+          if (c * 8 < ti.valid) emit(acc[c], c);
+      } else {
+        for (int c = grp; c < NT / 8; c += 2) {
+          if (c * 8 >= ti.valid) break;      // uniform: no valid rows left
+          uint32_t r0[8];
+          tmem_ld8(tmem + ((uint32_t)(32 * q) << 16) + c * 8 + buf * NT, r0);
+          tmem_ld_wait();
+          float acc8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc8[j] = __uint_as_float(r0[j]);
+          emit(acc8, c);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
       ++lt;
     }
   }
@@ -354,16 +412,16 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   }
 }
 
-template <int NT, int RAW, typename TO, bool RELU2, bool QA>
+template <int NT, int RAW, int NA, typename TO, bool RELU2, bool QA>
 static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
-  using S = WqSmem<NT, RAW>;
+  using S = WqSmem<NT, RAW, NA>;
   static_assert(S::kBytes <= 232448, "shared memory budget");
   // dequant groups work on up to kDqGroups steps at once: each ring needs at
   // least that many slots, or a waiter could target a phase two ahead (parity
   // alias); wq_slices_per_step keeps at least two W slots
-  static_assert(S::kMaxSW >= kDqGroups && RAW >= kDqGroups, "ring too shallow for the dequant groups");
-  static_assert(3 * S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
-  auto kern = umma_wq_kernel<NT, RAW, TO, RELU2, QA>;
+  static_assert(NA >= kDqGroups && RAW >= kDqGroups, "ring too shallow for the dequant groups");
+  static_assert(2 * NA + S::kMaxSW + 2 * RAW + 5 + 2 <= 128, "barrier region");
+  auto kern = umma_wq_kernel<NT, RAW, NA, TO, RELU2, QA>;
   static int configured = 0, sms = 0;
   if (!configured) {
     int dev = 0;
@@ -375,16 +433,16 @@ static cudaError_t wq_launch_t(const UmmaLaunch& L, cudaStream_t st) {
   }
   int grid = L.max_tiles < sms ? L.max_tiles : sms;
   if (grid < 1) grid = 1;
-  kern<<<grid, kWqThreads, S::kBytes, st>>>(L.amap0, L.wqmap, L.args);
+  kern<<<grid, kWqThreads, S::kBytes, st>>>(L.amap0, L.amap1, L.wqmap, L.args);
   return cudaGetLastError();
 }
 
-template <int NT, int RAW>
+template <int NT, int RAW, int NA>
 static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
   switch (L.epi) {
-    case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, RAW, __half, true, true>(L, st);    // W4A4 up
-    case UMMA_EPI_F16_RELU2: return wq_launch_t<NT, RAW, __half, true, false>(L, st);     // W4A16 up
-    case UMMA_EPI_F32: return wq_launch_t<NT, RAW, float, false, false>(L, st);           // down
+    case UMMA_EPI_F16_RELU2_Q: return wq_launch_t<NT, RAW, NA, __half, true, true>(L, st);    // W4A4 up
+    case UMMA_EPI_F16_RELU2: return wq_launch_t<NT, RAW, NA, __half, true, false>(L, st);     // W4A16 up
+    case UMMA_EPI_F32: return wq_launch_t<NT, RAW, NA, float, false, false>(L, st);           // down
     default: return cudaErrorInvalidValue;
   }
 }
@@ -392,10 +450,11 @@ static cudaError_t wq_launch_nt(const UmmaLaunch& L, cudaStream_t st) {
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st) {
   if (L.args.K1 != 0 || !L.args.wq) return cudaErrorInvalidValue;
   switch (L.nt) {
-    case 16: return wq_launch_nt<16, 9>(L, st);             // A 24 KB + records 166 KB
-    case 32: return wq_launch_nt<32, 9>(L, st);             // A 32 KB + records 166 KB
-    case 64: return wq_launch_nt<64, 6>(L, st);             // A 96 KB + records 110 KB
-    case 128: return wq_launch_nt<128, 4>(L, st);           // A 128 KB + records 74 KB
+    // <tile tokens, record batches, activation slots>
+    case 16: return wq_launch_nt<16, 9, 6>(L, st);          // A 48 KB + records 166 KB
+    case 32: return wq_launch_nt<32, 7, 5>(L, st);          // A 80 KB + records 129 KB
+    case 64: return wq_launch_nt<64, 6, 3>(L, st);          // A 96 KB + records 110 KB
+    case 128: return wq_launch_nt<128, 4, 2>(L, st);        // A 128 KB + records 74 KB
   }
   return cudaErrorInvalidValue;
 }
