@@ -119,9 +119,10 @@ typedef struct {
  * which moe_init quantises (moe_quantize_nvfp4's arithmetic) and does not
  * keep, OR the pre-quantised tensors below with w_up = w_down = NULL, as an
  * NVFP4 checkpoint ships them:
- *   codes  [E, rows, K/2]  E2M1, two per byte, the even element in the low nibble
- *   scales [E, rows, K/16] E4M3 block scales, one per 16 consecutive elements along K
- *   gscale [E]             fp32 global scale of each expert matrix
+ *   codes  [E, rows, K/2]        E2M1, two per byte, the even element in the low nibble
+ *   scales [E, rows, ceil(K/16)] E4M3 block scales, one per 16 consecutive elements
+ *                                along K (a row with K % 16 == 8 ends in a block of 8)
+ *   gscale [E]                   fp32 global scale of each expert matrix
  * with (rows, K) = (F, L) for up and (L, F) for down; a weight is
  * value(code) * value(scale) * gscale.  moe_init repacks them into its own
  * layouts; the caller may free them once moe_init returns.  NaN scales (E4M3
@@ -137,10 +138,10 @@ typedef struct {
   const void* w_down;          /* [E, L, F] dtype, or NULL (pre-quantised)    */
   int borrow;
   const uint8_t* up_codes;     /* [E, F, L/2]   pre-quantised NVFP4, or NULL  */
-  const uint8_t* up_scales;    /* [E, F, L/16]                                */
+  const uint8_t* up_scales;    /* [E, F, L/16] (L is a multiple of 64)        */
   const float* up_gscale;      /* [E]                                         */
   const uint8_t* down_codes;   /* [E, L, F/2]                                 */
-  const uint8_t* down_scales;  /* [E, L, F/16]                                */
+  const uint8_t* down_scales;  /* [E, L, ceil(F/16)]                          */
   const float* down_gscale;    /* [E]                                         */
   int weights_on_device;       /* 1: device pointers; 0: host pointers        */
 } moe_weights;
@@ -328,7 +329,9 @@ moe_status moe_route_noalloc(const void* hidden, const void* w_gate,
  *   codes            = E2M1(w / (value(scale) * gscale[m])) RNE ties-to-even, sat. at 6
  * with fp32 arithmetic before each encoding.  Outputs (device): codes
  * [n_mat, rows, K/2] two per byte, the even element in the low nibble;
- * scales [n_mat, rows, K/16]; gscale [n_mat].  K must be a multiple of 16.
+ * scales [n_mat, rows, ceil(K/16)]; gscale [n_mat].  K must be a multiple of
+ * 8; with K % 16 == 8 each row ends in a block of 8 elements, quantised like a
+ * full block whose other 8 elements are zero.
  * Uses a small temporary device buffer; synchronises `stream`.  moe_init runs
  * the same quantiser on the experts of NVFP4 layers. */
 moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int rows, int K,

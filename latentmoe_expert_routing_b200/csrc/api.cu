@@ -251,34 +251,39 @@ struct TempBuf {
 moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s) {
   const moe_config& c = h->cfg;
   const size_t E = h->e_loc, F = c.d_ff, L = c.d_latent;     // the experts this layer holds
-  const size_t recs_up = E * ((F + 127) / 128) * (L / 64), recs_dn = E * ((L + 127) / 128) * (F / 64);
+  const size_t recs_up = E * ((F + 127) / 128) * wq_kslices((int)L),
+               recs_dn = E * ((L + 127) / 128) * wq_kslices((int)F);
   if (!dev_alloc(h, &h->rec_up, recs_up * 4608) || !dev_alloc(h, &h->rec_dn, recs_dn * 4608) ||
       !dev_alloc(h, &h->gs_up, E * 4) || !dev_alloc(h, &h->gs_dn, E * 4))
     return MOE_ERR_OOM;
   const size_t n = E * F * L;
+  // scale bytes: one per 16 elements along K, a partial block at the end of a row
+  const size_t ns_up = E * F * ((L + 15) / 16), ns_dn = E * L * ((F + 15) / 16);
+  const size_t ns = ns_up > ns_dn ? ns_up : ns_dn;
   const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
   const bool pre = w->up_codes != nullptr;
   const bool dev = w->weights_on_device != 0;
   TempBuf codes, scales, dense, amax;
   if (w4a4) {                // kept: the block-scaled FP4 GEMMs read the plain layout
-    if (!dev_alloc(h, &h->wc_up, n / 2) || !dev_alloc(h, &h->ws_up, n / 16) ||
-        !dev_alloc(h, &h->wc_dn, n / 2) || !dev_alloc(h, &h->ws_dn, n / 16))
+    if (!dev_alloc(h, &h->wc_up, n / 2) || !dev_alloc(h, &h->ws_up, ns_up) ||
+        !dev_alloc(h, &h->wc_dn, n / 2) || !dev_alloc(h, &h->ws_dn, ns_dn))
       return MOE_ERR_OOM;
-  } else if (!(pre && dev) && (!codes.alloc(n / 2) || !scales.alloc(n / 16))) {
+  } else if (!(pre && dev) && (!codes.alloc(n / 2) || !scales.alloc(ns))) {
     return MOE_ERR_OOM;
   }
   if (!pre && (!amax.alloc(E * 4) || (!dev && !dense.alloc(n * 2)))) return MOE_ERR_OOM;
   struct Proj {
     int rows, K;
+    size_t nscales;
     const void* dense;
     const uint8_t *codes, *scales;
     const float* gs_src;
     uint8_t *keep_c, *keep_s, *rec;
     float* gs;
   } proj[2] = {
-      {(int)F, (int)L, w->w_up, w->up_codes, w->up_scales, w->up_gscale, h->wc_up, h->ws_up,
-       h->rec_up, h->gs_up},
-      {(int)L, (int)F, w->w_down, w->down_codes, w->down_scales, w->down_gscale, h->wc_dn,
+      {(int)F, (int)L, ns_up, w->w_up, w->up_codes, w->up_scales, w->up_gscale, h->wc_up,
+       h->ws_up, h->rec_up, h->gs_up},
+      {(int)L, (int)F, ns_dn, w->w_down, w->down_codes, w->down_scales, w->down_gscale, h->wc_dn,
        h->ws_dn, h->rec_dn, h->gs_dn}};
   cudaError_t e = cudaSuccess;
   for (const Proj& q : proj) {
@@ -289,7 +294,7 @@ moe_status quantize_experts(moe_handle* h, const moe_weights* w, cudaStream_t s)
     if (pre) {
       if (cu != q.codes) e = cudaMemcpyAsync(cu, q.codes, n / 2, cudaMemcpyDefault, s);
       if (e == cudaSuccess && su != q.scales)
-        e = cudaMemcpyAsync(su, q.scales, n / 16, cudaMemcpyDefault, s);
+        e = cudaMemcpyAsync(su, q.scales, q.nscales, cudaMemcpyDefault, s);
       if (e == cudaSuccess) e = cudaMemcpyAsync(q.gs, q.gs_src, E * 4, cudaMemcpyDefault, s);
     } else {
       const void* src = q.dense;
@@ -490,7 +495,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     // and write relu^2 scaled by 2^-8 (relu^2(v 2^-4) = relu^2(v) 2^-8) into fp16 H
     u.args.act_gscale = w4a4 ? (dyn ? h->act_gs : nullptr) : h->zp2 + 1;
     u.args.acc_mul = w4a4 ? 0.f : 0x1p-4f;
-    u.wqmap = h->rm_up[batch_idx(L / 64)];
+    u.wqmap = h->rm_up[batch_idx(wq_kslices(L))];
   }
   const bool pg = grouped_pair(c, P);     // SM pairs: 256-row weight blocks, half-token boxes
   if (pg) u.amap0 = h->am_zp[3];
@@ -504,7 +509,7 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     u.args.wq = h->rec_dn; u.args.wq_mblks = ceil_div(L, 128); u.args.gscale = h->gs_dn;
     u.args.act_gscale = nullptr;
     u.args.acc_mul = w4a4 ? 0.f : 0x1p8f;         // W4A16: H was stored times 2^-8
-    u.wqmap = h->rm_dn[batch_idx(F / 64)];
+    u.wqmap = h->rm_dn[batch_idx(wq_kslices(F))];
   }
   u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
   if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -652,10 +657,9 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
   if (c.dtype == MOE_BF16) {
     // tensor-core tiles: d_model and d_latent in whole 64-wide K steps (a GEMM's
     // first K segment and the exact-logit order); the expert and shared widths
-    // may end in a partial step (zero-filled TMA boxes, masked output columns),
-    // except for NVFP4 experts, whose records hold whole 64-wide slices
-    if (c.d_model % 64 || c.d_latent % 64 ||
-        (c.expert_fmt != MOE_EXPERT_DENSE && c.d_ff % 64)) {
+    // may end in a partial step (zero-filled TMA boxes, masked output columns;
+    // NVFP4 records past the width hold zero codes and scales)
+    if (c.d_model % 64 || c.d_latent % 64) {
       moe_destroy(h);
       return MOE_ERR_UNSUPPORTED;
     }
@@ -1022,7 +1026,7 @@ moe_status moe_profile_read(moe_handle* h, float* stage_ms, int n) {
 
 moe_status moe_quantize_nvfp4(const void* w, moe_dtype dtype, int n_mat, int rows, int K,
                               uint8_t* codes, uint8_t* scales, float* gscale, void* stream) {
-  if (!w || !codes || !scales || !gscale || n_mat <= 0 || rows <= 0 || K <= 0 || K % 16)
+  if (!w || !codes || !scales || !gscale || n_mat <= 0 || rows <= 0 || K <= 0 || K % 8)
     return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_BF16 && dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;

@@ -4,11 +4,14 @@
 // q = E2M1(w / (value(s_b) * s_g)); all arithmetic before the encodings in fp32.
 //
 // Plain layout (C ABI): codes [n_mat, rows, K/2] (two per byte, even element in
-// the low nibble), scales [n_mat, rows, K/16], gscale [n_mat].
+// the low nibble), scales [n_mat, rows, ceil(K/16)], gscale [n_mat].  K is a
+// multiple of 8; a row with K % 16 == 8 ends in a partial block of 8 elements,
+// quantised like a full block whose missing elements are zero.
 // GEMM layout (library internal): per (matrix, 128-row block, 64-K stage) one
 // contiguous 4608-byte record: codes as [half 0..1][row 0..127][16 bytes] (row r's
 // elements 32h..32h+31 at h*2048 + r*16), then 128 rows x 4 scale bytes; rows
-// past the matrix are zero.  The codes keep the plain byte order (element 2i in
+// past the matrix, and elements and blocks past K, are zero, and each block of
+// 128 rows has wq_kslices(K) records (a multiple of four).  The codes keep the plain byte order (element 2i in
 // the low nibble of byte i), which the hardware E2M1 -> f16x2 conversion reads
 // directly.
 #include <cuda_fp16.h>
@@ -16,6 +19,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "nvfp4.cuh"
+#include "umma_common.cuh"
 
 namespace lmoe {
 
@@ -42,20 +46,27 @@ __global__ void global_scale_kernel(const unsigned* __restrict__ amax, float* __
   if (i < n) gscale[i] = __fdiv_rn(__uint_as_float(amax[i]), 2688.0f);   // 6 * 448
 }
 
-// One thread per 16-element block.
+// One thread per 16-element block (the last block of a row may hold 8).
 template <typename T>
 __global__ void quantize_blocks_kernel(const T* __restrict__ w, int n_mat, int rows, int K,
                                        const float* __restrict__ gscale,
                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  const long nb = (long)n_mat * rows * (K / 16);
+  const int KB = (K + 15) / 16;                     // blocks per row
+  const long nb = (long)n_mat * rows * KB;
   const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= nb) return;
-  const int m = (int)(b / ((long)rows * (K / 16)));
+  const long row = b / KB;                          // over all matrices
+  const int kb = (int)(b - row * KB);
+  const int m = (int)(row / rows);
+  const int n = min(16, K - 16 * kb);               // 16, or 8 at the end of a row
   const float sg = gscale[m];
-  const T* p = w + b * 16;
+  const T* p = w + row * K + 16 * kb;
   float v[16], amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) { v[i] = to_f(p[i]); amax = fmaxf(amax, fabsf(v[i])); }
+  for (int i = 0; i < 16; ++i) {
+    v[i] = i < n ? to_f(p[i]) : 0.f;
+    amax = fmaxf(amax, fabsf(v[i]));
+  }
   const float den = __fmul_rn(6.0f, sg);
   const float ratio = den > 0.f ? __fdiv_rn(amax, den) : 0.f;
   const uint32_t sb = e4m3_encode_pos(ratio);
@@ -66,14 +77,18 @@ __global__ void quantize_blocks_kernel(const T* __restrict__ w, int n_mat, int r
     const uint32_t q = scale > 0.f ? e2m1_encode(__fdiv_rn(v[i], scale)) : 0u;
     if (i < 8) lo |= q << (4 * i); else hi |= q << (4 * (i - 8));
   }
-  *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(lo, hi);
+  // rows hold K/2 code bytes (a multiple of 4): 32-bit stores
+  uint32_t* cp = reinterpret_cast<uint32_t*>(codes + row * (K / 2) + 8 * kb);
+  cp[0] = lo;
+  if (n == 16) cp[1] = hi;
   scales[b] = (uint8_t)sb;
 }
 
 // plain layout -> GEMM layout
 __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                                    int n_mat, int rows, int K, uint8_t* __restrict__ out) {
-  const int nmb = (rows + 127) / 128, nks = K / 64;
+  const int nmb = (rows + 127) / 128, nks = wq_kslices(K);
+  const int KB = (K + 15) / 16, row_bytes = K / 2;
   const long rec = (long)blockIdx.x;                 // one record per block, 128 threads = rows
   if (rec >= (long)n_mat * nmb * nks) return;
   const int ks = (int)(rec % nks);
@@ -85,9 +100,12 @@ __global__ void repack_gemm_kernel(const uint8_t* __restrict__ codes, const uint
   uint32_t wd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   uint32_t s = 0;
   if (row < rows) {
-    const uint8_t* cp = codes + ((size_t)m * rows + row) * (K / 2) + ks * 32;
-    for (int i = 0; i < 8; ++i) wd[i] = *reinterpret_cast<const uint32_t*>(cp + 4 * i);
-    s = *reinterpret_cast<const uint32_t*>(scales + ((size_t)m * rows + row) * (K / 16) + ks * 4);
+    const uint8_t* cp = codes + ((size_t)m * rows + row) * row_bytes + ks * 32;
+    for (int i = 0; i < 8; ++i)
+      if (ks * 32 + 4 * i < row_bytes) wd[i] = *reinterpret_cast<const uint32_t*>(cp + 4 * i);
+    const uint8_t* sp = scales + ((size_t)m * rows + row) * KB + ks * 4;
+    for (int i = 0; i < 4; ++i)
+      if (ks * 4 + i < KB) s |= (uint32_t)sp[i] << (8 * i);
   }
   *reinterpret_cast<uint4*>(o + r * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
   *reinterpret_cast<uint4*>(o + 2048 + r * 16) = make_uint4(wd[4], wd[5], wd[6], wd[7]);
@@ -101,7 +119,7 @@ cudaError_t launch_quantize_nvfp4(const void* w, moe_dtype dt, int n_mat, int ro
   cudaError_t e = cudaMemsetAsync(amax_tmp, 0, sizeof(unsigned) * n_mat, st);
   if (e != cudaSuccess) return e;
   dim3 g1(ceil_div(per_mat, 256 * 16) < 1024 ? ceil_div(per_mat, 256 * 16) : 1024, n_mat);
-  const long nb = (long)n_mat * rows * (K / 16);
+  const long nb = (long)n_mat * rows * ((K + 15) / 16);
   if (dt == MOE_BF16) {
     matrix_amax_kernel<<<g1, 256, 0, st>>>((const __nv_bfloat16*)w, per_mat, amax_tmp);
     global_scale_kernel<<<ceil_div(n_mat, 256), 256, 0, st>>>(amax_tmp, gscale, n_mat);
@@ -130,7 +148,7 @@ cudaError_t launch_gemm_gscale(const float* gs, float* out, int n, cudaStream_t 
 
 cudaError_t launch_repack_gemm(const uint8_t* codes, const uint8_t* scales, int n_mat, int rows,
                                int K, uint8_t* out, cudaStream_t st) {
-  const long recs = (long)n_mat * ((rows + 127) / 128) * (K / 64);
+  const long recs = (long)n_mat * ((rows + 127) / 128) * wq_kslices(K);
   repack_gemm_kernel<<<(unsigned)recs, 128, 0, st>>>(codes, scales, n_mat, rows, K, out);
   return cudaGetLastError();
 }

@@ -29,6 +29,11 @@ constexpr int kWqRecordBytes = 4608;      // NVFP4 weight record: 128 x 32 B cod
 // accumulator per MMA thread, four of them, double-buffered for 16 tokens and
 // single for 32: 128 columns).  The host picks the record TMA box with the same rule.
 __host__ __device__ inline int wq_acc_cols(int nt) { return nt <= 32 ? 128 : 2 * nt; }
+// 64-K slices (records) per 128-row block of an NVFP4 matrix with K columns:
+// ceil(K / 64) rounded up to a multiple of 4, so that a pipeline step always
+// takes four slices; the slices past K hold zero codes and scales (the
+// activation tiles there are the TMA's zero fill)
+__host__ __device__ inline int wq_kslices(int K) { return (((K + 63) / 64) + 3) & ~3; }
 __host__ __device__ inline int wq_slices_per_step(int kt_all, int nt) {
   int ks = (kt_all % 4 == 0) ? 4 : (kt_all % 2 == 0 ? 2 : 1);
   while (ks > 1 && (512 - wq_acc_cols(nt)) / (32 * ks) < 2) ks >>= 1;

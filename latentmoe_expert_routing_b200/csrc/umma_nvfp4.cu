@@ -122,7 +122,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
   constexpr uint32_t NM = SPLIT ? 4 : 1;    // MMA threads
   constexpr int NB = S::kAccBufs;           // accumulator buffers per thread
   constexpr int kEpiThreads = SPLIT ? 128 : 256;
-  const int kt_all = a.K0 / kBK;
+  const int kt_all = wq_kslices(a.K0);       // records per 128-row block
   // a step is KS consecutive 64-K slices (one record batch, one TMA); every
   // tile has a multiple of KS slices
   const int KS = wq_slices_per_step(kt_all, NT);

@@ -312,16 +312,21 @@ def nvfp4_global_scale(w: np.ndarray) -> np.float32:
 
 
 def nvfp4_quantize(w: np.ndarray, s_g) -> tuple:
-    """Quantise w[rows, K] (K % 16 == 0) in 16-element blocks along K.
+    """Quantise w[rows, K] in 16-element blocks along K.
 
     Per block: s_b = E4M3(amax_b / (6 * s_g)); scale = value(s_b) * s_g;
     q_i = E2M1(w_i / scale) (0 when scale == 0).  All arithmetic before the
-    encodings is fp32 (IEEE division).  Returns (codes uint8 [rows, K] one code
-    per element, scales uint8 [rows, K/16])."""
+    encodings is fp32 (IEEE division).  A row whose length is not a multiple of
+    16 ends in a partial block: it is quantised like a full block whose missing
+    elements are zero (they change neither its maximum nor its other codes).
+    Returns (codes uint8 [rows, K] one code per element, scales uint8
+    [rows, ceil(K/16)])."""
     w = np.asarray(w, dtype=np.float32)
     rows, K = w.shape
-    assert K % 16 == 0
-    blk = w.reshape(rows, K // 16, 16)
+    nb = -(-K // 16)
+    if K % 16:
+        w = np.concatenate([w, np.zeros((rows, nb * 16 - K), np.float32)], axis=1)
+    blk = w.reshape(rows, nb, 16)
     amax = np.max(np.abs(blk), axis=-1).astype(np.float32)
     den = np.float32(np.float32(6.0) * np.float32(s_g))
     with np.errstate(divide="ignore", invalid="ignore"):
@@ -331,15 +336,16 @@ def nvfp4_quantize(w: np.ndarray, s_g) -> tuple:
     with np.errstate(divide="ignore", invalid="ignore"):
         y = np.where(scale[..., None] > 0, blk / scale[..., None],
                      np.float32(0)).astype(np.float32)
-    q = e2m1_encode_vec(y).reshape(rows, K)
+    q = e2m1_encode_vec(y).reshape(rows, nb * 16)[:, :K]
     return q, sb
 
 
 def nvfp4_dequantize(codes: np.ndarray, scales: np.ndarray, s_g) -> np.ndarray:
-    """fp64 values q * value(s_b) * s_g (exact: each product fits in fp64)."""
+    """fp64 values q * value(s_b) * s_g (exact: each product fits in fp64);
+    element k takes the scale of block k // 16."""
     rows, K = codes.shape
-    q = E2M1_TABLE[codes].reshape(rows, K // 16, 16)
-    return (q * E4M3_TABLE[scales][..., None] * float(s_g)).reshape(rows, K)
+    blk_of_k = np.arange(K) // 16
+    return E2M1_TABLE[codes] * E4M3_TABLE[scales][:, blk_of_k] * float(s_g)
 
 
 def nvfp4_roundtrip_activation(a: np.ndarray, s_g=np.float32(1.0)) -> np.ndarray:

@@ -27,7 +27,8 @@ def L():
 
 def _prequantised(w):
     """The oracle's NVFP4 quantisation of dense experts [E, rows, K], in the
-    ABI's plain layout: codes [E, rows, K/2], scales [E, rows, K/16], gscale [E]."""
+    ABI's plain layout: codes [E, rows, K/2], scales [E, rows, ceil(K/16)],
+    gscale [E]."""
     w = w.float().cpu().numpy()
     codes, scales, gs = [], [], []
     for m in w:
@@ -55,10 +56,13 @@ def _same(a, b):
         assert torch.equal(u.view(torch.int32), v.view(torch.int32))
 
 
-@pytest.mark.parametrize("fmt,T", [("w4a16", 3), ("w4a16", 200), ("w4a4", 64),
-                                   ("w4a4", 600), ("w4a4", 1200)])
-def test_prequantised_nvfp4_equals_quantise_at_init(L, fmt, T):
-    cfg = MID.replace(expert_fmt=fmt)
+@pytest.mark.parametrize("fmt,T,F", [("w4a16", 3, 512), ("w4a16", 200, 512), ("w4a4", 64, 512),
+                                     ("w4a4", 600, 512), ("w4a4", 1200, 512),
+                                     ("w4a16", 64, 328), ("w4a4", 600, 328)])
+def test_prequantised_nvfp4_equals_quantise_at_init(L, fmt, T, F):
+    """F = 328 ends each down-projection row in a block of 8: its scales are
+    [E, L, ceil(F/16)]."""
+    cfg = MID.replace(expert_fmt=fmt, F=F)
     W = L.weights_for(cfg)
     ref = _run(L, cfg, W, T)
     uc, us, ug = _prequantised(W["w_up"])

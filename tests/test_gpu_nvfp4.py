@@ -30,7 +30,7 @@ def _gpu_quantize(w):
     from latentmoe_expert_routing_b200 import binding as B
     n, rows, K = w.shape
     codes = torch.empty(n, rows, K // 2, dtype=torch.uint8, device="cuda")
-    scales = torch.empty(n, rows, K // 16, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(n, rows, (K + 15) // 16, dtype=torch.uint8, device="cuda")
     gs = torch.empty(n, dtype=torch.float32, device="cuda")
     dt = B.MOE_BF16 if w.dtype == torch.bfloat16 else B.MOE_FP32
     B.moe_quantize_nvfp4(w.data_ptr(), dt, n, rows, K, codes.data_ptr(), scales.data_ptr(),
@@ -48,10 +48,14 @@ def test_hardware_conversions_match_format(L):
     assert B.moe_selftest_nvfp4_convert(torch.cuda.current_stream().cuda_stream) == 0
 
 
+@pytest.mark.parametrize("K", [320, 328])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_quantizer_bit_exact(L, dtype):
+def test_quantizer_bit_exact(L, dtype, K):
+    """K = 328 ends every row in a block of 8 elements."""
     g = torch.Generator().manual_seed(3)
-    w = (torch.randn(4, 192, 320, generator=g) * 0.05)
+    w = (torch.randn(4, 192, K, generator=g) * 0.05)
+    w[0, 7, -8:] = 0.0                                   # an all-zero partial block
+    w[1, 9, -8:] = torch.tensor([6.0, -3.0, 1.5, 0.5, 0.0, 2.0, -4.0, 1.0]) * 0.01
     w[0, 0, :16] = 0.0                                   # all-zero block
     w[1, 3, :16] = torch.tensor([6.0, 3.0, 2.5, 1.75, 1.25, 0.75, 0.25, -5.0,
                                  -3.5, 0.5, 1.0, 1.5, 2.0, 4.0, -6.0, 0.0]) * 0.01
@@ -93,6 +97,23 @@ def test_nvfp4_mid_layer(L, fmt, T):
     expert leaves the second CTA without valid rows."""
     cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt=fmt, E=16, k=4, D=512,
                                          L=256, F=512, Fs=512)
+    lay, g, r = _run_full(L, cfg, T)
+    _assert_routing_exact(g, r)
+    rel, nmax, raw = out_metrics(g[0], r["out"])
+    assert rel <= REL_L2_NVFP4, (rel, nmax)
+    if fmt == "w4a16":
+        assert rel <= 1e-2, rel
+
+
+@pytest.mark.parametrize("fmt", ["w4a16", "w4a4"])
+@pytest.mark.parametrize("T", [3, 64, 200, 600])
+def test_nvfp4_ragged_expert_width(L, fmt, T):
+    """Expert width F = 328: not a multiple of 16, so each down-projection row
+    ends in an NVFP4 block of 8 (and W4A4's ReLU^2 activations too), the last
+    128-row block of the up projection holds 72 rows, and the down
+    projection's records end in a partial slice followed by zero slices."""
+    cfg = I.CONFIGS["tiny_fp32"].replace(dtype="bf16", expert_fmt=fmt, E=16, k=4, D=512,
+                                         L=256, F=328, Fs=328)
     lay, g, r = _run_full(L, cfg, T)
     _assert_routing_exact(g, r)
     rel, nmax, raw = out_metrics(g[0], r["out"])

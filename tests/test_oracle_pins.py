@@ -318,6 +318,41 @@ def test_nvfp4_error_bound_and_scales():
     assert rel < 0.12
 
 
+def test_nvfp4_partial_block_hand_example():
+    """A row of 24 elements: one full block and a partial block of 8.  The
+    partial block's scale comes from its own 8 values (amax 7: 7/6 = 1.1667
+    lies nearer the E4M3 value 1.125 than 1.25), and each value rounds on the
+    E2M1 grid scaled by 1.125 (7/1.125 = 6.22 -> 6; 0.3/1.125 = 0.267 -> 0.5;
+    -2/1.125 = -1.78 -> -2; 1/1.125 = 0.89 -> 1), worked out by hand."""
+    full = np.full(16, 0.75, np.float32)              # amax 0.75: s_b = 0.125 exactly
+    part = np.array([7.0, 0.3, -2.0, 1.0, 0.0, 0.0, 0.0, 0.0], np.float32)
+    w = np.concatenate([full, part])[None, :]
+    q, sb = O.nvfp4_quantize(w, np.float32(1.0))
+    assert q.shape == (1, 24) and sb.shape == (1, 2)
+    assert O.e4m3_value(int(sb[0, 0])) == 0.125 and O.e4m3_value(int(sb[0, 1])) == 1.125
+    deq = O.nvfp4_dequantize(q, sb, np.float32(1.0))
+    assert deq[0, :16].tolist() == [0.75] * 16
+    assert deq[0, 16:].tolist() == [6.75, 0.5625, -2.25, 1.125, 0.0, 0.0, 0.0, 0.0]
+
+
+def test_nvfp4_partial_block_is_local_and_roundtrips_representable_values():
+    rng = np.random.RandomState(13)
+    rows, K = 6, 40                                   # blocks of 16, 16 and 8
+    sg = np.float32(1.0)
+    sb = rng.randint(0x20, 0x48, size=(rows, 3)).astype(np.uint8)
+    q = rng.randint(0, 16, size=(rows, K)).astype(np.uint8)
+    q[:, [0, 16, 32]] = 7                            # +6 in every block, partial included
+    w = O.nvfp4_dequantize(q, sb, sg).astype(np.float32)
+    q2, sb2 = O.nvfp4_quantize(w, sg)
+    assert np.array_equal(sb2, sb)
+    assert np.array_equal(O.nvfp4_dequantize(q2, sb2, sg), O.nvfp4_dequantize(q, sb, sg))
+    # changing the full blocks changes neither the partial block's scale nor its codes
+    w3 = w.copy()
+    w3[:, :32] *= 3.0
+    q3, sb3 = O.nvfp4_quantize(w3, sg)
+    assert np.array_equal(sb3[:, 2], sb2[:, 2]) and np.array_equal(q3[:, 32:], q2[:, 32:])
+
+
 def test_pack_e2m1_low_nibble_first():
     c = np.array([[1, 2, 15, 0]], np.uint8)
     assert O.pack_e2m1(c).tolist() == [[0x21, 0x0F]]
