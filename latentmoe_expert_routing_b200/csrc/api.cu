@@ -51,6 +51,10 @@ struct moe_handle {
   // NVFP4 experts: GEMM-layout records and per-expert global scales
   uint8_t *rec_up = nullptr, *rec_dn = nullptr;
   CUtensorMap rm_up[3], rm_dn[3];                // record maps, batches of 1, 2, 4
+  // NVFP4 experts: z_perm / H as [slices][rows][64] with boxes of 4 slices
+  // (one load per pipeline step); am3_dn_ok: F is a multiple of 64
+  CUtensorMap am3_zp[5], am3_H[5];
+  bool am3_dn_ok = false;
   float *gs_up = nullptr, *gs_dn = nullptr;
   unsigned long long* stats = nullptr;           // exactly recomputed logits
   // W4A4 on the block-scaled FP4 tensor cores (128-token tiles): weights as
@@ -496,6 +500,9 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     u.args.act_gscale = w4a4 ? (dyn ? h->act_gs : nullptr) : h->zp2 + 1;
     u.args.acc_mul = w4a4 ? 0.f : 0x1p-4f;
     u.wqmap = h->rm_up[batch_idx(wq_kslices(L))];
+    if (batch_idx(wq_kslices(L)) == 2) {   // four slices per step: one token load per step
+      u.amap0 = h->am3_zp[gi]; u.amap1 = h->am3_zp[0]; u.args.act_slices = 4;
+    }
   }
   const bool pg = grouped_pair(c, P);     // SM pairs: 256-row weight blocks, half-token boxes
   if (pg) u.amap0 = h->am_zp[3];
@@ -510,6 +517,10 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     u.args.act_gscale = nullptr;
     u.args.acc_mul = w4a4 ? 0.f : 0x1p8f;         // W4A16: H was stored times 2^-8
     u.wqmap = h->rm_dn[batch_idx(wq_kslices(F))];
+    u.args.act_slices = 0;
+    if (h->am3_dn_ok && batch_idx(wq_kslices(F)) == 2) {
+      u.amap0 = h->am3_H[gi]; u.amap1 = h->am3_H[0]; u.args.act_slices = 4;
+    }
   }
   u.max_tiles = pg ? (int)((P / 256 + E) * (L / 256)) : (int)((P / ntg + E) * ceil_div(L, 128));
   if ((e = pg ? launch_umma_pair(u, s) : launch_umma(u, s)) != cudaSuccess) return MOE_ERR_CUDA;
@@ -689,6 +700,11 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
           make_tmap_bf16(&h->am_hsh[i], h->h_sh, T, Fs, kNT[i]);
     if (!m) { moe_destroy(h); return MOE_ERR_CUDA; }
     if (c.expert_fmt != MOE_EXPERT_DENSE) {
+      h->am3_dn_ok = F % 64 == 0;
+      for (int i = 0; i < 5 && m; ++i)
+        m = make_tmap_bf16_slices(&h->am3_zp[i], h->z_perm, P, L, kNT[i], 4) &&
+            (!h->am3_dn_ok || make_tmap_bf16_slices(&h->am3_H[i], h->H, P, F, kNT[i], 4));
+      if (!m) { moe_destroy(h); return MOE_ERR_CUDA; }
       moe_status q = quantize_experts(h, w, s);
       if (q != MOE_OK) { moe_destroy(h); return q; }
     }

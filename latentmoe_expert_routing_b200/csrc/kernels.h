@@ -140,6 +140,8 @@ struct UmmaArgs {
   const float* act_gscale;  // the activations' scale (one fp32 on the device: W4A4's global
                             // scale, or the inverse power of two W4A16 scaled them by) or NULL
   float acc_mul;            // NVFP4: a power of two the accumulator is multiplied by (0: 1)
+  int act_slices;           // NVFP4: > 0 when the token maps are 3-D (rows x 64-K slices) and
+                            // one load brings this many slices; 0: one 2-D load per slice
   int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
                             // fp32 partials out[slice][row][n] (slice stride below)
   long split_stride;        // elements between slices of the partial output
@@ -158,6 +160,11 @@ struct UmmaLaunch {
   int max_tiles;            // upper bound of the tile count (grid clamp)
 };
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int box_rows);
+// The same matrix as [K/64 slices][rows][64] (K a multiple of 64): a box of
+// `slices` slices x box_rows rows lands as `slices` consecutive 128-B-swizzled
+// [box_rows][64] tiles, as many 2-D boxes would
+bool make_tmap_bf16_slices(CUtensorMap* map, const void* base, long rows, int K, int box_rows,
+                           int slices);
 // NVFP4 GEMM records (4608 B each) as a 3-D uint8 tensor, box = `batch` records
 bool make_tmap_records(CUtensorMap* map, const void* base, long n_records, int batch);
 cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);

@@ -242,6 +242,20 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, long rows, int K, int bo
          CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_slices(CUtensorMap* map, const void* base, long rows, int K, int box_rows,
+                           int slices) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || !base || rows <= 0 || K <= 0 || (K % kBK) != 0 || slices < 1) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kBK, (cuuint64_t)rows, (cuuint64_t)(K / kBK)};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)kBK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kBK, (cuuint32_t)box_rows, (cuuint32_t)slices};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool make_tmap_u8(CUtensorMap* map, const void* base, long rows, int row_bytes, int box_bytes,
                   int box_rows, bool swizzle128) {
   EncodeTiledFn fn = encode_fn();

@@ -199,16 +199,21 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
         bool ok = true;
         // the MMA reads the tile's first n_eff rows: a tile of at most 16 valid
-        // rows loads 16-row boxes (half or less of the bytes)
+        // rows loads 16-row boxes (half or less of the bytes), its slices packed
+        // at 2 KB strides
         const bool short_tile = NT > 16 && ti.valid <= 16;
         const CUtensorMap* map = short_tile ? &amap16 : &amap;
-        const uint32_t step_bytes = KS * (short_tile ? 16 * kBK * 2 : S::kATileBytes);
+        const uint32_t tile_bytes = short_tile ? 16 * kBK * 2 : S::kATileBytes;
         for (int st = 0; st < nsteps; ++st, ++it) {
           if (!mbar_wait(&done[sa], pa)) { fail(13); ok = false; break; }
-          mbar_arrive_expect_tx(&a_full[sa], step_bytes);
+          mbar_arrive_expect_tx(&a_full[sa], KS * tile_bytes);
           uint8_t* dst = smem + sa * slot_bytes;
-          for (int ks = 0; ks < KS; ++ks)
-            tma_load_2d(dst + ks * S::kATileBytes, map, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
+          if (a.act_slices == KS) {          // [slices][rows][64] map: one load per step
+            tma_load_3d(dst, map, &a_full[sa], 0, ti.a_row0, st * KS);
+          } else {
+            for (int ks = 0; ks < KS; ++ks)
+              tma_load_2d(dst + ks * tile_bytes, map, &a_full[sa], (st * KS + ks) * kBK, ti.a_row0);
+          }
           if (++sa == (uint32_t)NA) { sa = 0; pa ^= 1; }
         }
         if (!ok) break;
@@ -236,6 +241,8 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // ragged tiles multiply only their valid rows, rounded up to N granularity 16
         const int n_eff = min(NT, (ti.valid + 15) & ~15);
         const uint32_t idesc = idesc_f16_f32(kBM, n_eff);
+        // slice stride of the step's activation tiles (short tiles: 16 rows)
+        const uint64_t b_step = ((NT > 16 && ti.valid <= 16) ? 16 * kBK * 2 : S::kATileBytes) >> 4;
         bool ok = true;
         for (int st = 0; st < nsteps; ++st) {
           // the step's A tiles (normally landed long before) and its W slot
@@ -243,7 +250,7 @@ umma_wq_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
           tc_fence_after();
           uint32_t wt = tmem + S::kWCol0 + s * 32 * KS;
           uint64_t bd = bdesc0 + (uint64_t)(sa * slot_desc);
-          for (int ks = 0; ks < KS; ++ks, wt += 32, bd += (S::kATileBytes >> 4)) {
+          for (int ks = 0; ks < KS; ++ks, wt += 32, bd += b_step) {
             if (SPLIT) {
               mma_bf16_ts(d, wt + 8 * j, bd + 2 * j, idesc, (st > 0 || ks > 0) ? 1u : 0u);
             } else {
