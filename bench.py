@@ -161,12 +161,14 @@ def _oracle_sample(cfg, W, x, n_tok, min_s=0.0, norm=None):
 
 
 def _measured_traffic(cfg, n_touched):
-    """DRAM bytes per grouped-GEMM launch from the committed ncu capture, scaled
-    by touched experts; None when the kernel sources changed since the capture
-    or the workload is not the dense-bf16 decode the capture covers."""
+    """DRAM bytes per grouped-GEMM launch from the committed ncu capture of the
+    decode-sized kernel (bf16 experts: umma_gemm_kernel; NVFP4 experts:
+    umma_wq_kernel), scaled by touched experts; None when the kernel's sources
+    changed since the capture or the workload is not one the capture covers."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "umma_gemm_traffic.json")
-    if cfg.dtype != "bf16" or cfg.expert_fmt != "dense" or not os.path.exists(p):
+    name = "umma_gemm_traffic.json" if cfg.expert_fmt == "dense" else "umma_wq_traffic.json"
+    p = os.path.join(ROOT, "profiles", name)
+    if cfg.dtype != "bf16" or not os.path.exists(p):
         return None
     d = json.load(open(p))
     h = hashlib.sha256()
