@@ -123,7 +123,7 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
   g.args.ksplit = S;
   g.args.dense_tiles = tiles * S;
   g.max_tiles = tiles * S;
-  if (S == 1 && half0 && umma_pair_eligible(g)) {
+  if (S == 1 && half0 && g.args.row_split == 0 && umma_pair_eligible(g)) {
     // 256 x 256 tiles on SM pairs, each CTA loading half of the token rows
     g.amap0 = *half0;
     if (half1) g.amap1 = *half1;
@@ -139,6 +139,10 @@ moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
   g.args.ldo = g.args.n_out;
   g.args.split_stride = (long)g.args.M * g.args.n_out;
   if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (g.args.row_split > 0)
+    return launch_split_reduce_rows(h->splitws, S, g.args.M, g.args.n_out, g.args.row_split, out,
+                                    g.args.out1, g.args.relu1, s) == cudaSuccess
+               ? MOE_OK : MOE_ERR_CUDA;
   return launch_split_reduce(h->splitws, S, g.args.M, g.args.n_out, out, epi, s) == cudaSuccess
              ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -411,12 +415,25 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   g.args.out = (mx || dyn) ? (void*)h->z32 : h->z;
   g.epi = (mx || dyn) ? UMMA_EPI_F32 : w4a4 ? UMMA_EPI_BF16_Q : UMMA_EPI_BF16;
   g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
-  g.wmap0 = h->wm_su;
-  g.args.n_out = Fs; g.args.ldo = Fs;
-  g.args.dense_tiles = ceil_div(Fs, 128) * ceil_div(T, ntd);
-  g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
-  if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
+  if (g.epi == UMMA_EPI_BF16 && ntd != 256 && L % 128 == 0) {
+    // decode-sized batches: fc1 and the shared up projection as one launch
+    // (rows [0, L) -> z, rows [L, L + Fs) -> h_sh with ReLU^2): one weight
+    // stream over all SMs, one split-K reduce
+    g.wmap1 = h->wm_su;
+    g.args.n_out = L + Fs;
+    g.args.row_split = L; g.args.out1 = h->h_sh; g.args.ldo1 = Fs; g.args.relu1 = 1;
+    g.args.dense_tiles = ceil_div(L + Fs, 128) * ceil_div(T, ntd);
+    g.max_tiles = g.args.dense_tiles;
+    if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
+    g.args.row_split = 0; g.args.out1 = nullptr;
+  } else {
+    if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
+    g.wmap0 = h->wm_su;
+    g.args.n_out = Fs; g.args.ldo = Fs;
+    g.args.dense_tiles = ceil_div(Fs, 128) * ceil_div(T, ntd);
+    g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
+    if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
+  }
   mark(MOE_STAGE_EXPERT_UP);
   if (dyn && launch_tensor_gscale(h->z32, (long)T * L, h->act_amax, h->act_gs, s) != cudaSuccess)
     return MOE_ERR_CUDA;

@@ -142,6 +142,13 @@ struct UmmaArgs {
   float acc_mul;            // NVFP4: a power of two the accumulator is multiplied by (0: 1)
   int act_slices;           // NVFP4: > 0 when the token maps are 3-D (rows x 64-K slices) and
                             // one load brings this many slices; 0: one 2-D load per slice
+  // dense mode, two GEMMs of one A in one launch: output rows [row_split, n_out)
+  // take their weights from wmap1 (row - row_split) and go to out1 (row stride
+  // ldo1, ReLU^2 when relu1); 0: one GEMM.  Needs K1 == 0 and row_split % 128 == 0.
+  int row_split;
+  void* out1;
+  int ldo1;
+  int relu1;
   int ksplit;               // dense mode: K slices per output tile (>= 1); > 1 writes
                             // fp32 partials out[slice][row][n] (slice stride below)
   long split_stride;        // elements between slices of the partial output
@@ -171,6 +178,10 @@ cudaError_t launch_umma(const UmmaLaunch& L, cudaStream_t st);
 // out[r][n] = epi(sum_s ws[s][r][n]) for s = 0..S-1 in order (split-K reduce)
 cudaError_t launch_split_reduce(const float* ws, int S, int M, int N, void* out, UmmaEpi epi,
                                 cudaStream_t st);
+// the same for a two-GEMM launch (UmmaArgs::row_split): bf16 out0 [M, row_split]
+// (no epilogue) and bf16 out1 [M, N - row_split] (ReLU^2 when relu1)
+cudaError_t launch_split_reduce_rows(const float* ws, int S, int M, int N, int row_split,
+                                     void* out0, void* out1, int relu1, cudaStream_t st);
 cudaError_t launch_umma_wq(const UmmaLaunch& L, cudaStream_t st);
 // two-SM variant for 256-token tiles (umma_gemm2.cu); the token maps (amap0,
 // amap1) must have 128-row boxes and grouped tile tables 256-row weight blocks

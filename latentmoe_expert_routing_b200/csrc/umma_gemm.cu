@@ -66,6 +66,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
     tma_prefetch_desc(&amap0);
     tma_prefetch_desc(&wmap0);
     if (a.K1 > 0) { tma_prefetch_desc(&wmap1); tma_prefetch_desc(&amap1); }
+    if (a.row_split > 0) tma_prefetch_desc(&wmap1);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::kTmemCols);
@@ -90,6 +91,9 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
         if (!decode_tile<NT>(a, s_tiles, s_off, tile, ti)) continue;
+        // second GEMM of a two-GEMM launch: its own weights, rows from 0
+        const bool rs1 = a.row_split > 0 && ti.n0 >= a.row_split;
+        const int wrow = rs1 ? ti.w_row0 - a.row_split : ti.w_row0;
         bool ok = true;
         for (int kt = ti.kb; kt < ti.ke; ++kt, ++it) {
           if (!mbar_wait(&empty[st], pe)) { fail(1); ok = false; break; }
@@ -97,7 +101,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
           mbar_arrive_expect_tx(&full[st], kWTileBytes + S::kATileBytes);
           const bool seg1 = kt >= kt0;
           const int k0 = (seg1 ? kt - kt0 : kt) * kBK;
-          tma_load_2d(sp, seg1 ? &wmap1 : &wmap0, &full[st], k0, ti.w_row0);
+          tma_load_2d(sp, (seg1 || rs1) ? &wmap1 : &wmap0, &full[st], k0, wrow);
           tma_load_2d(sp + kWTileBytes, seg1 ? &amap1 : &amap0, &full[st], k0, ti.a_row0);
           if (++st == STAGES) { st = 0; pe ^= 1; }
         }
@@ -163,6 +167,13 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
       const int n = ti.n0 + 32 * q + lane;   // output column of this thread
       const bool col_ok = n < a.n_out;
       const float gs = a.gscale ? a.gscale[ti.wgrp] : 1.f;
+      // a two-GEMM launch writes its second GEMM's rows to out1 (split-K
+      // partials keep the joint column index; the reduce separates them)
+      const bool rs1 = a.row_split > 0 && ti.n0 >= a.row_split && a.ksplit <= 1;
+      TO* const ob = rs1 ? reinterpret_cast<TO*>(a.out1) : out;
+      const int on = rs1 ? n - a.row_split : n;
+      const int oldo = rs1 ? a.ldo1 : a.ldo;
+      const bool relu = RELU2 || (rs1 && a.relu1);
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + buf * NT;
       auto emit = [&](const uint32_t (&r)[8], int c) {
         float v[8];
@@ -170,7 +181,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         for (int j = 0; j < 8; ++j) {
           v[j] = __uint_as_float(r[j]);
           if (a.gscale) v[j] = __fmul_rn(v[j], gs);
-          if (RELU2) v[j] = relu2(v[j]);
+          if (relu) v[j] = relu2(v[j]);
           if (!col_ok) v[j] = 0.f;
         }
         if (QA) nvfp4_roundtrip16x8(v);
@@ -178,7 +189,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap wmap0,
         for (int j = 0; j < 8; ++j) {
           const int row = c * 8 + j;
           if (row < ti.valid && col_ok)
-            store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
+            store_out(ob + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * oldo + on, v[j]);
         }
       };
       // two chunks in flight per wait; chunks past the valid rows are skipped
@@ -374,6 +385,46 @@ cudaError_t launch_split_reduce(const float* ws, int S, int M, int N, void* out,
     case UMMA_EPI_BF16_Q: split_reduce_kernel<__nv_bfloat16, false, true><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
     case UMMA_EPI_BF16_RELU2_Q: split_reduce_kernel<__nv_bfloat16, true, true><<<g, 256, 0, st>>>(ws, S, M, N, (__nv_bfloat16*)out); break;
   }
+  return cudaGetLastError();
+}
+
+// Split-K reduce of a two-GEMM launch: columns below row_split to out0 as
+// they are, the others to out1 (ReLU^2 when relu1); bf16 outputs.
+__global__ void split_reduce_rows_kernel(const float* __restrict__ ws, int S, int M, int N,
+                                         int row_split, __nv_bfloat16* __restrict__ out0,
+                                         __nv_bfloat16* __restrict__ out1, int relu1) {
+  const long b = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nb = N / 16;
+  if (b >= (long)M * nb) return;
+  const int r = (int)(b / nb), c0 = (int)(b - (long)r * nb) * 16;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float4* p = reinterpret_cast<const float4*>(ws + ((size_t)s * M + r) * N + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t = p[q];
+      v[4 * q] += t.x; v[4 * q + 1] += t.y; v[4 * q + 2] += t.z; v[4 * q + 3] += t.w;
+    }
+  }
+  const bool second = c0 >= row_split;
+  if (second && relu1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = relu2(v[i]);
+  }
+  __nv_bfloat16* o = second ? out1 + (size_t)r * (N - row_split) + (c0 - row_split)
+                            : out0 + (size_t)r * row_split + c0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) store_out(o + i, v[i]);
+}
+
+cudaError_t launch_split_reduce_rows(const float* ws, int S, int M, int N, int row_split,
+                                     void* out0, void* out1, int relu1, cudaStream_t st) {
+  if (N % 16 || row_split % 16) return cudaErrorInvalidValue;
+  const long n = (long)M * (N / 16);
+  split_reduce_rows_kernel<<<ceil_div(n, 256), 256, 0, st>>>(
+      ws, S, M, N, row_split, (__nv_bfloat16*)out0, (__nv_bfloat16*)out1, relu1);
   return cudaGetLastError();
 }
 
