@@ -106,8 +106,45 @@ const size_t kSplitWsElems = size_t(10) << 20;     // 40 MB of fp32 split-K part
 moe_status launch_dense_umma(moe_handle* h, UmmaLaunch g, cudaStream_t s,
                              const CUtensorMap* half0 = nullptr,
                              const CUtensorMap* half1 = nullptr) {
-  const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
   const int steps = (g.args.K0 + g.args.K1 + 63) / 64;
+  if (half0 && g.nt == 256 && g.args.M <= 256 && g.args.row_split == 0 &&
+      g.args.n_out % 256 == 0) {
+    // one token tile of up to 256 rows: 256 x 256 tiles on SM pairs, each CTA
+    // loading half of the token rows (a weight byte meets twice the tokens per
+    // byte moved), K split so that the pairs fill the GPU (the same cost model
+    // over pairs)
+    const int pairs = h->sms / 2;
+    const int ptiles = (g.args.n_out / 256) * ceil_div(g.args.M, 256);
+    int S = 1;
+    double best = 1e30;
+    for (int c = 1; c <= 64 && c <= steps; ++c) {
+      if (steps % c || (c > 1 && steps / c < 2)) continue;
+      if (c > 1 && (size_t)c * g.args.M * g.args.n_out > h->splitws_elems) continue;
+      if (c > 1 && g.args.n_out % 16) continue;
+      const int waves = ceil_div((long)ptiles * c, pairs);
+      const double cost = waves * (steps / (double)c + 2.0) + (c > 1 ? 1.0 : 0.0);
+      if (cost < best - 1e-9) { best = cost; S = c; }
+    }
+    UmmaLaunch p = g;
+    p.amap0 = *half0;
+    if (half1) p.amap1 = *half1;
+    p.args.ksplit = S;
+    p.args.dense_tiles = ptiles * S;
+    p.max_tiles = ptiles * S;
+    if (S > 1) {
+      p.epi = UMMA_EPI_F32;
+      p.args.out = h->splitws;
+      p.args.ldo = g.args.n_out;
+      p.args.split_stride = (long)g.args.M * g.args.n_out;
+    }
+    if (umma_pair_eligible(p)) {
+      if (launch_umma_pair(p, s) != cudaSuccess) return MOE_ERR_CUDA;
+      if (S == 1) return MOE_OK;
+      return launch_split_reduce(h->splitws, S, g.args.M, g.args.n_out, g.args.out, g.epi, s) ==
+                     cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
+  }
+  const int tiles = ceil_div(g.args.n_out, 128) * ceil_div(g.args.M, g.nt);
   // Pick the K split with the least modelled time: waves of the persistent grid
   // times (steps per slice + a fixed per-tile cost of about two steps).
   int S = 1;

@@ -121,6 +121,12 @@ constexpr int kPairBM = 256;                  // weight rows per pair tile (MMA 
 __device__ __forceinline__ bool decode_pair_tile(const UmmaArgs& a, const int32_t* s_tiles,
                                                  const int32_t* s_off, int tile, TileInfo& ti) {
   const int nmb = a.n_out / kPairBM;
+  // dense mode with split-K: `ksplit` consecutive tiles are the K slices of
+  // one output tile (fp32 partials, reduced by the caller)
+  const int S = (!a.offsets && a.ksplit > 1) ? a.ksplit : 1;
+  const int kt_all = (a.K0 + a.K1 + kBK - 1) / kBK;
+  const int slice = tile % S;
+  tile /= S;
   int e = 0, base = 0, cnt = a.M, local = tile;
   if (a.offsets) {
     int lo = 0, hi = a.E;
@@ -144,9 +150,9 @@ __device__ __forceinline__ bool decode_pair_tile(const UmmaArgs& a, const int32_
   ti.w_row0 = ti.wgrp * a.w_group_rows + ti.n0;
   ti.a_row0 = base + nb * kPairNT;
   ti.valid = min(kPairNT, cnt - nb * kPairNT);
-  ti.kb = 0;
-  ti.ke = (a.K0 + a.K1 + kBK - 1) / kBK;
-  ti.slice = 0;
+  ti.kb = slice * (kt_all / S);
+  ti.ke = ti.kb + kt_all / S;
+  ti.slice = slice;
   return true;
 }
 

@@ -201,7 +201,8 @@ umma_pair_kernel(const __grid_constant__ CUtensorMap wmap0,
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int row = c * 8 + j;
-          if (row < ti.valid && col_ok) store_out(out + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
+          if (row < ti.valid && col_ok)
+            store_out(out + ti.slice * a.split_stride + (size_t)(ti.a_row0 + row) * a.ldo + n, v[j]);
         }
       };
       // blocks of 32 columns (one TMEM load and one wait each), alternating
@@ -263,10 +264,11 @@ static cudaError_t pair_launch_t(const UmmaLaunch& L, cudaStream_t st) {
 }
 
 // The pair kernel takes 256-token tiles (its token maps have 128-row boxes:
-// each CTA loads half a tile), weight matrices with rows in multiples of 256,
-// no split-K and bf16 weights.
+// each CTA loads half a tile), weight matrices with rows in multiples of 256
+// and bf16 weights; split-K (dense mode) writes fp32 partials.
 bool umma_pair_eligible(const UmmaLaunch& L) {
-  return L.nt == 256 && L.args.n_out % kPairBM == 0 && L.args.ksplit <= 1 && !L.args.wq &&
+  return L.nt == 256 && L.args.n_out % kPairBM == 0 && !L.args.wq &&
+         (L.args.ksplit <= 1 || (!L.args.offsets && L.epi == UMMA_EPI_F32)) &&
          (!L.args.offsets || L.args.w_group_rows % kPairBM == 0) &&
          (L.epi == UMMA_EPI_BF16 || L.epi == UMMA_EPI_BF16_RELU2 || L.epi == UMMA_EPI_F32 ||
           L.epi == UMMA_EPI_BF16_Q);
