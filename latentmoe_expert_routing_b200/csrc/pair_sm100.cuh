@@ -107,17 +107,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-// D (+)= A * B^T with A (each CTA's 128 rows, 16 K) read from both CTAs'
-// TMEM at the same address and B from both CTAs' shared memory, M = 256
-__device__ __forceinline__ void mma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
 // Bounded wait (about two seconds of SM clock) with cluster-scope acquire, for
 // barriers that the peer CTA arrives on: its prior writes (shared or tensor
 // memory, fenced before its arrival) are visible once the phase completes.
