@@ -158,13 +158,18 @@ def test_bf16_wide_tiles_and_many_experts(L):
     _assert_out(g[0], r["out"])
 
 
-@pytest.mark.parametrize("bias_kind", ["normal", "zipf"])
-def test_bf16_sm_pair_tiles(L, bias_kind):
+@pytest.mark.parametrize("bias_kind,T", [("normal", 1200), ("zipf", 1200), ("normal", 64),
+                                         ("normal", 200), ("zipf", 256)])
+def test_bf16_sm_pair_tiles(L, bias_kind, T):
     """256-token tiles whose weight matrices have rows in multiples of 256 run
     on SM pairs (two-CTA MMA): grouped up/down and the dense fc1, shared-up and
     fc2 GEMMs here.  Zipf bias gives experts with many full tiles and experts
-    with a handful of tokens (ragged tiles down to one 16-row MMA step)."""
-    cfg = TINY.replace(dtype="bf16", E=16, k=4, D=512, L=256, F=512, Fs=512, T=1200,
+    with a handful of tokens (ragged tiles down to one 16-row MMA step).
+    T = 200 and 256 (one token tile) run the dense GEMMs on SM pairs with a
+    K split (fp32 partials, fixed-order reduce); T = 64 runs fc1 and the
+    shared up projection as one launch (rows split between two weights and
+    two outputs)."""
+    cfg = TINY.replace(dtype="bf16", E=16, k=4, D=512, L=256, F=512, Fs=512, T=T,
                        bias_kind=bias_kind)
     lay, g, r = _run_full(L, cfg)
     _assert_routing_exact(g, r)
