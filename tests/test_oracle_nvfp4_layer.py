@@ -43,10 +43,11 @@ def _e4m3(code):
 def representable(rng, rows, K, s_g):
     """[rows, K] fp32 matrix of values q * s_b * s_g: every 16-block holds a +-6
     element, block (0, 0) has s_b = 448 (so the matrix amax is 2688 * s_g), one
-    other block is all zero."""
-    nb = K // 16
+    other block is all zero.  K may end in a partial block of 8 elements (its
+    +-6 then lies among those 8)."""
+    nb = -(-K // 16)
     codes = rng.randint(0, 16, size=(rows, nb, 16))
-    codes[:, :, rng.randint(0, 16)] = 7 + 8 * rng.randint(0, 2)     # +-6 in each block
+    codes[:, :, rng.randint(0, 8)] = 7 + 8 * rng.randint(0, 2)      # +-6 in each block
     sb = np.array([[_e4m3(c) for c in r] for r in rng.randint(0x28, 0x70, size=(rows, nb))])
     sb[0, 0] = 448.0
     q = np.array([[[(-1.0 if c & 8 else 1.0) * _E2M1[c & 7] for c in b] for b in r]
@@ -54,7 +55,7 @@ def representable(rng, rows, K, s_g):
     w = q * sb[..., None] * float(s_g)
     if rows > 1 and nb > 1:
         w[rows - 1, nb - 1] = 0.0
-    w = w.reshape(rows, K)
+    w = w.reshape(rows, nb * 16)[:, :K]
     assert np.array_equal(w.astype(np.float32).astype(np.float64), w)
     assert np.max(np.abs(w)) == 2688.0 * float(s_g)
     return w.astype(np.float32)
@@ -88,6 +89,28 @@ def test_w4a16_equals_dense_on_representable_experts():
     dense, q = _run(*a, "dense"), _run(*a, "w4a16")
     assert np.array_equal(q, dense)
     assert np.abs(dense).max() > 0
+
+
+def test_w4a16_equals_dense_with_partial_blocks():
+    """Expert width F = 40: the down projection's rows (K = F) end in a block of
+    8 elements, quantised as a block whose missing elements are zero; on
+    representable experts the W4A16 layer still equals the dense one."""
+    rng = np.random.RandomState(3)
+    T, D, L, E, k, F, Fs = 6, 48, 32, 4, 2, 40, 32
+    up = np.stack([representable(rng, F, L, SG[e]) for e in range(E)])
+    down = np.stack([representable(rng, L, F, SG[E + e]) for e in range(E)])
+    f32 = lambda *s: (rng.standard_normal(s) / np.sqrt(s[-1])).astype(np.float32)
+    x = rng.standard_normal((T, D)).astype(np.float32)
+    a = (x, f32(E, D), (0.1 * rng.standard_normal(E)).astype(np.float32), f32(L, D),
+         f32(D, L), f32(Fs, D), f32(D, Fs), up, down, k)
+    dense, q = _run(*a, "dense"), _run(*a, "w4a16")
+    assert np.array_equal(q, dense)
+    assert np.abs(dense).max() > 0
+    # a mistaken reading (the partial block's scale from a 16-element window
+    # that reaches into the next row) would change the codes: the oracle's
+    # quantiser keeps each row's blocks to that row
+    q0, sb0 = O.nvfp4_quantize(down[0], np.float32(O.nvfp4_global_scale(down[0])))
+    assert sb0.shape == (L, 3) and q0.shape == (L, F)
 
 
 def _w4a4_case(seed=1):
