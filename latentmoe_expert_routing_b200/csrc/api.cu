@@ -38,6 +38,10 @@ struct moe_handle {
   // captured on the second call with the same T (the first configures every
   // kernel eagerly) on a private stream and replayed on the caller's stream
   cudaStream_t cap_stream = nullptr;
+  // G1 (fc1, shared up) runs on `side`, forked from the caller's stream and
+  // joined before the experts, so that it overlaps the router
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   cudaGraphExec_t host_graph = nullptr;
   int host_graph_T = 0, host_eager_T = 0, host_graph_off = 0;
   // tensor-core path (bf16): permuted latent rows and cached TMA maps
@@ -422,17 +426,15 @@ moe_status launch_g5(moe_handle* h, int M, const CUtensorMap& zc_map, const CUte
   return launch_dense_umma(h, g, s, &zc_half, &hsh_half);
 }
 
-template <typename Mark>
-moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMap* xhalf, int T,
-                        void* out, const int32_t* idx,
-                        const float* wts, Mark& mark, cudaStream_t s, float* zc_part) {
+// step 5 and the shared expert's up projection (G1): both read x, neither
+// depends on the routing
+moe_status launch_g1(moe_handle* h, const CUtensorMap& xmap, const CUtensorMap* xhalf, int T,
+                     cudaStream_t s) {
   const moe_config& c = h->cfg;
-  const int D = c.d_model, L = c.d_latent, E = c.n_experts, k = c.top_k;
-  const int F = c.d_ff, Fs = c.d_ff_shared;
+  const int D = c.d_model, L = c.d_latent, k = c.top_k;
+  const int Fs = c.d_ff_shared;
   const long P = (long)T * k;
-  const int di = nt_index(T), gi = grouped_nt_index(c, P);
-  const int ntd = kNT[di], ntg = kNT[gi];
-  cudaError_t e;
+  const int ntd = kNT[nt_index(T)];
   moe_status st;
 
   UmmaLaunch g{};
@@ -446,7 +448,6 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
   g.args.K0 = D; g.args.K1 = 0; g.args.n_out = L; g.args.ldo = L;
   g.args.dense_tiles = ceil_div(L, 128) * ceil_div(T, ntd);
   const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
-  const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
   const bool mx = use_mxf4(c, P) && h->zq;    // W4A4 on the block-scaled FP4 tensor cores
   const bool dyn = w4a4 && h->act_gs;         // the latent's per-tensor global scale
   g.args.out = (mx || dyn) ? (void*)h->z32 : h->z;
@@ -471,6 +472,26 @@ moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMa
     g.args.out = h->h_sh; g.epi = UMMA_EPI_BF16_RELU2; g.max_tiles = g.args.dense_tiles;
     if ((st = launch_dense_umma(h, g, s, xhalf)) != MOE_OK) return st;
   }
+  return MOE_OK;
+}
+
+template <typename Mark>
+moe_status forward_umma(moe_handle* h, const CUtensorMap& xmap, const CUtensorMap* xhalf, int T,
+                        void* out, const int32_t* idx,
+                        const float* wts, Mark& mark, cudaStream_t s, float* zc_part) {
+  // G1 ran before (launch_g1, on the side stream, joined into s)
+  (void)xmap; (void)xhalf;
+  const moe_config& c = h->cfg;
+  const int L = c.d_latent, E = c.n_experts, k = c.top_k;
+  const int F = c.d_ff;
+  const long P = (long)T * k;
+  const int di = nt_index(T), gi = grouped_nt_index(c, P);
+  const int ntg = kNT[gi];
+  cudaError_t e;
+  const bool w4a4 = c.expert_fmt == MOE_EXPERT_NVFP4_W4A4;
+  const bool wq = c.expert_fmt != MOE_EXPERT_DENSE;
+  const bool mx = use_mxf4(c, P) && h->zq;    // W4A4 on the block-scaled FP4 tensor cores
+  const bool dyn = w4a4 && h->act_gs;         // the latent's per-tensor global scale
   mark(MOE_STAGE_EXPERT_UP);
   if (dyn && launch_tensor_gscale(h->z32, (long)T * L, h->act_amax, h->act_gs, s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -617,6 +638,9 @@ void moe_destroy(moe_handle* h) {
   cudaSetDevice(h->device);
   if (h->host_graph) cudaGraphExecDestroy(h->host_graph);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+  if (h->ev_join) cudaEventDestroy(h->ev_join);
   for (void* p : h->owned) cudaFree(p);
   for (cudaEvent_t e : h->ev)
     if (e) cudaEventDestroy(e);
@@ -729,6 +753,13 @@ moe_status moe_init_ep(moe_handle** out, const moe_config* cfg, const moe_weight
       return MOE_ERR_UNSUPPORTED;
     }
     cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      moe_destroy(h);
+      return MOE_ERR_CUDA;
+    }
     h->splitws_elems = kSplitWsElems;
     if (!dev_alloc(h, &h->splitws, h->splitws_elems * 4) ||
         !dev_alloc(h, &h->logit_parts, router_parts_elems((int)D, (int)E, (int)T) * 4) ||
@@ -843,10 +874,20 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
   // steps 1-4: logits, sigmoid, biased selection, weights; step 6 bookkeeping
   CUtensorMap xmap, xhalf;
   const bool wide = nt_index(T) == 2;    // 256-token tiles: SM-pair GEMMs load half boxes
+  bool forked = false;
+  moe_status g1_status = MOE_OK;
   if (dt == MOE_BF16) {
     // tensor-core logits; the certified selection below makes them exact
     if (!make_tmap_bf16(&xmap, hidden, T, D, kNT[nt_index(T)])) return MOE_ERR_CUDA;
     if (wide && !make_tmap_bf16(&xhalf, hidden, T, D, 128)) return MOE_ERR_CUDA;
+    // G1 does not depend on the routing: it runs on the side stream meanwhile
+    // (forked here, joined before the experts; both streams only read x)
+    if (cudaEventRecord(h->ev_fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(h->side, h->ev_fork, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    g1_status = launch_g1(h, xmap, wide ? &xhalf : nullptr, T, h->side);
+    if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess) return MOE_ERR_CUDA;
+    forked = true;
     UmmaLaunch g{};
     g.wmap0 = h->wm_gate; g.amap0 = xmap; g.nt = kNT[nt_index(T)];
     g.args.err = h->err; g.args.E = 1; g.args.M = T;
@@ -855,7 +896,10 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
     g.args.dense_tiles = ceil_div(E, 128) * ceil_div(T, g.nt) * g.args.ksplit;
     g.args.split_stride = (long)T * E;
     g.args.out = h->logit_parts; g.epi = UMMA_EPI_F32; g.max_tiles = g.args.dense_tiles;
-    if (launch_umma(g, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_umma(g, s) != cudaSuccess) {
+      cudaStreamWaitEvent(s, h->ev_join, 0);
+      return MOE_ERR_CUDA;
+    }
   } else {
     launch_router_logits(hidden, h->w_gate, h->logits, T, D, E, dt, s);
   }
@@ -890,6 +934,9 @@ static moe_status forward_impl(moe_handle* h, const void* hidden, int T, void* o
   mark(MOE_STAGE_DENSE_IN);
 
   if (dt == MOE_BF16) {
+    // join G1 (the side stream's work) before anything reads z or h_sh
+    if (forked && cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (g1_status != MOE_OK) return g1_status;
     moe_status us = forward_umma(h, xmap, wide ? &xhalf : nullptr, T, out, idx, wts, mark, s,
                                  zc_part);
     if (us != MOE_OK) return us;
