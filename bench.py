@@ -213,6 +213,34 @@ def _gen_device():
     return "cuda" if torch.cuda.is_available() else "cpu"
 
 
+def _workload_config(a, cfg, world, n_touched):
+    """The workload as both arms name it: shape, format, launch and L2 note."""
+    from latentmoe_expert_routing_b200 import inputs as I
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.D, "d_latent": cfg.L,
+            "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
+            "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
+            "bias": cfg.bias_kind, "outlier_rows": len(I.outlier_rows(cfg)),
+            "parallelism": f"replicas{world}",
+            "cuda_graph": not a.no_graph,
+            "block": bool(a.block),
+            "l2": "no flush: each step streams the touched experts' weights "
+                  f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"}
+
+
+def _oracle_touched(cfg, W, x, norm=None):
+    """Experts that the oracle's router sends at least one of the T rows to."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    f = lambda t: t.detach().float().cpu().numpy()
+    rows = f(x)
+    if norm is not None:
+        y = O.rmsnorm_spec(rows, f(norm[0]), norm[1])
+        rows = O.round_fp64_to_bf16(y) if cfg.dtype == "bf16" else y.astype(np.float32)
+    l = O.router_logits(rows, f(W["w_gate"]))
+    _, _, idx, _ = O.route(l, f(W["gate_bias"]), cfg.k, cfg.rsf, cfg.n_group, cfg.topk_group)
+    return len(set(idx.reshape(-1).tolist()))
+
+
 def run_reference(a):
     rank, world, _ = _dist()
     if rank != 0:
@@ -222,19 +250,21 @@ def run_reference(a):
     cfg = I.CONFIGS[a.config]
     dev = _gen_device()
     W = _weights(cfg, dev)
-    x = I.hidden(cfg, dev)
+    x = I.hidden(cfg, dev, T=cfg.T, start_row=0)
+    norm = (I.norm_weight(cfg, dev), 1e-5) if a.block else None
     n_tok = cfg.T if cfg.T * cfg.D <= 64 * 256 else 2
     for _ in range(a.warmup):
-        _oracle_sample(cfg, W, x, n_tok)
-    times = [_oracle_sample(cfg, W, x, n_tok)[1] for _ in range(a.steps)]
+        _oracle_sample(cfg, W, x, n_tok, norm=norm)
+    times = [_oracle_sample(cfg, W, x, n_tok, norm=norm)[1] for _ in range(a.steps)]
     value = n_tok * a.steps / sum(times)
-    sample = f"first {n_tok} of {cfg.T} tokens per step, fp64 numpy oracle"
+    sample = (f"first {n_tok} of {cfg.T} tokens per step, fp64 numpy oracle"
+              + (" (block)" if a.block else ""))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": 1, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": 1e3 * sum(times) / a.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "sample_tokens": n_tok},
+        "config": _workload_config(a, cfg, world, _oracle_touched(cfg, W, x, norm)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -433,15 +463,7 @@ def _measure(a, cfg, W, rank, world, local, cpu_leg):
     res = {
         "value": D.job_throughput(T, world, ms_max * 1e-3), "ms_per_step": ms_max,
         "dtype": cfg.dtype if cfg.expert_fmt == "dense" else f"{cfg.dtype}+nvfp4-{cfg.expert_fmt}",
-        "config": {"workload": cfg.name, "T": T, "d_model": cfg.D, "d_latent": cfg.L,
-                   "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
-                   "d_ff_shared": cfg.Fs, "expert_fmt": cfg.expert_fmt,
-                   "bias": cfg.bias_kind, "outlier_rows": len(I.outlier_rows(cfg)),
-                   "parallelism": f"replicas{world}",
-                   "cuda_graph": graph is not None,
-                   "block": bool(a.block),
-                   "l2": "no flush: each step streams the touched experts' weights "
-                         f"({2 * _expert_bytes(cfg, n_touched) / 1e9:.1f} GB) > 126 MB L2"},
+        "config": _workload_config(a, cfg, world, n_touched),
         "roofline": roof,
         "layer_roofline": _layer_roofline(cfg, T, ms_max, hbm, tf, tf_sus, src, n_touched),
         "stages_ms": stage_ms,

@@ -18,11 +18,21 @@ def _json_lines(out):
     return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
 
 
-def _check(line, steps):
+# the workload keys that the GPU arm's line carries too: both arms name the
+# same configuration, so the two lines can be compared key for key
+CONFIG_KEYS = ["workload", "T", "d_model", "d_latent", "experts", "top_k", "d_ff",
+               "d_ff_shared", "expert_fmt", "bias", "outlier_rows", "parallelism",
+               "cuda_graph", "block", "l2"]
+
+
+def _check(line, steps, world=1):
     for k in KEYS:
         assert k in line, k
     assert line["impl"] == "reference" and line["steps"] == steps and line["value"] > 0
-    assert line["config"]["workload"] == "tiny_fp32"
+    c = line["config"]
+    assert sorted(c) == sorted(CONFIG_KEYS)
+    assert c["workload"] == "tiny_fp32" and c["T"] == 64 and c["experts"] == 16
+    assert c["parallelism"] == f"replicas{world}"
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     e = line["e2e"]
@@ -52,4 +62,4 @@ def test_reference_arm_under_two_ranks_prints_once():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
-    _check(lines[0], 1)
+    _check(lines[0], 1, world=2)
