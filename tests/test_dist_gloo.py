@@ -1,4 +1,4 @@
-"""Multi-rank plumbing on CPU: two gloo ranks agree on the slowest rank's time
+"""Multi-rank plumbing on CPU: gloo ranks agree on the slowest rank's time
 and the whole-job throughput (the bench's N>1 path, without GPUs)."""
 import os
 import socket
@@ -53,7 +53,7 @@ def test_single_rank_needs_no_process_group():
     assert D.job_throughput(64, 1, 0.002) == 32000.0
 
 
-def _ep_worker(rank, world, port, q):
+def _ep_worker(rank, world, port, q, T=37):
     """One expert-parallel rank on the CPU: the compute of each step is the
     oracle's arithmetic on this rank's experts; the exchange, the shard split
     and the rank-order sum are the library's multi-rank code."""
@@ -64,7 +64,7 @@ def _ep_worker(rank, world, port, q):
     from latentmoe_expert_routing_b200 import dist as D
     from latentmoe_expert_routing_b200 import inputs as I
     from oracle import moe_oracle as O
-    cfg = I.CONFIGS["tiny_fp32"].replace(T=37)
+    cfg = I.CONFIGS["tiny_fp32"].replace(T=T)
     x = I.hidden(cfg).numpy()
     W = {n: f(cfg).numpy() for n, f in (("g", I.w_gate), ("b", I.gate_bias), ("fc1", I.w_fc1),
                                         ("fc2", I.w_fc2), ("su", I.w_shared_up),
@@ -103,8 +103,13 @@ def _ep_worker(rank, world, port, q):
     D.finish()
 
 
-def test_expert_parallel_exchange_on_two_gloo_ranks():
-    """Two CPU ranks each hold half of the experts: gathered in rank order and
+@pytest.mark.parametrize("world,T,starts", [
+    (2, 37, [0, 19]),                 # shards 0..18 and 19..36
+    (4, 37, [0, 10, 19, 28]),         # 10, 9, 9, 9 rows
+    (4, 3, [0, 1, 2, 3]),             # fewer rows than ranks: the last shard is empty
+])
+def test_expert_parallel_exchange_on_gloo_ranks(world, T, starts):
+    """CPU ranks each hold E / world of the experts: gathered in rank order and
     finished on token shards, the outputs equal the whole oracle layer's."""
     import numpy as np
     from latentmoe_expert_routing_b200 import inputs as I
@@ -112,17 +117,19 @@ def test_expert_parallel_exchange_on_two_gloo_ranks():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    ps = [ctx.Process(target=_ep_worker, args=(r, 2, port, q)) for r in range(2)]
+    ps = [ctx.Process(target=_ep_worker, args=(r, world, port, q, T)) for r in range(world)]
     for p in ps:
         p.start()
-    res = sorted([q.get(timeout=120) for _ in range(2)], key=lambda r: r[0])
+    res = sorted([q.get(timeout=120) for _ in range(world)], key=lambda r: r[0])
     for p in ps:
         p.join(120)
         assert p.exitcode == 0
-    assert [r[1] for r in res] == [0, 19]            # shards 0..18 and 19..36
+    assert [r[1] for r in res] == starts
     out = np.concatenate([r[2] for r in res])
-    assert np.array_equal(res[0][3], res[1][3])      # both ranks routed alike
-    cfg = I.CONFIGS["tiny_fp32"].replace(T=37)
+    assert out.shape[0] == T
+    for r in res[1:]:
+        assert np.array_equal(res[0][3], r[3])      # every rank routed alike
+    cfg = I.CONFIGS["tiny_fp32"].replace(T=T)
     f = lambda g: g(cfg).numpy()
     ref = O.forward(I.hidden(cfg).numpy(), f(I.w_gate), f(I.gate_bias), f(I.w_fc1), f(I.w_fc2),
                     f(I.w_shared_up), f(I.w_shared_down),
