@@ -31,7 +31,7 @@ import math
 import numpy as np
 
 # ---------------------------------------------------------------------------
-# Router logits (section 5.6, step 1: gate = linear(x.float(), W.float()))
+# Router logits (section 5.6, step 1: the gate logits, x times W_gate^T in fp32)
 # ---------------------------------------------------------------------------
 
 
