@@ -115,3 +115,79 @@ def test_skewed_bias_concentrates_load():
     _, _, idx, _ = O.route(l, I.gate_bias(cfg).numpy(), cfg.k, cfg.rsf)
     counts, _, _, _ = O.dispatch(idx, cfg.E)
     assert O.max_violation(counts) > 20
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each plausible slip in the oracle's layer (report section
+# 5.6 steps 1-7, sections 5.1 and 5.3-5.4) breaks at least one pin above.
+# The mistakes are planted in the oracle, on the CPU, and undone afterwards.
+# ---------------------------------------------------------------------------
+
+def _holds(pin):
+    try:
+        pin()
+    except AssertionError:
+        return False
+    return True
+
+
+_LAYER_PINS = {
+    "k_equals_E": test_k_equals_E_is_dense_weighted_sum,
+    "k1": test_k1_is_single_mlp_with_weight_rsf,
+    "shared_only": test_zero_experts_and_fc2_leave_only_shared_mlp,
+    "routing": test_routing_matches_direct_definition_on_tiny,
+}
+
+
+def test_layer_pins_hold_for_the_oracle():
+    assert all(_holds(p) for p in _LAYER_PINS.values())
+
+
+def _plant(monkeypatch, mistake):
+    route, relu2, logits = O.route, O.relu2, O.router_logits
+
+    def reroute(fix):
+        def wrapped(l, bias, k, rsf, *a, **kw):
+            s, choice, idx, w = route(l, bias, k, rsf, *a, **kw)
+            return s, choice, idx, fix(s, choice, idx, w, rsf)
+        monkeypatch.setattr(O, "route", wrapped)
+
+    def gathered(v, idx):
+        return np.take_along_axis(v, idx, axis=1).astype(np.float32)
+
+    if mistake == "relu_not_squared":             # section 5.1: the square dropped
+        monkeypatch.setattr(O, "relu2", lambda v: np.maximum(v, 0.0))
+    elif mistake == "no_scaling_factor":          # the routed scaling factor left out
+        reroute(lambda s, c, idx, w, rsf: (w / np.float32(rsf)).astype(np.float32))
+    elif mistake == "unnormalised_weights":       # raw scores, not divided by their sum
+        reroute(lambda s, c, idx, w, rsf: gathered(s, idx) * np.float32(rsf))
+    elif mistake == "weights_from_biased_score":  # the bias leaking into the weights
+        def fix(s, c, idx, w, rsf):
+            r = gathered(c, idx)
+            return (r / r.sum(1, keepdims=True) * np.float32(rsf)).astype(np.float32)
+        reroute(fix)
+    elif mistake == "weights_in_wrong_slots":     # slot j weighted by slot j+1's weight
+        reroute(lambda s, c, idx, w, rsf: np.roll(w, 1, axis=1))
+    elif mistake == "bias_ignored_in_selection":  # plain top-k of the scores
+        monkeypatch.setattr(O, "route", lambda l, bias, *a, **kw:
+                            route(l, np.zeros_like(bias), *a, **kw))
+    elif mistake == "gate_rows_misindexed":       # expert e scored with row E-1-e
+        monkeypatch.setattr(O, "router_logits", lambda x, w: logits(x, w[::-1]))
+    elif mistake == "shared_expert_dropped":      # the shared MLP's activation lost
+        monkeypatch.setattr(O, "relu2", lambda v: relu2(v) * (v.shape[-1] != TINY.Fs))
+    elif mistake == "shared_relu_not_squared":    # the shared MLP's square dropped
+        monkeypatch.setattr(O, "relu2", lambda v: relu2(v) if v.shape[-1] != TINY.Fs else
+                            np.maximum(v, 0.0))
+    else:
+        raise ValueError(mistake)
+
+
+@pytest.mark.parametrize("mistake,caught_by", [
+    ("relu_not_squared", "k1"), ("no_scaling_factor", "k1"),
+    ("unnormalised_weights", "k_equals_E"), ("weights_from_biased_score", "k_equals_E"),
+    ("weights_in_wrong_slots", "k_equals_E"), ("bias_ignored_in_selection", "k1"),
+    ("gate_rows_misindexed", "routing"), ("shared_expert_dropped", "shared_only"),
+    ("shared_relu_not_squared", "shared_only")])
+def test_planted_mistakes_break_a_layer_pin(monkeypatch, mistake, caught_by):
+    _plant(monkeypatch, mistake)
+    assert not _holds(_LAYER_PINS[caught_by])
