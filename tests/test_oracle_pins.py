@@ -445,6 +445,21 @@ def test_rmsnorm_closed_forms_and_invariants():
     assert np.all(np.abs(O.rmsnorm_spec(x, g, 1e-2)) < np.abs(O.rmsnorm_spec(x, g, 0.0)))
 
 
+def test_rmsnorm_eps_inside_the_root():
+    """eps sits under the square root: with mean(x^2) + eps a perfect square
+    every step is exact, so x = 0.75 (eps 0.4375: root 1) and x = 1.5 (eps
+    1.75: root 2) give y = 0.75 g exactly; eps added after the root would give
+    0.75 / 1.1875 and 1.5 / 3.25."""
+    D = 512
+    g = (1.0 + 0.1 * np.random.RandomState(6).standard_normal(D)).astype(np.float32)
+    for c, eps in ((0.75, 0.4375), (1.5, 1.75)):
+        y = O.rmsnorm_spec(np.full((2, D), c), g, eps)
+        assert np.array_equal(y, np.tile(0.75 * g.astype(np.float64), (2, 1)))
+    half = np.zeros((1, D))
+    half[0, ::2] = 1.0                              # mean square 0.5, eps 0.5: root 1
+    assert np.array_equal(O.rmsnorm_spec(half, g, 0.5), half * g.astype(np.float64))
+
+
 def test_bf16_rounding_from_fp64_against_brute_force():
     """round_fp64_to_bf16 equals the nearest point of an enumerated bf16 grid
     (ties to the even significand), including exact midpoints."""
