@@ -36,7 +36,12 @@
  *
  * Streams.  `stream` arguments are cudaStream_t values passed as void*
  * (NULL = the legacy default stream).  A handle is used on one stream at a
- * time; calls on it are asynchronous unless stated otherwise.
+ * time; calls on it are asynchronous unless stated otherwise.  A bf16 layer's
+ * forward runs its input projections (fc1, shared up) on a non-blocking
+ * stream that the handle owns: forked from `stream` by an event at the start
+ * and joined back into `stream` by an event before the experts, so all of the
+ * call's work is ordered after earlier work on `stream` and before later work
+ * on it, and a graph captured from `stream` holds both branches.
  */
 #ifndef LATENTMOE_H
 #define LATENTMOE_H
