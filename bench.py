@@ -18,6 +18,7 @@ Prints one JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import atexit
 import json
 import os
 import statistics
@@ -72,6 +73,7 @@ class Clocks:
         self.proc = None
 
     def __enter__(self):
+        atexit.register(self.__exit__)       # no sampler outlives the process
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
@@ -88,7 +90,7 @@ class Clocks:
             self.rows.append([c.strip() for c in line.split(",")])
 
     def __exit__(self, *a):
-        if self.proc:
+        if self.proc and self.proc.poll() is None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -490,8 +492,10 @@ def _measure(a, cfg, W, rank, world, local, cpu_leg):
 
 
 # the other workloads of the headline metric, timed after the headline one on
-# the same weights (Ultra shape, bf16 dense weights; NVFP4 layers quantise them)
-EXTRA_WORKLOADS = ["ultra_prefill_bf16", "ultra_decode_w4a16", "skewed_prefill_w4a4"]
+# the same weights (Ultra shape, bf16 dense weights; NVFP4 layers quantise them),
+# and the decode batch under the other reading of its router-bias spread
+EXTRA_WORKLOADS = ["ultra_prefill_bf16", "ultra_decode_w4a16", "skewed_prefill_w4a4",
+                   "ultra_decode_bf16_bias_sd001"]
 
 
 def run_ours(a):
@@ -517,7 +521,10 @@ def run_ours(a):
         if c.bias_kind != cfg.bias_kind:
             Wc["gate_bias"] = I.gate_bias(c, "cuda")
         torch.cuda.empty_cache()
-        extras[name] = _measure(a, c, Wc, rank, world, local, cpu_leg=False)
+        try:
+            extras[name] = _measure(a, c, Wc, rank, world, local, cpu_leg=False)
+        except Exception as ex:          # one workload's failure keeps the others' lines
+            extras[name] = {"error": f"{type(ex).__name__}: {ex}"[:300]}
     if rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
                 "steps": a.steps, "warmup": max(a.warmup, 3),

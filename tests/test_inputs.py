@@ -95,6 +95,15 @@ def test_zipf_bias_profile():
     assert abs(p[0].item() / p[1].item() - 2 ** 1.1) < 1e-4
 
 
+def test_bias_spread_readings():
+    """N(0, 0.01) read as a variance (std 0.1, the decode workload) and as a
+    standard deviation (0.01, its companion): the same draws, scaled."""
+    b1 = I.gate_bias(I.CONFIGS["ultra_decode_bf16"]).double()
+    b2 = I.gate_bias(I.CONFIGS["ultra_decode_bf16_bias_sd001"]).double()
+    assert 0.085 < b1.std().item() < 0.115 and 0.0085 < b2.std().item() < 0.0115
+    assert torch.allclose(b2, 0.1 * b1, rtol=0, atol=1e-8)
+
+
 @pytest.mark.gpu
 def test_generator_bit_identical_on_gpu():
     """The CPU oracle and the GPU path read the same tensors when each
