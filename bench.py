@@ -524,6 +524,8 @@ def run_ours(a):
         try:
             extras[name] = _measure(a, c, Wc, rank, world, local, cpu_leg=False)
         except Exception as ex:          # one workload's failure keeps the others' lines
+            if world > 1:                # ranks must not part ways between collectives
+                raise
             extras[name] = {"error": f"{type(ex).__name__}: {ex}"[:300]}
     if rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
