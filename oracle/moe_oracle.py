@@ -172,7 +172,7 @@ def route(logits: np.ndarray, bias: np.ndarray, k: int, rsf: float,
 
 
 # ---------------------------------------------------------------------------
-# Token -> expert bookkeeping (section 5.6 step 6: one_hot / expert_hit),
+# Token -> expert bookkeeping (section 5.6 step 6: the expert mask and hit list),
 # written as its plain definition: a stable grouping of the (token, slot) pairs.
 # ---------------------------------------------------------------------------
 
