@@ -5,6 +5,8 @@ grouping checked by its defining properties at full size, 16+ output rows
 against the oracle (first and last token tiles, the ragged last tile of the
 most loaded expert, outlier rows), and the tensor-core router logits against
 the error bound the certified selection relies on."""
+import warnings
+
 import numpy as np
 import pytest
 import torch
@@ -118,5 +120,6 @@ def test_tensor_core_logits_within_the_certified_bound(ultra):
         ratios[cfg.name] = _logit_error_ratio(lay.router_logits(cfg.T)[rows], x[rows], W,
                                               cfg.D // _splits(cfg.T))
         lay.close()
-    print("tensor-core logit error / bound:", ratios)
+    # reported in the run's warnings summary, which pytest prints even with -q
+    warnings.warn(f"tensor-core logit error / bound without the margin: {ratios}")
     assert all(v <= 1.0 for v in ratios.values()), ratios
